@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the paged KV cache path on one B200 (or N replicas).
+
+Workload (default): the 8B-GQA shared-prefix batch -- 256 sequences, 32 query
+heads over 8 kv heads, head_dim 128, bf16, 16-token blocks; every sequence
+shares 4 physical prefix blocks (64 tokens) and has total context uniform in
+[65, 8192].  The native host allocator lays the batch out (shared prefix,
+on-demand blocks from a shuffled free list) and hands out this step's slots.
+
+One timed step = the whole device path of a decode step:
+  block_copy (copy-on-write pairs, if any) -> paged_kv_write -> paged_attention_decode
+on inputs already resident in HBM.  The K/V stream (4.3 GB) is far larger
+than L2 (126 MB), so no L2 flush is needed between steps.
+
+value  = effective KV GB/s = sum_s ctx_s * Hkv * D * 2 (K and V) * elem / step time
+e2e    = the same metric with, per step, pinned host -> device copies of the
+         step's inputs and a device -> host copy of the output in the timed region
+roofline = decode kernel(s) only: algorithmic bytes (K/V + Q + out + tables)
+           per launch / mean launch time (CUDA events on the launching stream)
+
+`--impl reference` times the plain CPU oracle on a bounded sample of the same
+workload on the host cores (the slow baseline), and prints the same line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "paged decode attention: effective KV GB/s (% of HBM peak), seq-steps/s"
+WORKLOAD_NAMES = {2: "7b", 3: "13b", 4: "8b_gqa_prefix", 5: "8b_gqa_sampling"}
+FALLBACK_HBM_GBS = 6650.0
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# workload state
+# ----------------------------------------------------------------------------
+class Step:
+    """Everything one decode step needs, resident on the GPU."""
+
+
+def build_step(number: int, device, rank: int = 0):
+    import paged_kv_cache_398_b200 as pkv
+    from paged_kv_cache_398_b200.workloads import make_workload
+
+    seed = rank_seed(number, rank)
+    w = make_workload(number, device=device, seed=seed)   # lengths on host, values on the GPU
+    S = w.num_seqs
+    st = Step()
+    st.w = w
+    st.host_alloc_us = None
+    if number == 5:
+        # parallel sampling: the generator's tables already hold the shared
+        # prompt blocks; the step's copy-on-write pairs come with them
+        tables, lens, pairs = w.block_tables, w.context_lens, w.copy_pairs
+        slots = pkv.pkv_slot_mapping(tables, lens - 1)
+    else:
+        perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(seed + 7))
+        alloc = pkv.BlockAllocator(w.num_blocks, w.block_size, initial_order=perm)
+        prefix_tokens = 64 if number == 4 else 0
+        prefix = []
+        if prefix_tokens:
+            alloc.add(-1)
+            alloc.append_tokens(-1, prefix_tokens)
+            prefix = alloc.block_table(-1)
+        for s in range(S):
+            alloc.add(s)
+            if prefix:
+                alloc.share_prefix(s, prefix, prefix_tokens)
+            alloc.append_tokens(s, int(w.context_lens[s]) - 1 - prefix_tokens)
+        seqs = list(range(S))
+        t0 = time.perf_counter()
+        slots, pairs = alloc.append_one_batch(seqs)          # this step's slots (+ CoW pairs)
+        tables, lens = alloc.batch_tables(seqs, w.max_blocks_per_seq)
+        st.host_alloc_us = (time.perf_counter() - t0) * 1e6
+        assert torch.equal(lens, w.context_lens)
+        st.alloc = alloc
+    st.tables_host, st.lens_host, st.slots_host, st.pairs = tables, lens, slots, pairs
+    st.block_tables = tables.to(device)
+    st.context_lens = lens.to(device)
+    st.slots = slots.to(device)
+    st.q, st.k_cache, st.v_cache = w.q, w.k_cache, w.v_cache
+    st.k_new, st.v_new = w.k_new, w.v_new
+    st.out = torch.empty_like(w.q)
+    st.max_ctx = int(lens.max())
+    ws_bytes = pkv.paged_attention_workspace_bytes(S, w.num_q_heads, w.head_dim, st.max_ctx)
+    st.workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    e = w.q.element_size()
+    ctx = lens.to(torch.int64)
+    nblk = (ctx + w.block_size - 1) // w.block_size
+    st.kv_bytes = int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * e
+    uniq_blocks = len(set(tables[tables >= 0].tolist())) if number in (4, 5) else int(nblk.sum())
+    st.kv_unique_bytes = uniq_blocks * w.num_kv_heads * w.block_size * w.head_dim * 2 * e  # upper bound
+    st.decode_bytes = (st.kv_bytes + 2 * S * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S)
+    st.write_bytes = 2 * 2 * S * w.num_kv_heads * w.head_dim * e + 8 * S
+    st.copy_bytes = 2 * 2 * pairs.shape[0] * w.num_kv_heads * w.block_size * w.head_dim * e
+    st.max_parts = (st.max_ctx + pkv.PARTITION_TOKENS - 1) // pkv.PARTITION_TOKENS
+    st.launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
+    return st
+
+
+def run_step(st, ev=None):
+    import paged_kv_cache_398_b200 as pkv
+    if st.pairs.shape[0]:
+        pkv.block_copy(st.k_cache, st.v_cache, st.pairs)
+    pkv.paged_kv_write(st.k_new, st.v_new, st.k_cache, st.v_cache, st.slots)
+    if ev is not None:
+        ev[0].record()
+    pkv.paged_attention_decode(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                               st.w.scale, st.max_ctx, workspace=st.workspace)
+    if ev is not None:
+        ev[1].record()
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        p = torch.cuda.get_device_properties(device_index)
+        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0".upper()
+        self.samples = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if not parts[0].upper().endswith(self.bus[-7:]):   # "BB:DD.F" of this GPU
+                continue
+            self.samples.append((time.monotonic(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        win = [p for t, p in self.samples if t0 <= t <= t1]
+        where = "timed region"
+        if not win:
+            win = [p for _, p in self.samples]
+            where = "whole run (no sample fell inside the timed region)"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in win if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in win for n, v in zip(names, p[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(win[0][2]), "power_w_max": max((num(p[3]) or 0) for p in win),
+                "reasons": reasons, "samples": len(win), "window": where}
+
+
+# ----------------------------------------------------------------------------
+# the oracle on the host cores
+# ----------------------------------------------------------------------------
+def sub_workload(w, tables, lens, pairs, seqs):
+    """The listed sequences' blocks (plus copy sources) copied to the host and
+    relabelled 0..n-1, with their tables, as an oracle input."""
+    from paged_kv_cache_398_b200.workloads import DecodeWorkload
+    B = w.block_size
+    need = []
+    for s in seqs:
+        need += tables[s, :-(-int(lens[s]) // B)].tolist()
+    dsts = set(need)
+    sub_pairs = [(int(a), int(b)) for a, b in pairs.tolist() if int(b) in dsts]
+    need += [a for a, _ in sub_pairs]
+    ids = sorted(set(need))
+    remap = {b: i for i, b in enumerate(ids)}
+    idx = torch.tensor(ids, dtype=torch.int64, device=w.k_cache.device)
+    sbt = torch.full((len(seqs), tables.shape[1]), -1, dtype=torch.int32)
+    for r, s in enumerate(seqs):
+        n = -(-int(lens[s]) // B)
+        sbt[r, :n] = torch.tensor([remap[b] for b in tables[s, :n].tolist()], dtype=torch.int32)
+    sel = torch.tensor(seqs, dtype=torch.int64, device=w.q.device)
+    return DecodeWorkload(
+        name=w.name + "-sample", dtype=w.dtype, num_seqs=len(seqs), num_q_heads=w.num_q_heads,
+        num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=B, num_blocks=len(ids),
+        context_lens=lens[seqs].contiguous(), block_tables=sbt,
+        copy_pairs=torch.tensor([(remap[a], remap[b]) for a, b in sub_pairs], dtype=torch.int64).reshape(-1, 2),
+        q=w.q[sel].cpu(), k_cache=w.k_cache[idx].cpu(), v_cache=w.v_cache[idx].cpu(),
+        k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(), scale=w.scale, seed=w.seed)
+
+
+def oracle_step_timed(sub, threads: int) -> float:
+    """Run the oracle's copy + write + decode on `sub`; returns wall seconds."""
+    import concurrent.futures as cf
+
+    import oracle
+    from oracle.allocator_model import slot_for_position
+    B = sub.block_size
+    slots = torch.tensor([slot_for_position(sub.block_tables[s].tolist(), int(sub.context_lens[s]) - 1, B)
+                          for s in range(sub.num_seqs)], dtype=torch.int64)
+    k, v = sub.k_cache.clone(), sub.v_cache.clone()
+    t0 = time.perf_counter()
+    if sub.copy_pairs.numel():
+        oracle.block_copy(k, v, sub.copy_pairs)
+    oracle.kv_write(k, v, sub.k_new, sub.v_new, slots)
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda s: oracle.paged_decode_seq(s, sub.q, k, v, sub.block_tables, sub.context_lens,
+                                                      sub.scale), range(sub.num_seqs)))
+    return time.perf_counter() - t0
+
+
+def sample_kv_bytes(sub) -> int:
+    return int(sub.context_lens.to(torch.int64).sum()) * sub.num_kv_heads * sub.head_dim * 2 * sub.q.element_size()
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def pick_sample(lens, work_seconds_target: float, per_token_s: float):
+    """Leading sequences whose oracle work adds up to about the target."""
+    seqs, acc = [], 0.0
+    for s in range(len(lens)):
+        seqs.append(s)
+        acc += int(lens[s]) * per_token_s
+        if acc >= work_seconds_target:
+            break
+    return seqs
+
+
+def cpu_baseline(st, threads: int):
+    lens, tables, pairs = st.lens_host, st.tables_host, st.pairs
+    probe = sub_workload(st.w, tables, lens, pairs, [0])
+    t1 = oracle_step_timed(probe, 1)
+    per_tok = t1 / max(1, int(lens[0]))
+    seqs = pick_sample(lens, 15.0, per_tok)
+    sub = sub_workload(st.w, tables, lens, pairs, seqs)
+    t = oracle_step_timed(sub, threads)
+    return {"value": sample_kv_bytes(sub) / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": (f"{len(seqs)} of {len(lens)} sequences (all {sub.num_q_heads} query heads): "
+                       f"copy + slot write + decode by the fp64 C oracle, {t:.2f} s wall on {threads} threads"),
+            "seconds": t}
+
+
+# ----------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from paged_kv_cache_398_b200.workloads import make_workload
+    threads = cpu_threads()
+    # a bounded sample of the workload's recipe, built on the host only
+    n = args.reference_seqs
+    w = make_workload(args.workload, device="cpu", **({"num_prompts": max(1, n // 4)} if args.workload == 5
+                                                       else {"num_seqs": n}))
+    lens, tables, pairs = w.context_lens, w.block_tables, w.copy_pairs
+    sub = sub_workload(w, tables, lens, pairs, list(range(w.num_seqs)))
+    for _ in range(args.warmup):
+        oracle_step_timed(sub, threads)
+    times = [oracle_step_timed(sub, threads) for _ in range(args.steps)]
+    total = sum(times)
+    kvb = sample_kv_bytes(sub)
+    value = kvb * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": str(w.dtype).replace("torch.", ""), "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.workload], "sample_seqs": w.num_seqs,
+                   "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size},
+        "seq_steps_per_s": w.num_seqs * args.steps / total,
+        "cpu_baseline": {"kind": "oracle", "cores": threads, "value": value, "unit": "GB/s",
+                         "sample": f"{w.num_seqs} sequences of the workload recipe per step, fp64 C oracle "
+                                   f"(copy + slot write + decode) on {threads} host threads"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def reduce_over_ranks(dist, device, times_ms, amounts):
+    """Max over ranks of each time, sum over ranks of each amount (timing and
+    byte counts only; the decode path itself exchanges nothing)."""
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    a = torch.tensor(list(amounts), dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(a, op=dist.ReduceOp.SUM)
+    return t.tolist() + a.tolist()
+
+
+def rank_seed(number: int, rank: int) -> int:
+    """Each replica decodes its own batch of the same shape."""
+    return 398000 + number + 1000 * rank
+
+
+def run_ours(args):
+    import paged_kv_cache_398_b200 as pkv
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    st = build_step(args.workload, dev, rank)
+    torch.cuda.synchronize(dev)
+    threads = cpu_threads()
+    # the oracle sample is copied off the device before the first product step
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(st, threads)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for _ in range(args.warmup):
+        run_step(st)
+    barrier()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t_wall0 = time.monotonic()
+    start.record()
+    for i in range(args.steps):
+        run_step(st, evs[i])
+    end.record()
+    barrier()
+    t_wall1 = time.monotonic()
+    ms = start.elapsed_time(end)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+
+    # ---- end to end: host inputs in, host output out, every step ------------
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_in = {"q": pin(st.q), "k_new": pin(st.k_new), "v_new": pin(st.v_new), "slots": pin(st.slots),
+            "tables": pin(st.block_tables), "lens": pin(st.context_lens)}
+    d_in = {"q": st.q, "k_new": st.k_new, "v_new": st.v_new, "slots": st.slots, "tables": st.block_tables,
+            "lens": st.context_lens}
+    h_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for k2, t in h_in.items():
+            d_in[k2].copy_(t, non_blocking=True)
+        run_step(st)
+        h_out.copy_(st.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    e2e_steps = args.steps
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    barrier()
+    t_wall2 = time.monotonic()
+    e2e_ms = e0.elapsed_time(e1)
+    clocks.stop()
+
+    ms_max, e2e_max, kv_total, uniq_total = reduce_over_ranks(
+        dist, dev, [ms, e2e_ms], [float(st.kv_bytes), float(st.kv_unique_bytes)])
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = hbm_peak()
+    S = st.w.num_seqs
+    value = kv_total * args.steps / (ms_max / 1e3) / 1e9
+    dec_mean = statistics.mean(dec_ms)
+    achieved = st.decode_bytes / (dec_mean / 1e3) / 1e9
+    clk = clocks.summary(t_wall0, t_wall1)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": str(st.w.dtype).replace("torch.", ""),
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAMES[args.workload], "num_seqs": S,
+                   "num_q_heads": st.w.num_q_heads, "num_kv_heads": st.w.num_kv_heads,
+                   "head_dim": st.w.head_dim, "block_size": st.w.block_size,
+                   "context_tokens": int(st.lens_host.sum()), "max_context_len": st.max_ctx,
+                   "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB of K/V per step), no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": 100.0 * value / peak,
+        "seq_steps_per_s": S * world * args.steps / (ms_max / 1e3),
+        "unique_kv_gbps": uniq_total * args.steps / (ms_max / 1e3) / 1e9,
+        "kernel_ms": {"decode_mean": dec_mean, "decode_min": min(dec_ms),
+                      "write_and_copy_mean": ms_max / args.steps - dec_mean},
+        "roofline": {"kernel": "paged_attention_decode (partition kernel + split-K reduce)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": st.decode_bytes},
+        "cpu_baseline": ({k: v for k, v in base.items() if k != "seconds"} if base else None),
+        "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_steps},
+        "gpu_launches": st.launches_per_step * args.steps,
+        "host_alloc_us_per_step": st.host_alloc_us,
+        "clocks": clk,
+        "wall_s_timed": t_wall1 - t_wall0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seqs", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

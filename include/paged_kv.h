@@ -1,0 +1,297 @@
+/*
+ * paged_kv.h -- C ABI of the paged KV cache decode path for NVIDIA B200
+ * (sm_100a).
+ *
+ * The KV cache of every sequence is stored in fixed-size physical blocks of
+ * 16 tokens.  A per-sequence block table maps logical block j (tokens
+ * 16j .. 16j+15) to a physical block anywhere in one shared pool.  Blocks are
+ * handed out when a sequence needs them and returned when it finishes.
+ * Sequences that share a prompt share its physical blocks, and a shared
+ * block is copied before a sequence writes into it.
+ *   Sources: "PagedAttention: How vLLM Serves AI Like an Operating System",
+ *   sections "How It Works", "PagedAttention Memory Layout", "The Magic: No
+ *   Pre-allocation" and "Copy-on-Write: Sharing KV Cache"; "vLLM
+ *   Architecture and PagedAttention", "Page Table Visualization".
+ *
+ * Conventions shared by every call:
+ *  - Memory.  The caller owns all memory.  Device buffers are raw device
+ *    pointers, for example from torch.  No device call here allocates device
+ *    memory; paged_attention_decode takes a caller-supplied workspace whose
+ *    size paged_attention_workspace_bytes reports.  Pointers marked HOST are
+ *    host memory, read before the call returns.
+ *  - Streams.  `stream` is a cudaStream_t passed as void*; NULL means the
+ *    legacy default stream.  Device calls only enqueue work and return
+ *    without synchronising.
+ *  - Cache layout.  k_cache and v_cache are each
+ *    [num_blocks][num_kv_heads][block_size][head_dim], row-major, in the
+ *    element type `dtype`.  Every (block, kv head) tile is therefore one
+ *    contiguous block_size * head_dim run.
+ *  - Slots.  Token position t of a sequence lives in physical block
+ *    table[t / block_size], at offset t % block_size.  Its slot number is
+ *    physical_block * block_size + offset.
+ *  - Errors.  Every call returns a status code: PKV_OK or a negative
+ *    PKV_ERR_*.  No exception crosses the ABI.  Arguments that the host can
+ *    check are checked before anything is enqueued.  Values that only the
+ *    device sees (block ids in tables, slots, context lengths) are checked by
+ *    the kernels.  A kernel never reads or writes outside the buffers
+ *    described here: it skips the bad item and sets a flag in a sticky
+ *    per-device status word, which pkv_device_status reads.
+ *  - Supported decode shapes: block_size 16, head_dim 64 or 128,
+ *    num_q_heads / num_kv_heads in {1, 2, 4, 8}.  Element type fp32, fp16
+ *    or bf16, with fp32 accumulation.  Other shapes return
+ *    PKV_ERR_UNSUPPORTED.
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define PKV_OK 0
+#define PKV_ERR_INVALID_ARG (-1)   /* bad pointer, size, shape or id         */
+#define PKV_ERR_UNSUPPORTED (-2)   /* valid but not built (dtype/shape)      */
+#define PKV_ERR_CUDA (-3)          /* a CUDA call failed: pkv_last_cuda_error */
+#define PKV_ERR_OUT_OF_BLOCKS (-4) /* the free list cannot cover the request */
+#define PKV_ERR_BAD_BLOCK (-5)     /* block id outside the pool / not held   */
+#define PKV_ERR_DEVICE (-6)        /* a device-side check failed (flags set) */
+
+/* ---- element types ----------------------------------------------------- */
+#define PKV_F32 0
+#define PKV_F16 1
+#define PKV_BF16 2
+
+/* ---- device status flags (pkv_device_status) --------------------------- */
+#define PKV_DEV_BAD_BLOCK_ID 1   /* a block table entry outside [0, num_blocks) */
+#define PKV_DEV_BAD_SLOT 2       /* a slot >= num_blocks * block_size           */
+#define PKV_DEV_BAD_CONTEXT 4    /* context_len < 1, beyond the table row, or
+                                    above the max_context_len of the launch   */
+#define PKV_DEV_WAIT_TIMEOUT 8   /* an on-chip copy wait gave up (bounded spin) */
+
+/*
+ * paged_kv_write -- store the new tokens' key and value rows in their slots.
+ * (The cache is filled block by block as tokens arrive: "How It Works",
+ *  "The Magic: No Pre-allocation".)
+ *
+ *  k_new, v_new   device, [num_tokens][num_kv_heads][head_dim], dtype
+ *  k_cache,
+ *  v_cache        device, cache layout above; rows of written slots change
+ *  slot_mapping   device, int64 [num_tokens]; slot of each token.  A negative
+ *                 slot skips that token (padding).  A slot at or beyond
+ *                 num_blocks * block_size is skipped and raises
+ *                 PKV_DEV_BAD_SLOT.  Slots must be distinct; if two tokens
+ *                 name one slot, which row lands there is unspecified.
+ *  head_dim * element size must be a multiple of 16 bytes, and all four
+ *  data pointers must be 16-byte aligned.
+ * The copy is bit-exact.  num_tokens == 0 is a no-op.
+ */
+int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                   const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+                   int32_t head_dim, int32_t block_size, int32_t num_blocks, int32_t dtype,
+                   void* stream);
+
+/*
+ * paged_attention_workspace_bytes -- size of the workspace that
+ * paged_attention_decode needs for this batch shape.  The value is 0 when
+ * max_context_len fits in one partition (PKV_PARTITION_TOKENS tokens).
+ * Otherwise the workspace holds, per (sequence, query head, partition), an
+ * fp32 running max, an fp32 sum and head_dim fp32 partial outputs.
+ */
+#define PKV_PARTITION_TOKENS 512
+size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                       int32_t max_context_len);
+
+/*
+ * paged_attention_decode -- one decode step of attention over the paged
+ * cache.  The result equals ordinary softmax attention over the sequence's
+ * tokens laid out contiguously: the paging changes where the tokens are
+ * stored, not what is computed ("Throughput Impact: The Numbers": no
+ * approximations).
+ *
+ *   out[s][i][:] = sum_t softmax_t(scale * q[s][i] . K_s[t]) * V_s[t]
+ *
+ * Here t runs over the first context_lens[s] token positions of sequence s,
+ * K_s[t] / V_s[t] are read for kv head i / (num_q_heads / num_kv_heads)
+ * through block_tables[s], and each query head group reads each K/V block
+ * once.
+ *
+ *  out            device, [num_seqs][num_q_heads][head_dim], dtype
+ *  q              device, [num_seqs][num_q_heads][head_dim], dtype
+ *  k_cache,
+ *  v_cache        device, cache layout above (read only)
+ *  block_tables   device, int32 [num_seqs][max_blocks_per_seq]; only the
+ *                 first ceil(context_lens[s] / block_size) entries of row s
+ *                 are read, the rest may hold anything.  An entry outside
+ *                 [0, num_blocks) raises PKV_DEV_BAD_BLOCK_ID and block 0 is
+ *                 read in its place.
+ *  context_lens   device, int32 [num_seqs]: tokens to attend to, counting
+ *                 the step's new token, which the caller must already have
+ *                 written with paged_kv_write.  A value < 1, above
+ *                 max_blocks_per_seq * block_size or above max_context_len
+ *                 raises PKV_DEV_BAD_CONTEXT.  For < 1 the output row is
+ *                 zero; for the other two the length is clamped.
+ *  max_context_len  host int, >= every context_lens[s]; it sizes the grid,
+ *                 so the host never reads device data.
+ *  scale          softmax scale, usually 1/sqrt(head_dim)
+ *  workspace      device, >= paged_attention_workspace_bytes(...) bytes,
+ *                 256-byte aligned; may be NULL when that size is 0.  It is
+ *                 scratch for the call and is overwritten.
+ * Accumulation is fp32.  The result is rounded once to dtype.  It depends
+ * only on the values, never on where the blocks sit in the pool: permuting
+ * the physical placement gives bit-identical output.
+ */
+int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t max_context_len,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * block_copy -- copy-on-write copies: for each pair (src, dst), physical
+ * block dst becomes a copy of block src, in the keys and the values of
+ * every kv head.  ("Copy-on-Write: Sharing KV Cache": a request that must
+ * modify a shared block copies it first.)
+ *
+ *  pairs          HOST, int64 [num_pairs][2] as (src, dst).  The whole list
+ *                 is checked before any copy is enqueued:
+ *                   - ids must lie in [0, num_blocks);
+ *                   - src != dst;
+ *                   - no dst may appear twice;
+ *                   - no dst may also be a src in the same call.
+ *                 A list that breaks any rule, whose result would depend on
+ *                 copy order, returns PKV_ERR_INVALID_ARG.
+ *  The copy is bit-exact.  num_pairs == 0 is a no-op.  Both cache pointers
+ *  must be 16-byte aligned.
+ */
+int block_copy(void* k_cache, void* v_cache, const int64_t* pairs, int32_t num_pairs,
+               int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+               int32_t dtype, void* stream);
+
+/*
+ * pkv_slot_mapping -- HOST helper: slots_out[s] = slot of token position
+ * positions[s] of sequence s, given its block-table row (host int32
+ * [num_seqs][max_blocks_per_seq]).  Returns PKV_ERR_INVALID_ARG for a
+ * position whose logical block lies beyond the row, and PKV_ERR_BAD_BLOCK
+ * for a negative table entry.  A negative position yields slot -1.
+ */
+int pkv_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* positions, int32_t num_seqs, int32_t block_size,
+                     int64_t* slots_out);
+
+/*
+ * pkv_device_status -- read, and if `clear` is nonzero reset, the sticky
+ * status word of `device`.  This synchronises that device.  *flags_out
+ * receives an OR of PKV_DEV_* flags, or 0.
+ */
+int pkv_device_status(int32_t device, int32_t* flags_out, int32_t clear);
+
+/* The last cudaError_t seen by any call in this thread, as an int. */
+int pkv_last_cuda_error(void);
+
+/* A static, human-readable name for a PKV_* status code. */
+const char* pkv_status_string(int status);
+
+/* ======================================================================== *
+ * Host block allocator: pool of physical blocks, free list, reference
+ * counts, per-sequence block tables, and copy-on-write decisions.
+ * ("How It Works"; "The Magic: No Pre-allocation"; "Copy-on-Write: Sharing
+ *  KV Cache", "Parallel Sampling" and "Prefix Caching"; "vLLM
+ *  Architecture": the KV cache manager that allocates and frees blocks.)
+ *
+ * Policy:
+ *  - The free list is a stack.  initial_order gives the order in which blocks
+ *    are first handed out (NULL = 0, 1, 2, ...).  A freed block goes on top.
+ *  - A sequence gets a new block exactly when its token count crosses a
+ *    multiple of block_size, so n tokens hold ceil(n / block_size) blocks.
+ *  - Freeing a sequence releases its blocks from the last logical block to
+ *    the first; a block returns to the free list when its count reaches 0.
+ *  - Before a sequence writes into a partially filled block that others
+ *    also hold (count > 1), it moves to a fresh private block and reports the
+ *    (src, dst) copy pair.  The last holder (count == 1) writes in place.
+ *  - A call that cannot get every block it needs returns
+ *    PKV_ERR_OUT_OF_BLOCKS and changes nothing.
+ * Sequence ids are arbitrary int64 values chosen by the caller.
+ * One allocator is not thread-safe; use one per thread or lock around it.
+ * ======================================================================== */
+typedef struct pkv_allocator pkv_allocator;
+
+typedef struct pkv_alloc_stats {
+    int32_t num_blocks;
+    int32_t free_blocks;
+    int32_t used_blocks;          /* num_blocks - free_blocks                 */
+    int32_t shared_blocks;        /* blocks with reference count > 1          */
+    int64_t num_seqs;
+    int64_t num_tokens;           /* sum of the sequences' token counts       */
+    int64_t fragmentation_tokens; /* sum over sequences of unused slots in
+                                     their blocks (at most block_size - 1 each) */
+} pkv_alloc_stats;
+
+/* num_blocks >= 0, block_size >= 1; initial_order: HOST int32 [num_blocks]
+ * permutation of 0..num_blocks-1, or NULL.  *out receives the handle. */
+int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* initial_order,
+                     pkv_allocator** out);
+void pkv_alloc_destroy(pkv_allocator* a);
+
+/* Register an empty sequence.  An id already in use -> PKV_ERR_INVALID_ARG. */
+int pkv_seq_add(pkv_allocator* a, int64_t seq);
+
+/* Reserve slots for n >= 0 new tokens of `seq`.  slots_out (HOST int64 [n],
+ * may be NULL) receives their slots in order.  If the first write lands in
+ * a shared partial block, the sequence moves to a fresh block first:
+ * *cow_out = 1 and cow_pair_out (HOST int64 [2], may be NULL) = (src, dst).
+ * Otherwise *cow_out = 0.  cow_out may be NULL. */
+int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slots_out,
+                          int64_t* cow_pair_out, int32_t* cow_out);
+
+/* One new token for each of n_seqs distinct sequences, in order (one
+ * decode step).  slots_out: HOST int64 [n_seqs].  cow_pairs_out: HOST int64
+ * [n_seqs][2], may be NULL.  The first *n_cow_out rows receive the copy
+ * pairs.  All-or-nothing: if the free list cannot cover every sequence,
+ * nothing changes. */
+int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
+                         int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out);
+
+/* Release a finished sequence ("its pages are immediately freed"). */
+int pkv_seq_free(pkv_allocator* a, int64_t seq);
+
+/* New sequence `child` sharing every block of `parent` (parallel sampling). */
+int pkv_seq_fork(pkv_allocator* a, int64_t parent, int64_t child);
+
+/* Point an empty sequence at existing allocated blocks (a shared system
+ * prompt).  blocks: HOST int32 [n_blocks], each with count >= 1.  n_tokens
+ * must satisfy ceil(n_tokens / block_size) == n_blocks. */
+int pkv_seq_share_prefix(pkv_allocator* a, int64_t seq, const int32_t* blocks, int32_t n_blocks,
+                         int32_t n_tokens);
+
+/* Copy the block table of `seq` into out (HOST int32 [cap]).  *n_out receives
+ * its length.  If the table is longer than cap, the call returns
+ * PKV_ERR_INVALID_ARG and writes nothing. */
+int pkv_seq_block_table(const pkv_allocator* a, int64_t seq, int32_t* out, int32_t cap,
+                        int32_t* n_out);
+int pkv_seq_num_tokens(const pkv_allocator* a, int64_t seq, int32_t* out);
+
+/* Block tables and context lengths of n_seqs sequences, ready for
+ * paged_attention_decode.  tables_out: HOST int32
+ * [n_seqs][max_blocks_per_seq]; entries past a table's end are set to pad.
+ * context_lens_out: HOST int32 [n_seqs], may be NULL. */
+int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
+                     int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
+                     int32_t* context_lens_out);
+
+int32_t pkv_num_free(const pkv_allocator* a);
+/* The free blocks in the order they will be handed out (HOST int32 [cap]). */
+int pkv_free_list(const pkv_allocator* a, int32_t* out, int32_t cap, int32_t* n_out);
+/* Reference count of a block (0 = free); -1 for an id outside the pool. */
+int32_t pkv_refcount(const pkv_allocator* a, int32_t block);
+int pkv_alloc_get_stats(const pkv_allocator* a, pkv_alloc_stats* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

@@ -37,6 +37,12 @@ Policy choices the pages leave open (the product follows the same ones):
 from __future__ import annotations
 
 
+def slot_for_position(block_table, position: int, block_size: int) -> int:
+    """Slot of token `position` of a sequence with this block table: its
+    physical block times the block size plus its offset in the block."""
+    return int(block_table[position // block_size]) * block_size + position % block_size
+
+
 class OutOfBlocks(Exception):
     pass
 
@@ -122,7 +128,7 @@ class AllocatorModel:
         for p in range(ntok, ntok + n):
             if p % B == 0:
                 blocks.append(self._pop())
-            slots.append(blocks[p // B] * B + p % B)
+            slots.append(slot_for_position(blocks, p, B))
         seq["ntok"] = ntok + n
         return slots, cow
 

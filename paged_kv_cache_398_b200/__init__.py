@@ -1,0 +1,27 @@
+"""Paged KV cache decode path for NVIDIA B200 (sm_100a).
+
+The KV cache lives in fixed-size, non-contiguous 16-token physical blocks
+reached through per-sequence block tables ("PagedAttention: How vLLM Serves
+AI Like an Operating System").  The package is a thin Python binding over the
+C ABI of ``include/paged_kv.h``:
+
+* ``paged_kv_write``          -- slot write of the new tokens' K/V
+* ``paged_attention_decode``  -- decode attention through the block tables
+* ``block_copy``              -- copy-on-write block copy
+* ``BlockAllocator``          -- host block allocator (free list, refcounts, CoW)
+
+The native library ``libpaged_kv.so`` is built in-tree by
+``paged_kv_cache_398_b200.build``.  There is no CPU fallback.
+"""
+
+from ._lib import LibraryMissing, PagedKVError
+from .allocator import BlockAllocator, OutOfBlocks
+from .binding import (BLOCK_SIZE, PARTITION_TOKENS, block_copy, paged_attention_decode,
+                      paged_attention_workspace_bytes, paged_kv_write, pkv_device_status,
+                      pkv_slot_mapping)
+
+__all__ = [
+    "BLOCK_SIZE", "PARTITION_TOKENS", "BlockAllocator", "LibraryMissing", "OutOfBlocks",
+    "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_workspace_bytes",
+    "paged_kv_write", "pkv_device_status", "pkv_slot_mapping",
+]

@@ -1,0 +1,141 @@
+"""Python binding of the C ABI in include/paged_kv.h (argument marshalling only).
+
+Each function has the name of the C entry point it calls.  It reads sizes
+from tensor shapes, checks that the tensors are contiguous, on the GPU and
+of one element type, and passes raw pointers and torch's current CUDA stream.
+Every step of the computation runs in the library's CUDA kernels.  Failures
+raise ``PagedKVError``, carrying the library's status code.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from ._lib import C, PagedKVError, check, lib
+
+_DTYPE = {torch.float32: C["PKV_F32"], torch.float16: C["PKV_F16"], torch.bfloat16: C["PKV_BF16"]}
+BLOCK_SIZE = 16
+PARTITION_TOKENS = C["PKV_PARTITION_TOKENS"]
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPE[t.dtype]
+    except KeyError:
+        raise PagedKVError("dtype", C["PKV_ERR_UNSUPPORTED"]) from None
+
+
+def _cuda(name: str, t: torch.Tensor, dtype=None, ndim=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    return t
+
+
+def _stream(device: torch.device, stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cache_shape(k_cache, v_cache):
+    _cuda("k_cache", k_cache, ndim=4)
+    _cuda("v_cache", v_cache, k_cache.dtype, 4)
+    if k_cache.shape != v_cache.shape or k_cache.device != v_cache.device:
+        raise ValueError("k_cache and v_cache must have one shape and device")
+    NB, Hkv, B, D = k_cache.shape
+    return NB, Hkv, B, D
+
+
+def paged_kv_write(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """Store k_new/v_new [T, Hkv, D] in the slots slot_mapping [T] (int64)."""
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    _cuda("k_new", k_new, k_cache.dtype, 3)
+    _cuda("v_new", v_new, k_cache.dtype, 3)
+    _cuda("slot_mapping", slot_mapping, torch.int64, 1)
+    T = slot_mapping.shape[0]
+    if tuple(k_new.shape) != (T, Hkv, D) or tuple(v_new.shape) != (T, Hkv, D):
+        raise ValueError("k_new/v_new must be [T, Hkv, D] matching slot_mapping and the cache")
+    rc = lib().paged_kv_write(k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                              slot_mapping.data_ptr(), T, Hkv, D, B, NB, _dtype_code(k_cache),
+                              _stream(k_cache.device, stream))
+    check("paged_kv_write", rc)
+
+
+def paged_attention_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                                    max_context_len: int) -> int:
+    return int(lib().paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                           max_context_len: int, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """Decode attention through the block tables; writes and returns `out` [S, Hq, D].
+
+    context_lens counts the step's new token (write it first with
+    paged_kv_write).  max_context_len (a host int >= every length) sizes the
+    grid.  workspace: a CUDA tensor of at least
+    paged_attention_workspace_bytes(...) bytes, or None to let torch
+    allocate one for this call.
+    """
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    _cuda("q", q, k_cache.dtype, 3)
+    _cuda("out", out, k_cache.dtype, 3)
+    _cuda("block_tables", block_tables, torch.int32, 2)
+    _cuda("context_lens", context_lens, torch.int32, 1)
+    S, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (S, Hq, D):
+        raise ValueError("q/out must be [S, Hq, D] with the cache's head_dim")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables/context_lens must have one row per sequence")
+    need = paged_attention_workspace_bytes(S, Hq, D, max_context_len)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _cuda("workspace", workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    rc = lib().paged_attention_decode(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      block_tables.data_ptr(), block_tables.shape[1],
+                                      context_lens.data_ptr(), S, int(max_context_len), Hq, Hkv, D, B, NB,
+                                      float(scale), _dtype_code(k_cache), ws_ptr or None, ws_bytes,
+                                      _stream(q.device, stream))
+    check("paged_attention_decode", rc)
+    return out
+
+
+def block_copy(k_cache, v_cache, pairs, stream=None) -> None:
+    """Copy-on-write copies; pairs: host int64 [N, 2] (src, dst) tensor or list."""
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    pr = torch.as_tensor(pairs, dtype=torch.int64, device="cpu").reshape(-1, 2).contiguous()
+    rc = lib().block_copy(k_cache.data_ptr(), v_cache.data_ptr(), pr.data_ptr(), pr.shape[0], Hkv, D, B,
+                          NB, _dtype_code(k_cache), _stream(k_cache.device, stream))
+    check("block_copy", rc)
+
+
+def pkv_slot_mapping(block_tables: torch.Tensor, positions: torch.Tensor, block_size: int = BLOCK_SIZE):
+    """Host helper: slot of positions[s] in sequence s given host tables [S, MB]."""
+    bt = torch.as_tensor(block_tables, dtype=torch.int32).contiguous()
+    pos = torch.as_tensor(positions, dtype=torch.int32).contiguous()
+    if bt.device.type != "cpu" or pos.device.type != "cpu":
+        raise ValueError("pkv_slot_mapping takes host tensors")
+    out = torch.empty(pos.shape[0], dtype=torch.int64)
+    rc = lib().pkv_slot_mapping(bt.data_ptr(), bt.shape[1], pos.data_ptr(), pos.shape[0], block_size,
+                                out.data_ptr())
+    check("pkv_slot_mapping", rc)
+    return out
+
+
+def pkv_device_status(device: int = 0, clear: bool = True) -> int:
+    """Sticky device-side flags (PKV_DEV_*) of `device`; synchronises it."""
+    flags = ctypes.c_int32(0)
+    rc = lib().pkv_device_status(device, ctypes.byref(flags), 1 if clear else 0)
+    check("pkv_device_status", rc)
+    return int(flags.value)

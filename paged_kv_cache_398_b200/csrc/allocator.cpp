@@ -1,0 +1,330 @@
+// Host block allocator of the paged KV cache: a pool of fixed-size physical
+// blocks, a free list, per-block reference counts and per-sequence block
+// tables, with copy-on-write for shared partially filled blocks.
+//
+// Follows "PagedAttention: How vLLM Serves AI Like an Operating System":
+//   "How It Works"                 -- blocks, block tables, scattered blocks
+//   "The Magic: No Pre-allocation" -- one block at arrival, another at token
+//                                     17, 33, ...; at most 15 slots wasted
+//   "Copy-on-Write: Sharing KV Cache", "Parallel Sampling", "Prefix Caching"
+//                                  -- shared blocks, copy before modifying
+// and "vLLM Architecture and PagedAttention" ("Page Table Visualization":
+// a finished sequence's pages are freed immediately).
+//
+// The policy choices the pages leave open are stated in include/paged_kv.h.
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "paged_kv.h"
+
+namespace {
+
+struct Seq {
+    std::vector<int32_t> blocks;
+    int64_t ntok = 0;
+};
+
+}  // namespace
+
+struct pkv_allocator {
+    int32_t num_blocks = 0;
+    int32_t block_size = 16;
+    std::vector<int32_t> free_stack;  // back() is handed out next
+    std::vector<int32_t> ref;         // reference count per block
+    std::unordered_map<int64_t, Seq> seqs;
+    int32_t shared = 0;               // blocks with ref > 1
+
+    int32_t pop()
+    {
+        int32_t b = free_stack.back();
+        free_stack.pop_back();
+        ref[b] = 1;
+        return b;
+    }
+    void incref(int32_t b)
+    {
+        if (++ref[b] == 2) ++shared;
+    }
+    // returns true when the block became free
+    bool decref(int32_t b)
+    {
+        if (ref[b]-- == 2) --shared;
+        if (ref[b] == 0) {
+            free_stack.push_back(b);
+            return true;
+        }
+        return false;
+    }
+    // blocks an append of n tokens takes from the free list
+    int64_t needs(const Seq& s, int64_t n) const
+    {
+        if (n == 0) return 0;
+        int64_t cow = (s.ntok % block_size != 0 && ref[s.blocks.back()] > 1) ? 1 : 0;
+        int64_t total = (s.ntok + n + block_size - 1) / block_size;
+        return cow + total - (int64_t)s.blocks.size();
+    }
+    // caller has checked needs() against the free list
+    void append(Seq& s, int64_t n, int64_t* slots, int64_t* cow_pair, int32_t* cow)
+    {
+        int32_t did_cow = 0;
+        if (n > 0 && s.ntok % block_size != 0 && ref[s.blocks.back()] > 1) {
+            int32_t src = s.blocks.back();
+            int32_t dst = pop();
+            decref(src);
+            s.blocks.back() = dst;
+            did_cow = 1;
+            if (cow_pair) {
+                cow_pair[0] = src;
+                cow_pair[1] = dst;
+            }
+        }
+        for (int64_t i = 0; i < n; ++i) {
+            int64_t p = s.ntok + i;
+            if (p % block_size == 0) s.blocks.push_back(pop());
+            if (slots) slots[i] = (int64_t)s.blocks[p / block_size] * block_size + p % block_size;
+        }
+        s.ntok += n;
+        if (cow) *cow = did_cow;
+    }
+    Seq* find(int64_t id)
+    {
+        auto it = seqs.find(id);
+        return it == seqs.end() ? nullptr : &it->second;
+    }
+    const Seq* find(int64_t id) const
+    {
+        auto it = seqs.find(id);
+        return it == seqs.end() ? nullptr : &it->second;
+    }
+};
+
+extern "C" {
+
+int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* initial_order,
+                     pkv_allocator** out)
+{
+    if (!out || num_blocks < 0 || block_size < 1) return PKV_ERR_INVALID_ARG;
+    *out = nullptr;
+    pkv_allocator* a = new (std::nothrow) pkv_allocator();
+    if (!a) return PKV_ERR_INVALID_ARG;
+    a->num_blocks = num_blocks;
+    a->block_size = block_size;
+    a->ref.assign(num_blocks, 0);
+    a->free_stack.resize(num_blocks);
+    if (initial_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int32_t i = 0; i < num_blocks; ++i) {
+            int32_t b = initial_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                delete a;
+                return PKV_ERR_INVALID_ARG;
+            }
+            seen[b] = 1;
+            a->free_stack[num_blocks - 1 - i] = b;
+        }
+    } else {
+        for (int32_t i = 0; i < num_blocks; ++i) a->free_stack[num_blocks - 1 - i] = i;
+    }
+    *out = a;
+    return PKV_OK;
+}
+
+void pkv_alloc_destroy(pkv_allocator* a) { delete a; }
+
+int pkv_seq_add(pkv_allocator* a, int64_t seq)
+{
+    if (!a || a->find(seq)) return PKV_ERR_INVALID_ARG;
+    a->seqs.emplace(seq, Seq{});
+    return PKV_OK;
+}
+
+int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slots_out,
+                          int64_t* cow_pair_out, int32_t* cow_out)
+{
+    if (!a || n < 0) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->find(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    if (a->needs(*s, n) > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    a->append(*s, n, slots_out, cow_pair_out, cow_out);
+    return PKV_OK;
+}
+
+int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
+                         int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out)
+{
+    if (!a || n_seqs < 0 || (n_seqs > 0 && (!seqs || !slots_out))) return PKV_ERR_INVALID_ARG;
+    std::vector<Seq*> recs(n_seqs);
+    int64_t need = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        recs[i] = a->find(seqs[i]);
+        if (!recs[i]) return PKV_ERR_INVALID_ARG;
+        need += a->needs(*recs[i], 1);
+    }
+    {
+        std::vector<int64_t> ids(seqs, seqs + n_seqs);
+        std::sort(ids.begin(), ids.end());
+        if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PKV_ERR_INVALID_ARG;
+    }
+    if (need > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    int32_t ncow = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        int64_t pair[2];
+        int32_t cow = 0;
+        a->append(*recs[i], 1, slots_out + i, pair, &cow);
+        if (cow) {
+            if (cow_pairs_out) {
+                cow_pairs_out[2 * ncow] = pair[0];
+                cow_pairs_out[2 * ncow + 1] = pair[1];
+            }
+            ++ncow;
+        }
+    }
+    if (n_cow_out) *n_cow_out = ncow;
+    return PKV_OK;
+}
+
+int pkv_seq_free(pkv_allocator* a, int64_t seq)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->find(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
+    a->seqs.erase(seq);
+    return PKV_OK;
+}
+
+int pkv_seq_fork(pkv_allocator* a, int64_t parent, int64_t child)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    const Seq* p = a->find(parent);
+    if (!p || a->find(child)) return PKV_ERR_INVALID_ARG;
+    Seq c = *p;
+    for (int32_t b : c.blocks) a->incref(b);
+    a->seqs.emplace(child, std::move(c));
+    return PKV_OK;
+}
+
+int pkv_seq_share_prefix(pkv_allocator* a, int64_t seq, const int32_t* blocks, int32_t n_blocks,
+                         int32_t n_tokens)
+{
+    if (!a || n_blocks < 0 || n_tokens < 0 || (n_blocks > 0 && !blocks)) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->find(seq);
+    if (!s || !s->blocks.empty() || s->ntok != 0) return PKV_ERR_INVALID_ARG;
+    if ((int64_t)(n_tokens + a->block_size - 1) / a->block_size != n_blocks) return PKV_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_blocks; ++i) {
+        if (blocks[i] < 0 || blocks[i] >= a->num_blocks || a->ref[blocks[i]] < 1) return PKV_ERR_BAD_BLOCK;
+    }
+    for (int32_t i = 0; i < n_blocks; ++i) a->incref(blocks[i]);
+    s->blocks.assign(blocks, blocks + n_blocks);
+    s->ntok = n_tokens;
+    return PKV_OK;
+}
+
+int pkv_seq_block_table(const pkv_allocator* a, int64_t seq, int32_t* out, int32_t cap,
+                        int32_t* n_out)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    const Seq* s = a->find(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    int32_t n = (int32_t)s->blocks.size();
+    if (n_out) *n_out = n;
+    if (n > cap || (n > 0 && !out)) return PKV_ERR_INVALID_ARG;
+    if (n > 0) std::memcpy(out, s->blocks.data(), sizeof(int32_t) * n);
+    return PKV_OK;
+}
+
+int pkv_seq_num_tokens(const pkv_allocator* a, int64_t seq, int32_t* out)
+{
+    if (!a || !out) return PKV_ERR_INVALID_ARG;
+    const Seq* s = a->find(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    *out = (int32_t)s->ntok;
+    return PKV_OK;
+}
+
+int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
+                     int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
+                     int32_t* context_lens_out)
+{
+    if (!a || n_seqs < 0 || max_blocks_per_seq < 0 || (n_seqs > 0 && (!seqs || !tables_out)))
+        return PKV_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const Seq* s = a->find(seqs[i]);
+        if (!s || (int64_t)s->blocks.size() > max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
+    }
+    for (int32_t i = 0; i < n_seqs; ++i) {
+        const Seq* s = a->find(seqs[i]);
+        int32_t* row = tables_out + (int64_t)i * max_blocks_per_seq;
+        int32_t n = (int32_t)s->blocks.size();
+        if (n > 0) std::memcpy(row, s->blocks.data(), sizeof(int32_t) * n);
+        for (int32_t j = n; j < max_blocks_per_seq; ++j) row[j] = pad;
+        if (context_lens_out) context_lens_out[i] = (int32_t)s->ntok;
+    }
+    return PKV_OK;
+}
+
+int32_t pkv_num_free(const pkv_allocator* a) { return a ? (int32_t)a->free_stack.size() : -1; }
+
+int pkv_free_list(const pkv_allocator* a, int32_t* out, int32_t cap, int32_t* n_out)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    int32_t n = (int32_t)a->free_stack.size();
+    if (n_out) *n_out = n;
+    if (n > cap || (n > 0 && !out)) return PKV_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) out[i] = a->free_stack[n - 1 - i];
+    return PKV_OK;
+}
+
+int32_t pkv_refcount(const pkv_allocator* a, int32_t block)
+{
+    if (!a || block < 0 || block >= a->num_blocks) return -1;
+    return a->ref[block];
+}
+
+int pkv_alloc_get_stats(const pkv_allocator* a, pkv_alloc_stats* out)
+{
+    if (!a || !out) return PKV_ERR_INVALID_ARG;
+    out->num_blocks = a->num_blocks;
+    out->free_blocks = (int32_t)a->free_stack.size();
+    out->used_blocks = a->num_blocks - out->free_blocks;
+    out->shared_blocks = a->shared;
+    out->num_seqs = (int64_t)a->seqs.size();
+    int64_t tok = 0, frag = 0;
+    for (const auto& kv : a->seqs) {
+        tok += kv.second.ntok;
+        frag += (int64_t)kv.second.blocks.size() * a->block_size - kv.second.ntok;
+    }
+    out->num_tokens = tok;
+    out->fragmentation_tokens = frag;
+    return PKV_OK;
+}
+
+int pkv_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* positions, int32_t num_seqs, int32_t block_size,
+                     int64_t* slots_out)
+{
+    if (num_seqs < 0 || block_size < 1 || max_blocks_per_seq < 0 ||
+        (num_seqs > 0 && (!block_tables || !positions || !slots_out)))
+        return PKV_ERR_INVALID_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t p = positions[s];
+        if (p < 0) continue;
+        if (p / block_size >= max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
+        if (block_tables[(int64_t)s * max_blocks_per_seq + p / block_size] < 0) return PKV_ERR_BAD_BLOCK;
+    }
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t p = positions[s];
+        if (p < 0) {
+            slots_out[s] = -1;
+            continue;
+        }
+        int64_t phys = block_tables[(int64_t)s * max_blocks_per_seq + p / block_size];
+        slots_out[s] = phys * block_size + p % block_size;
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"

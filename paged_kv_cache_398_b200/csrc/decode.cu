@@ -1,0 +1,603 @@
+// paged_attention_decode: one decode step of attention whose keys and values
+// sit in fixed-size, non-contiguous physical blocks reached through
+// per-sequence block tables.  ("PagedAttention: How vLLM Serves AI Like an
+// Operating System", "How It Works" and "PagedAttention Memory Layout"; the
+// result is ordinary softmax attention -- "Throughput Impact: The Numbers":
+// no approximations.)
+//
+// Design (B200, sm_100a):
+//  * Work unit = (partition p of PKV_PARTITION_TOKENS tokens, kv head h,
+//    sequence s): one CTA.  The G = Hq / Hkv query heads that share kv head h
+//    are computed together, so each K/V block is read from HBM once per kv
+//    head, not once per query head.
+//  * Each (block, kv head) tile is one contiguous 16 x head_dim run in the
+//    cache layout, so it is fetched with two 1-D bulk copies (K and V; TMA
+//    engine, no tensor map, no multicast) into shared memory, completing on
+//    an mbarrier.  Every warp owns a ring of kStages tile pairs and walks
+//    its share of the partition's blocks (round-robin) with its own
+//    pipeline.  All waits are bounded (about 1 s) and report a timeout
+//    through the status word instead of hanging.
+//  * Q.K: each lane holds 16 bytes of the head dimension of one token for
+//    all G query heads (fp32, pre-scaled by scale * log2 e).  The partial
+//    dot products of a whole block are summed across the lanes of a token
+//    by a transposed shuffle reduction: each level halves the values a
+//    lane keeps.
+//  * Online softmax in fp32 (exp2), masked to the sequence's length, then
+//    P.V with fp32 accumulators.  Warps are merged in shared memory.  A
+//    sequence longer than one partition writes (max, sum, partial output)
+//    to the workspace, and a second kernel merges its partitions in a fixed
+//    order.
+//  * Partitioning depends only on the context length, so the result is
+//    bit-identical under any permutation of the physical placement.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kBlock = 16;
+constexpr int kPartTokens = PKV_PARTITION_TOKENS;
+constexpr int kPartBlocks = kPartTokens / kBlock;
+constexpr int kWarps = 4;
+constexpr int kStages = 2;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+template <typename T, int D, int G>
+struct Cfg {
+    static constexpr int kVec = 16 / (int)sizeof(T);   // elements per 16 bytes
+    static constexpr int kLpt = D / kVec;              // lanes per token row
+    static constexpr int kTpi = 32 / kLpt;             // tokens per warp iteration
+    static constexpr int kIters = kBlock / kTpi;       // iterations per block
+    static constexpr int kTileBytes = kBlock * D * (int)sizeof(T);
+    static constexpr int kNv = kIters * G;             // partial dots per lane per block
+    static constexpr int kItems = kBlock * G;          // scores per block
+    static constexpr int kItemsPerLane = (kItems + 31) / 32;
+    static_assert(kLpt >= 1 && kLpt <= 32 && 32 % kLpt == 0, "bad row split");
+    static_assert(32 % G == 0, "G must divide the warp");
+    // shared memory carve-up (bytes)
+    static constexpr int kTilesBytes = kWarps * kStages * 2 * kTileBytes;
+    static constexpr int kBarOff = kTilesBytes;
+    static constexpr int kScoreOff = kBarOff + kWarps * kStages * 8;
+    static constexpr int kBlkOff = kScoreOff + kWarps * kItems * 4;
+    static constexpr int kSmemBytes = kBlkOff + kPartBlocks * 4;
+    // the cross-warp merge reuses the tile area
+    static constexpr int kMergeBytes = kWarps * G * (D + 2) * 4;
+    static_assert(kMergeBytes <= kTilesBytes, "merge area does not fit");
+};
+
+// Transposed butterfly: sum N values across the lane bits MASK, MASK/2, .., 1.
+// While N >= 2 each level keeps half of the values (the half selected by the
+// lane's bit) and adds the partner's copy of that half; once one value is
+// left the remaining levels are plain butterflies.
+template <int N, int MASK>
+__device__ __forceinline__ void treduce(float* v, int lane)
+{
+    if constexpr (MASK > 0) {
+        if constexpr (N >= 2) {
+            constexpr int H = N / 2;
+            const bool up = (lane & MASK) != 0;
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                const float send = up ? v[k] : v[k + H];
+                const float keep = up ? v[k + H] : v[k];
+                v[k] = keep + __shfl_xor_sync(0xffffffffu, send, MASK);
+            }
+            treduce<H, MASK / 2>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], MASK);
+            treduce<1, MASK / 2>(v, lane);
+        }
+    }
+}
+
+// Index (into the original N values) of the first value a lane keeps.
+template <int N, int MASK>
+__device__ __forceinline__ int treduce_base(int lane)
+{
+    if constexpr (MASK > 0 && N >= 2) {
+        return ((lane & MASK) ? N / 2 : 0) + treduce_base<N / 2, MASK / 2>(lane);
+    } else {
+        return 0;
+    }
+}
+
+// Lane bits on which values are duplicated (plain butterfly levels).
+template <int N, int MASK>
+__host__ __device__ constexpr int treduce_dup_mask()
+{
+    if constexpr (MASK == 0) {
+        return 0;
+    } else if constexpr (N >= 2) {
+        return treduce_dup_mask<N / 2, MASK / 2>();
+    } else {
+        return MASK | treduce_dup_mask<1, MASK / 2>();
+    }
+}
+
+// Lane 0 of a warp: fetch the K and V tiles at element offset `off` into the
+// tile pair at `dst` (K then V), completing on `bar`.
+template <int kTileBytes, typename T>
+__device__ __forceinline__ void issue_tile_pair(uint8_t* dst, uint64_t* bar, const T* k_cache,
+                                                const T* v_cache, int64_t off, uint64_t policy)
+{
+    // order this warp's earlier generic reads of the tiles before the async writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    pkv::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+    pkv::bulk_load(dst, k_cache + off, kTileBytes, bar, policy);
+    pkv::bulk_load(dst + kTileBytes, v_cache + off, kTileBytes, bar, policy);
+}
+
+struct SeqRange {
+    int ctx;       // tokens attended (after clamping)
+    int nparts;    // partitions of this sequence
+    bool bad;      // context length < 1
+};
+
+__device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int max_ctx,
+                                              bool report, int* status)
+{
+    SeqRange r;
+    int ctx = __ldg(context_lens + s);
+    int flag = 0;
+    if (ctx < 1) {
+        flag = 1;
+        ctx = 0;
+    }
+    if (ctx > mb * kBlock) {
+        flag = 1;
+        ctx = mb * kBlock;
+    }
+    if (ctx > max_ctx) {
+        flag = 1;
+        ctx = max_ctx;
+    }
+    if (flag && report) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
+    r.ctx = ctx;
+    r.nparts = (ctx + kPartTokens - 1) / kPartTokens;
+    r.bad = ctx < 1;
+    return r;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32)
+    decode_partition_kernel(T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
+                            const T* __restrict__ q, const T* __restrict__ k_cache,
+                            const T* __restrict__ v_cache, const int32_t* __restrict__ block_tables,
+                            int32_t mb, const int32_t* __restrict__ context_lens, int32_t max_ctx,
+                            int32_t num_q_heads, int32_t num_kv_heads, int32_t num_blocks,
+                            float scale_log2, int32_t max_parts, int* status)
+{
+    using C = Cfg<T, D, G>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0,
+                                  status);
+    if (sr.bad) {
+        // nothing to attend to: a zero row (flagged above)
+        if (p == 0) {
+            for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+                pkv::store_out(out + ((int64_t)s * num_q_heads + h * G) * D + i, 0.0f);
+            }
+        }
+        return;
+    }
+    if (p >= sr.nparts) return;
+
+    const int nblk_seq = (sr.ctx + kBlock - 1) / kBlock;
+    const int blk0 = p * kPartBlocks;
+    const int nb = min(kPartBlocks, nblk_seq - blk0);
+    const int last_valid = sr.ctx - (nblk_seq - 1) * kBlock;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
+    float* s_sc = reinterpret_cast<float*>(smem + C::kScoreOff) + warp * C::kItems;
+    int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
+    uint8_t* my_tiles = smem + warp * (kStages * 2 * C::kTileBytes);
+
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
+        if (b < 0 || b >= num_blocks) {
+            pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
+            b = 0;
+        }
+        s_blk[i] = b;
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) pkv::mbar_init(&bars[st], 1);
+        pkv::fence_mbar_init();
+    }
+    __syncthreads();
+
+    // this warp's blocks: j = warp + k * kWarps, k < nw
+    const int nw = nb > warp ? (nb - warp + kWarps - 1) / kWarps : 0;
+    const int64_t tile_elems = (int64_t)kBlock * D;
+    uint64_t policy = 0;
+    if (lane == 0) policy = pkv::policy_evict_first();
+
+    if (lane == 0) {
+        for (int k = 0; k < nw && k < kStages; ++k) {
+            issue_tile_pair<C::kTileBytes>(my_tiles + (k % kStages) * 2 * C::kTileBytes, &bars[k % kStages],
+                                           k_cache, v_cache,
+                                           ((int64_t)s_blk[warp + k * kWarps] * num_kv_heads + h) * tile_elems,
+                                           policy);
+        }
+    }
+
+    // this lane's slice of the G query vectors, in the log2 domain
+    const int c = lane % C::kLpt;
+    const int tsub = lane / C::kLpt;
+    float qf[G][C::kVec];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(
+            q + ((int64_t)s * num_q_heads + h * G + g) * D + c * C::kVec);
+        pkv::Elem<T>::to_float(raw, qf[g]);
+#pragma unroll
+        for (int e = 0; e < C::kVec; ++e) qf[g][e] *= scale_log2;
+    }
+
+    // which (token, head) each reduced value stands for
+    constexpr int kR = C::kNv >= C::kLpt ? C::kNv / C::kLpt : 1;
+    const int jbase = treduce_base<C::kNv, C::kLpt / 2>(lane);
+    constexpr int kDup = treduce_dup_mask<C::kNv, C::kLpt / 2>();
+    const bool owner = (lane & kDup) == 0;
+    const int g_lane = lane % G;  // the head of this lane's softmax items
+
+    float m_run[G];
+    float acc[G][C::kVec];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m_run[g] = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < C::kVec; ++e) acc[g][e] = 0.0f;
+    }
+    float l_part = 0.0f;   // this lane's share of the softmax sum of head g_lane
+    bool timed_out = false;
+    int consumed = 0;
+
+    for (int k = 0; k < nw; ++k) {
+        const int st = k % kStages;
+        if (!pkv::mbar_wait(&bars[st], (k / kStages) & 1, kWaitLimitNs)) {
+            timed_out = true;
+            break;
+        }
+        const T* sk = reinterpret_cast<const T*>(my_tiles + st * 2 * C::kTileBytes);
+        const T* sv = reinterpret_cast<const T*>(my_tiles + st * 2 * C::kTileBytes + C::kTileBytes);
+        const int valid = (blk0 + warp + k * kWarps == nblk_seq - 1) ? last_valid : kBlock;
+
+        // ---- Q.K for the block's 16 tokens -----------------------------
+        float part[C::kNv];
+#pragma unroll
+        for (int it = 0; it < C::kIters; ++it) {
+            const int t = it * C::kTpi + tsub;
+            const uint4 raw = *reinterpret_cast<const uint4*>(sk + t * D + c * C::kVec);
+            float kf[C::kVec];
+            pkv::Elem<T>::to_float(raw, kf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float d0 = 0.0f;
+#pragma unroll
+                for (int e = 0; e < C::kVec; ++e) d0 = fmaf(qf[g][e], kf[e], d0);
+                part[it * G + g] = d0;
+            }
+        }
+        treduce<C::kNv, C::kLpt / 2>(part, lane);
+        if (owner) {
+#pragma unroll
+            for (int r = 0; r < kR; ++r) {
+                const int j = jbase + r;
+                const int t = (j / G) * C::kTpi + tsub;
+                s_sc[t * G + (j % G)] = part[r];
+            }
+        }
+        __syncwarp();
+
+        // ---- online softmax ----------------------------------------------
+        float x[C::kItemsPerLane];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < C::kItemsPerLane; ++u) {
+            const int idx = lane + 32 * u;
+            x[u] = -INFINITY;
+            if (idx < C::kItems && idx / G < valid) x[u] = s_sc[idx];
+            mx = fmaxf(mx, x[u]);
+        }
+#pragma unroll
+        for (int o = G; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float alpha[G];
+        bool rescale = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float bm = __shfl_sync(0xffffffffu, mx, g);
+            const float mn = fmaxf(m_run[g], bm);
+            alpha[g] = exp2f(m_run[g] - mn);
+            rescale |= (mn != m_run[g]);
+            m_run[g] = mn;
+        }
+        float m_mine = m_run[0], a_mine = alpha[0];  // values of head g_lane (no local memory)
+#pragma unroll
+        for (int g = 1; g < G; ++g) {
+            if (g == g_lane) {
+                m_mine = m_run[g];
+                a_mine = alpha[g];
+            }
+        }
+        float psum = 0.0f;
+#pragma unroll
+        for (int u = 0; u < C::kItemsPerLane; ++u) {
+            const int idx = lane + 32 * u;
+            const float pr = exp2f(x[u] - m_mine);
+            if (idx < C::kItems) s_sc[idx] = pr;
+            psum += pr;
+        }
+        l_part = l_part * a_mine + psum;
+        if (rescale) {
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < C::kVec; ++e) acc[g][e] *= alpha[g];
+        }
+        __syncwarp();
+
+        // ---- P.V ----------------------------------------------------------
+#pragma unroll
+        for (int it = 0; it < C::kIters; ++it) {
+            const int t = it * C::kTpi + tsub;
+            if (t < valid) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(sv + t * D + c * C::kVec);
+                float vf[C::kVec];
+                pkv::Elem<T>::to_float(raw, vf);
+                float pg[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) pg[g] = s_sc[t * G + g];
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < C::kVec; ++e) acc[g][e] = fmaf(pg[g], vf[e], acc[g][e]);
+            }
+        }
+        __syncwarp();
+        ++consumed;
+        if (lane == 0 && k + kStages < nw) {
+            const int kn = k + kStages;
+            issue_tile_pair<C::kTileBytes>(my_tiles + st * 2 * C::kTileBytes, &bars[st], k_cache, v_cache,
+                                           ((int64_t)s_blk[warp + kn * kWarps] * num_kv_heads + h) * tile_elems,
+                                           policy);
+        }
+    }
+
+    if (timed_out) {
+        if (lane == 0) pkv::raise_flag(status, PKV_DEV_WAIT_TIMEOUT);
+        // let the copies still in flight land before the smem is reused
+        for (int k = consumed; k < nw && k < consumed + kStages; ++k) {
+            pkv::mbar_wait(&bars[k % kStages], (k / kStages) & 1, kWaitLimitNs);
+        }
+    }
+
+    // ---- merge the lanes of this warp ------------------------------------
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) l_part += __shfl_xor_sync(0xffffffffu, l_part, o);
+#pragma unroll
+    for (int o = C::kLpt; o < 32; o <<= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < C::kVec; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+
+    __syncthreads();  // every warp is done with its tiles: reuse them for the merge
+    float* mg = reinterpret_cast<float*>(smem);  // [kWarps][G][D + 2]: m, l, acc[D]
+    float* mine = mg + warp * G * (D + 2);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        if (lane == g) {
+            mine[g * (D + 2)] = m_run[g];
+            mine[g * (D + 2) + 1] = l_part;  // lane g holds the full sum of head g
+        }
+    }
+    if (tsub == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < C::kVec; ++e) mine[g * (D + 2) + 2 + c * C::kVec + e] = acc[g][e];
+    }
+    __syncthreads();
+
+    const int hq0 = h * G;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+        const int g = i / D, d = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[(w * G + g) * (D + 2)]);
+        float L = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float* rec = mg + (w * G + g) * (D + 2);
+            const float wgt = exp2f(rec[0] - M);  // empty warp: m = -inf -> 0
+            L = fmaf(rec[1], wgt, L);
+            O = fmaf(rec[2 + d], wgt, O);
+        }
+        const int64_t row = (int64_t)s * num_q_heads + hq0 + g;
+        if (sr.nparts == 1) {
+            pkv::store_out(out + row * D + d, O / L);
+        } else {
+            ws_acc[(row * max_parts + p) * D + d] = O;
+            if (d == 0) {
+                ws_ml[(row * max_parts + p) * 2] = M;
+                ws_ml[(row * max_parts + p) * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+// Merge the partitions of every (sequence, query head) that has more than
+// one: out = sum_p acc_p 2^(m_p - M) / sum_p l_p 2^(m_p - M), M = max_p m_p,
+// in partition order.  One warp per (sequence, query head).
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+    decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
+                         const float* __restrict__ ws_ml, const int32_t* __restrict__ context_lens,
+                         int32_t num_seqs, int32_t num_q_heads, int32_t mb, int32_t max_ctx,
+                         int32_t max_parts)
+{
+    constexpr int kPer = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (row >= (int64_t)num_seqs * num_q_heads) return;
+    const int s = (int)(row / num_q_heads);
+    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, false, nullptr);
+    if (sr.bad || sr.nparts <= 1) return;
+    const float* ml = ws_ml + row * max_parts * 2;
+    const float* acc = ws_acc + row * max_parts * D;
+
+    float M = -INFINITY;
+    for (int p0 = 0; p0 < sr.nparts; p0 += 32) {
+        const int pp = p0 + lane;
+        float m = pp < sr.nparts ? ml[pp * 2] : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        M = fmaxf(M, m);
+    }
+    float L = 0.0f;
+    float o[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) o[e] = 0.0f;
+    for (int p0 = 0; p0 < sr.nparts; p0 += 32) {
+        const int pp = p0 + lane;
+        float w = 0.0f, lw = 0.0f;
+        if (pp < sr.nparts) {
+            w = exp2f(ml[pp * 2] - M);
+            lw = ml[pp * 2 + 1] * w;
+        }
+        const int n = min(32, sr.nparts - p0);
+        for (int j = 0; j < n; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            L += __shfl_sync(0xffffffffu, lw, j);
+            const float* a = acc + (int64_t)(p0 + j) * D + lane * kPer;
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) o[e] = fmaf(a[e], wj, o[e]);
+        }
+    }
+    const float inv = 1.0f / L;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) pkv::store_out(out + row * D + lane * kPer + e, o[e] * inv);
+}
+
+template <typename T, int D, int G>
+int launch(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* bt,
+           int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
+           int32_t NB, float scale, void* ws, cudaStream_t stream, int* status)
+{
+    using C = Cfg<T, D, G>;
+    // The shared-memory opt-in is a per-device property of the kernel.
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+        return PKV_ERR_CUDA;
+    }
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(decode_partition_kernel<T, D, G>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) {
+            pkv::record_cuda_error(e);
+            return PKV_ERR_CUDA;
+        }
+        configured[dev] = true;
+    }
+    const int max_parts = (max_ctx + kPartTokens - 1) / kPartTokens;
+    float* ws_acc = static_cast<float*>(ws);
+    float* ws_ml = ws_acc ? ws_acc + (size_t)S * Hq * max_parts * D : nullptr;
+    const float scale_log2 = (float)((double)scale * 1.4426950408889634);
+    dim3 grid((unsigned)max_parts, (unsigned)Hkv, (unsigned)S);
+    decode_partition_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
+        static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), static_cast<const T*>(k_cache),
+        static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2, max_parts, status);
+    int rc = pkv::check_launch();
+    if (rc != PKV_OK || max_parts == 1) return rc;
+    const int64_t rows = (int64_t)S * Hq;
+    decode_reduce_kernel<T, D><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(
+        static_cast<T*>(out), ws_acc, ws_ml, cl, S, Hq, mb, max_ctx, max_parts);
+    return pkv::check_launch();
+}
+
+template <typename T, int D>
+int dispatch_g(int G, void* out, const void* q, const void* kc, const void* vc, const int32_t* bt,
+               int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
+               int32_t NB, float scale, void* ws, cudaStream_t st, int* status)
+{
+    switch (G) {
+        case 1: return launch<T, D, 1>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+        case 2: return launch<T, D, 2>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+        case 4: return launch<T, D, 4>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+        case 8: return launch<T, D, 8>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+int dispatch_d(int D, int G, void* out, const void* q, const void* kc, const void* vc, const int32_t* bt,
+               int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
+               int32_t NB, float scale, void* ws, cudaStream_t st, int* status)
+{
+    if (D == 64) return dispatch_g<T, 64>(G, out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+    if (D == 128) return dispatch_g<T, 128>(G, out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+    return PKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                                  int32_t head_dim, int32_t max_context_len)
+{
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+    const size_t parts = ((size_t)max_context_len + kPartTokens - 1) / kPartTokens;
+    if (parts <= 1) return 0;
+    return (size_t)num_seqs * num_q_heads * parts * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+extern "C" int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t num_seqs,
+                                      int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                                      int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (pkv::dtype_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        num_blocks < 1 || max_blocks_per_seq < 1 || !isfinite(scale))
+        return PKV_ERR_INVALID_ARG;
+    if (block_size != kBlock || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (max_context_len < 1 || num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (!pkv::aligned16(q) || !pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) ||
+        ((uintptr_t)out % pkv::dtype_bytes(dtype)) || ((uintptr_t)block_tables & 3u) ||
+        ((uintptr_t)context_lens & 3u))
+        return PKV_ERR_INVALID_ARG;
+    const size_t need = paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+        return PKV_ERR_INVALID_ARG;
+    int* status = pkv::status_word_for_current_device();
+    if (!status) return PKV_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    switch (dtype) {
+        case PKV_F32:
+            return dispatch_d<float>(head_dim, G, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                     context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
+                                     num_blocks, scale, workspace, st, status);
+        case PKV_F16:
+            return dispatch_d<__half>(head_dim, G, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                      context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
+                                      num_blocks, scale, workspace, st, status);
+        default:
+            return dispatch_d<__nv_bfloat16>(head_dim, G, out, q, k_cache, v_cache, block_tables,
+                                             max_blocks_per_seq, context_lens, num_seqs, max_context_len,
+                                             num_q_heads, num_kv_heads, num_blocks, scale, workspace, st,
+                                             status);
+    }
+}

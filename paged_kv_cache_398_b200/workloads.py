@@ -246,3 +246,42 @@ def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min
                           context_lens=torch.tensor(ctx, dtype=torch.int32), block_tables=bt,
                           copy_pairs=pairs, q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new,
                           v_new=v_new, scale=1.0 / math.sqrt(D), seed=seed, meta=meta)
+
+
+def make_custom(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype,
+                device="cpu", *, seed: int = 1234, spare_blocks: int = 3,
+                max_blocks_per_seq=None, pad_random: bool = False) -> DecodeWorkload:
+    """A batch with the given context lengths and head shape, blocks dealt
+    from a seeded permutation of a pool with `spare_blocks` unused blocks."""
+    g = torch.Generator().manual_seed(seed)
+    B = BLOCK_SIZE
+    ctx = [int(c) for c in context_lens]
+    need = sum(_nblk(max(c, 1), B) for c in ctx)
+    NB = need + spare_blocks
+    perm = torch.randperm(NB, generator=g).tolist()
+    tables, k = [], 0
+    for c in ctx:
+        n = _nblk(max(c, 1), B)
+        tables.append(perm[k:k + n])
+        k += n
+    MB = max_blocks_per_seq or max(len(t) for t in tables)
+    bt = torch.full((len(ctx), MB), -1, dtype=torch.int32)
+    for s, row in enumerate(tables):
+        bt[s, :len(row)] = torch.tensor(row, dtype=torch.int32)
+    S, Hq, Hkv, D = len(ctx), num_q_heads, num_kv_heads, head_dim
+    dev = torch.device(device)
+    gd = g if dev.type == "cpu" else torch.Generator(device=dev).manual_seed(seed)
+    q = _randn((S, Hq, D), dtype, gd, dev)
+    k_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
+    v_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
+    k_new = _randn((S, Hkv, D), dtype, gd, dev)
+    v_new = _randn((S, Hkv, D), dtype, gd, dev)
+    if pad_random:
+        junk = torch.randint(0, NB, bt.shape, generator=g, dtype=torch.int32)
+        bt = torch.where(bt < 0, junk, bt)
+    return DecodeWorkload(name="custom", dtype=dtype, num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv,
+                          head_dim=D, block_size=B, num_blocks=NB,
+                          context_lens=torch.tensor(ctx, dtype=torch.int32), block_tables=bt,
+                          copy_pairs=torch.empty(0, 2, dtype=torch.int64), q=q, k_cache=k_cache,
+                          v_cache=v_cache, k_new=k_new, v_new=v_new, scale=1.0 / math.sqrt(D),
+                          seed=seed, meta={"workload": "custom"})

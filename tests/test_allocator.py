@@ -1,0 +1,195 @@
+"""The native host block allocator against the oracle's list model (CPU only).
+
+Every operation is applied to both; block tables, slots, copy pairs, free
+lists, reference counts and statistics must agree exactly.  The pages'
+worked examples run through the native allocator as well.
+"""
+
+import random
+
+import pytest
+
+import paged_kv_cache_398_b200 as pkv
+from oracle.allocator_model import AllocatorModel, InvalidArgument, OutOfBlocks
+from tests.conftest import load_golden
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from paged_kv_cache_398_b200.build import build_library
+    build_library()
+
+
+def _same(a: pkv.BlockAllocator, m: AllocatorModel, seqs):
+    assert a.free_list() == m.free_list()
+    assert a.num_free() == m.num_free()
+    for s in seqs:
+        assert a.block_table(s) == m.block_table(s)
+        assert a.num_tokens(s) == m.num_tokens(s)
+    for b in range(m.num_blocks):
+        assert a.refcount(b) == m.refcount(b)
+    st, sm = a.stats(), m.stats()
+    for k in sm:
+        assert st[k] == sm[k], k
+
+
+def test_worked_examples_native():
+    gold = load_golden("worked_block_tables.json")
+    order = [0, 2, 6, 4, 7, 1, 3, 9, 5, 8, 10, 11]
+    a = pkv.BlockAllocator(12, 16, initial_order=order)
+    for sid, req, ntok in ((0, "A", 40), (1, "B", 48), (2, "C", 20)):
+        a.add(sid)
+        a.append_tokens(sid, ntok)
+        assert a.block_table(sid) == gold["block_tables"][req]
+    assert sorted(a.free_list()) == gold["free_blocks"]
+
+    g = load_golden("on_demand_growth.json")
+    a = pkv.BlockAllocator(100, 16)
+    a.add(1)
+    have = 0
+    for tokens, blocks in g["tokens_to_blocks"]:
+        a.append_tokens(1, tokens - have)
+        have = tokens
+        assert len(a.block_table(1)) == blocks
+    assert a.stats()["fragmentation_tokens"] <= g["max_waste_tokens"]
+
+    ps = load_golden("parallel_sampling.json")
+    a = pkv.BlockAllocator(20, 16)
+    a.add(100)
+    a.append_tokens(100, 6 * 16)
+    for j in range(4):
+        a.fork(100, j)
+    a.free(100)
+    for j in range(4):
+        a.append_tokens(j, 32)
+        assert a.block_table(j) == ps["prompt_blocks"] + ps["unique_blocks"][j]
+    assert a.stats()["used_blocks"] == 14
+
+    pre = load_golden("prefix_sharing.json")
+    a = pkv.BlockAllocator(5000, 16)
+    a.add(-1)
+    a.append_tokens(-1, 64)
+    for u in range(pre["users"]):
+        a.add(u)
+        a.share_prefix(u, pre["prefix_blocks"], 64)
+    a.free(-1)
+    assert a.stats()["used_blocks"] == pre["blocks_with_sharing"]
+    assert a.refcount(0) == pre["users"]
+
+    rel = load_golden("immediate_release.json")
+    a = pkv.BlockAllocator(20, 16)
+    a.add(0)
+    a.append_tokens(0, 6 * 16 - 1)
+    before = a.num_free()
+    a.free(0)
+    assert a.num_free() - before == rel["pages_of_finished_sequence"]
+
+
+def test_copy_on_write_native():
+    a = pkv.BlockAllocator(32, 16)
+    a.add(0)
+    a.append_tokens(0, 40)
+    for j in (1, 2, 3):
+        a.fork(0, j)
+    pairs = []
+    for j in (1, 2, 3, 0):
+        slots, cow = a.append_tokens(j, 1)
+        if cow:
+            pairs.append(cow)
+    assert pairs == [(2, 3), (2, 4), (2, 5)]
+    assert a.refcount(2) == 1
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_random_operations_match_model(seed):
+    rng = random.Random(seed)
+    NB = rng.choice([24, 64, 200])
+    order = list(range(NB))
+    rng.shuffle(order)
+    a = pkv.BlockAllocator(NB, 16, initial_order=order)
+    m = AllocatorModel(NB, 16, initial_order=order)
+    live, next_id = [], 0
+    for step in range(400):
+        op = rng.random()
+        try:
+            if op < 0.2 or not live:
+                m.add(next_id)
+                a.add(next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op < 0.55:
+                s = rng.choice(live)
+                n = rng.choice([0, 1, 1, 1, 3, 15, 16, 17, 40])
+                try:
+                    want = m.append_tokens(s, n)
+                except OutOfBlocks:
+                    with pytest.raises(pkv.OutOfBlocks):
+                        a.append_tokens(s, n)
+                else:
+                    got = a.append_tokens(s, n)
+                    assert got == (want[0], want[1])
+            elif op < 0.65:
+                batch = rng.sample(live, k=min(len(live), rng.randint(1, 6)))
+                try:
+                    ws, wp = m.append_one_batch(batch)
+                except OutOfBlocks:
+                    with pytest.raises(pkv.OutOfBlocks):
+                        a.append_one_batch(batch)
+                else:
+                    gs, gp = a.append_one_batch(batch)
+                    assert gs.tolist() == ws and [tuple(p) for p in gp.tolist()] == wp
+            elif op < 0.8:
+                s = rng.choice(live)
+                m.fork(s, next_id)
+                a.fork(s, next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op < 0.87 and live:
+                s = rng.choice(live)
+                if m.num_tokens(s) == 0:
+                    src = rng.choice(live)
+                    blocks = m.block_table(src)
+                    full = len(blocks) * 16
+                    if blocks and m.num_tokens(src) == full:
+                        m.share_prefix(s, blocks, full)
+                        a.share_prefix(s, blocks, full)
+            else:
+                s = rng.choice(live)
+                m.free(s)
+                a.free(s)
+                live.remove(s)
+        except InvalidArgument:
+            pytest.fail("model rejected a generated operation")
+        _same(a, m, live)
+
+
+def test_invalid_operations_native():
+    a = pkv.BlockAllocator(4, 16)
+    a.add(0)
+    with pytest.raises(pkv.PagedKVError):
+        a.add(0)
+    with pytest.raises(pkv.PagedKVError):
+        a.free(9)
+    with pytest.raises(pkv.PagedKVError):
+        a.fork(9, 10)
+    a.append_tokens(0, 64)
+    with pytest.raises(pkv.OutOfBlocks):
+        a.append_tokens(0, 1)
+    assert a.block_table(0) == [0, 1, 2, 3]
+    with pytest.raises(pkv.PagedKVError):
+        pkv.BlockAllocator(3, 16, initial_order=[0, 0, 1])
+    a.add(1)
+    with pytest.raises(pkv.PagedKVError):
+        a.share_prefix(1, [0, 1], 40)      # 40 tokens need 3 blocks
+    with pytest.raises(pkv.PagedKVError):
+        a.append_one_batch([0, 0])
+
+
+def test_batch_tables_pad():
+    a = pkv.BlockAllocator(10, 16)
+    for s, n in ((0, 5), (1, 33)):
+        a.add(s)
+        a.append_tokens(s, n)
+    t, lens = a.batch_tables([1, 0], 4, pad=-1)
+    assert t.tolist() == [[1, 2, 3, -1], [0, -1, -1, -1]]
+    assert lens.tolist() == [33, 5]

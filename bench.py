@@ -60,12 +60,15 @@ class Step:
     """Everything one decode step needs, resident on the GPU."""
 
 
-def build_step(number: int, device, rank: int = 0):
+def build_step(number: int, device, rank: int = 0, num_seqs=None):
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 
     seed = rank_seed(number, rank)
-    w = make_workload(number, device=device, seed=seed)   # lengths on host, values on the GPU
+    kw = {}
+    if num_seqs:
+        kw = {"num_prompts": max(1, num_seqs // 4)} if number == 5 else {"num_seqs": num_seqs}
+    w = make_workload(number, device=device, seed=seed, **kw)   # lengths on host, values on the GPU
     S = w.num_seqs
     st = Step()
     st.w = w
@@ -275,7 +278,7 @@ def cpu_baseline(st, threads: int):
     probe = sub_workload(st.w, tables, lens, pairs, [0])
     t1 = oracle_step_timed(probe, 1)
     per_tok = t1 / max(1, int(lens[0]))
-    seqs = pick_sample(lens, 15.0, per_tok)
+    seqs = pick_sample(lens, 30.0, per_tok)
     sub = sub_workload(st.w, tables, lens, pairs, seqs)
     t = oracle_step_timed(sub, threads)
     return {"value": sample_kv_bytes(sub) / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -358,7 +361,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    st = build_step(args.workload, dev, rank)
+    st = build_step(args.workload, dev, rank, args.num_seqs)
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
     # the oracle sample is copied off the device before the first product step
@@ -466,12 +469,14 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-seqs", type=int, default=16)
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="smaller batch of the same recipe (profiling); the default is the full workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -59,6 +59,8 @@ extern "C" {
 #define PKV_ERR_OUT_OF_BLOCKS (-4) /* the free list cannot cover the request */
 #define PKV_ERR_BAD_BLOCK (-5)     /* block id outside the pool / not held   */
 #define PKV_ERR_DEVICE (-6)        /* a device-side check failed (flags set) */
+#define PKV_ERR_SCRATCH_LIMIT (-7) /* the batch needs more scratch than the
+                                      fixed array of the no-alloc variant   */
 
 /* ---- element types ----------------------------------------------------- */
 #define PKV_F32 0
@@ -150,6 +152,44 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                            int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * paged_attention_decode_noalloc -- paged_attention_decode without a
+ * caller-supplied workspace, for callers that cannot allocate device memory
+ * when they decode.  Examples: code that runs while a stream is being
+ * captured into a CUDA graph (allocating is not allowed there), runtimes
+ * whose device memory is a fixed arena handed out at start-up, and embedders
+ * that must never call the CUDA allocator.  It has no counterpart in the
+ * pages; it is an interface convenience of this library.
+ *
+ * The arguments and the result are those of paged_attention_decode.  The
+ * split-K scratch comes from one fixed array of PKV_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) in the library's own device memory.  Every GPU that loads the
+ * library's decode module holds that array until the process exits.  The
+ * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
+ *
+ *  - Limit: if paged_attention_workspace_bytes(num_seqs, num_q_heads,
+ *    head_dim, max_context_len) exceeds PKV_NOALLOC_SCRATCH_BYTES, the call
+ *    returns PKV_ERR_SCRATCH_LIMIT and enqueues nothing.  Example that fits:
+ *    128 sequences x 32 query heads x 8192 tokens at head_dim 128 need 34 MB.
+ *  - First call on a device: it resolves the array's device address
+ *    (cudaGetSymbolAddress) and sets the decode kernels' shared-memory
+ *    limit, once per device, with that device current.  Make that first call
+ *    before any stream capture.
+ *  - Sharing: all calls on one device share the one array, which keeps the
+ *    last call's contents.  Nothing in it needs to start at zero: each call
+ *    writes every scratch entry before reading it.  Calls that overlap on
+ *    the GPU (for example on two streams without ordering between them)
+ *    race on the array; order them on one stream or by events.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES 67108864
+int paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                   int32_t num_seqs, int32_t max_context_len, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                   int32_t num_blocks, float scale, int32_t dtype, void* stream);
 
 /*
  * block_copy -- copy-on-write copies: for each pair (src, dst), physical

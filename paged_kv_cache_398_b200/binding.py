@@ -111,6 +111,31 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                   max_context_len: int, stream=None) -> torch.Tensor:
+    """paged_attention_decode with the library's fixed scratch array instead
+    of a workspace: for callers that cannot allocate device memory when they
+    decode.  Batches needing more than PKV_NOALLOC_SCRATCH_BYTES of scratch
+    raise PagedKVError (PKV_ERR_SCRATCH_LIMIT).  Calls that overlap on the
+    GPU share that array and race."""
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    _cuda("q", q, k_cache.dtype, 3)
+    _cuda("out", out, k_cache.dtype, 3)
+    _cuda("block_tables", block_tables, torch.int32, 2)
+    _cuda("context_lens", context_lens, torch.int32, 1)
+    S, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (S, Hq, D):
+        raise ValueError("q/out must be [S, Hq, D] with the cache's head_dim")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables/context_lens must have one row per sequence")
+    rc = lib().paged_attention_decode_noalloc(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(),
+                                              v_cache.data_ptr(), block_tables.data_ptr(), block_tables.shape[1],
+                                              context_lens.data_ptr(), S, int(max_context_len), Hq, Hkv, D, B, NB,
+                                              float(scale), _dtype_code(k_cache), _stream(q.device, stream))
+    check("paged_attention_decode_noalloc", rc)
+    return out
+
+
 def block_copy(k_cache, v_cache, pairs, stream=None) -> None:
     """Copy-on-write copies; pairs: host int64 [N, 2] (src, dst) tensor or list."""
     NB, Hkv, B, D = _cache_shape(k_cache, v_cache)

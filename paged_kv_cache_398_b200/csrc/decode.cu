@@ -31,6 +31,8 @@
 //    bit-identical under any permutation of the physical placement.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -600,4 +602,61 @@ extern "C" int paged_attention_decode(void* out, const void* q, const void* k_ca
                                              num_q_heads, num_kv_heads, num_blocks, scale, workspace, st,
                                              status);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Callers that cannot allocate device memory when
+// they decode get the split-K scratch from this fixed array instead of a
+// workspace of their own.  See paged_attention_decode_noalloc in paged_kv.h.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the array on the current device, resolved once per device.
+// In host code `g_noalloc_scratch` names a host-side stand-in, not device memory,
+// so it must never be handed to a kernel directly.
+int noalloc_scratch(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+        pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+        return PKV_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+            return PKV_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                              const void* v_cache, const int32_t* block_tables,
+                                              int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                              int32_t num_seqs, int32_t max_context_len, int32_t num_q_heads,
+                                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                              int32_t num_blocks, float scale, int32_t dtype, void* stream)
+{
+    const size_t need = paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len);
+    if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != PKV_OK) return rc;
+    return paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                  num_seqs, max_context_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                                  num_blocks, scale, dtype, scratch, (size_t)PKV_NOALLOC_SCRATCH_BYTES, stream);
 }

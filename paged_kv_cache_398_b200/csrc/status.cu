@@ -88,6 +88,7 @@ const char* pkv_status_string(int status)
         case PKV_ERR_OUT_OF_BLOCKS: return "out of free blocks";
         case PKV_ERR_BAD_BLOCK: return "bad block id";
         case PKV_ERR_DEVICE: return "device-side check failed";
+        case PKV_ERR_SCRATCH_LIMIT: return "batch needs more scratch than the fixed no-alloc array";
         default: return "unknown status";
     }
 }

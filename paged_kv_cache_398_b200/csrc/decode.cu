@@ -31,7 +31,10 @@
 //    bit-identical under any permutation of the physical placement.
 #include <math.h>
 
+#include <cudaTypedefs.h>
+
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -486,14 +489,61 @@ __global__ void __launch_bounds__(128)
     for (int e = 0; e < kPer; ++e) pkv::store_out(out + row * D + lane * kPer + e, o[e] * inv);
 }
 
-template <typename T, int D, int G>
-int launch(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* bt,
-           int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
-           int32_t NB, float scale, void* ws, cudaStream_t stream, int* status)
+}  // namespace
+
+#include "decode_tc.cuh"
+
+namespace {
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    using C = Cfg<T, D, G>;
-    // The shared-memory opt-in is a per-device property of the kernel.
-    static bool configured[64] = {};
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess) {
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        }
+    });
+    return fn;
+}
+
+// Tensor map over a cache viewed as [num_blocks * Hkv * 16 rows][D] 16-bit
+// elements, in boxes of 16 rows x 64 elements with the 128-byte swizzle.
+template <typename T>
+int encode_cache_map(CUtensorMap* map, const void* cache, int64_t rows, int D)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) {
+        pkv::record_cuda_error(cudaErrorNotSupported);
+        return PKV_ERR_CUDA;
+    }
+    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)D * sizeof(T)};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUtensorMapDataType ty =
+        sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const CUresult r = enc(map, ty, 2, const_cast<void*>(cache), gdim, gstride, box, estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        pkv::record_cuda_error(cudaErrorInvalidValue);
+        return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+// Once per device and kernel instantiation: allow more than 48 KiB of
+// dynamic shared memory.
+template <typename K>
+int allow_smem(K kernel, int bytes, bool* configured)
+{
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) {
@@ -501,23 +551,52 @@ int launch(void* out, const void* q, const void* k_cache, const void* v_cache, c
         return PKV_ERR_CUDA;
     }
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(decode_partition_kernel<T, D, G>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) {
             pkv::record_cuda_error(e);
             return PKV_ERR_CUDA;
         }
         configured[dev] = true;
     }
+    return PKV_OK;
+}
+
+template <typename T, int D, int G>
+int launch(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* bt,
+           int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
+           int32_t NB, float scale, void* ws, cudaStream_t stream, int* status)
+{
     const int max_parts = (max_ctx + kPartTokens - 1) / kPartTokens;
     float* ws_acc = static_cast<float*>(ws);
     float* ws_ml = ws_acc ? ws_acc + (size_t)S * Hq * max_parts * D : nullptr;
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
     dim3 grid((unsigned)max_parts, (unsigned)Hkv, (unsigned)S);
-    decode_partition_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
-        static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), static_cast<const T*>(k_cache),
-        static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2, max_parts, status);
-    int rc = pkv::check_launch();
+    int rc;
+    if constexpr (sizeof(T) == 2) {
+        // fp16 / bf16: tensor-core kernel fed by tiled TMA
+        using C = TcCfg<D>;
+        static bool configured[64] = {};
+        rc = allow_smem(decode_partition_tc_kernel<T, D, G>, C::kSmemBytes, configured);
+        if (rc != PKV_OK) return rc;
+        const int64_t rows = (int64_t)NB * Hkv * kBlock;
+        if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+        CUtensorMap tm_k, tm_v;
+        if ((rc = encode_cache_map<T>(&tm_k, k_cache, rows, D)) != PKV_OK) return rc;
+        if ((rc = encode_cache_map<T>(&tm_v, v_cache, rows, D)) != PKV_OK) return rc;
+        decode_partition_tc_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
+            tm_k, tm_v, static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), bt, mb, cl, max_ctx, Hq,
+            Hkv, NB, scale_log2, max_parts, status);
+    } else {
+        // fp32: CUDA-core kernel fed by 1-D bulk copies
+        using C = Cfg<T, D, G>;
+        static bool configured[64] = {};
+        rc = allow_smem(decode_partition_kernel<T, D, G>, C::kSmemBytes, configured);
+        if (rc != PKV_OK) return rc;
+        decode_partition_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
+            static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), static_cast<const T*>(k_cache),
+            static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2, max_parts, status);
+    }
+    rc = pkv::check_launch();
     if (rc != PKV_OK || max_parts == 1) return rc;
     const int64_t rows = (int64_t)S * Hq;
     decode_reduce_kernel<T, D><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(

@@ -1,0 +1,352 @@
+// Tensor-core partition kernel of paged_attention_decode for 16-bit inputs
+// (fp16 / bf16).  Included by decode.cu, which owns the launcher and the
+// split-K reduce kernel.
+//
+// Per (partition, kv head, sequence) CTA, as in the CUDA-core kernel:
+// 4 warps, each walking its share of the partition's 16-token blocks with
+// its own 2-stage pipeline of (K tile, V tile) pairs.  The differences:
+//
+//  * Tiles arrive by 2-D tiled TMA (cp.async.bulk.tensor, no multicast) from
+//    a tensor map over the cache viewed as [num_blocks * Hkv * 16][head_dim],
+//    in boxes of 16 rows x 64 elements with the 128-byte swizzle.  The swizzle
+//    makes the ldmatrix reads below free of shared-memory bank conflicts.
+//  * Q.K^T and P.V run on the tensor cores as mma.sync m16n8k16 with fp32
+//    accumulation.  The G query heads of the kv head fill rows 0..G-1 of the
+//    16-row operand; the other rows are zero.  Per 16-token block and
+//    head_dim 128: 16 MMAs for the scores (2 token tiles x 8 k-steps) and 16
+//    for P.V (16 head-dim tiles, k = the block's 16 tokens).
+//  * Q stays in registers as MMA fragments (exact 16-bit inputs, scaled
+//    after the product in fp32).  The probabilities go from the score
+//    accumulators straight into the P.V operand (rounded to the input type;
+//    the running sum uses the unrounded fp32 values).
+//  * In the sequence's last, partial block, the V operand rows of tokens past
+//    the length are zeroed, and their scores are set to -inf, so whatever
+//    the unused slots hold cannot reach the result.
+#pragma once
+
+#include <cuda.h>
+
+namespace {
+
+template <typename T>
+struct Mma;
+
+template <>
+struct Mma<__nv_bfloat16> {
+    __device__ __forceinline__ static void run(float* d, const uint32_t* a, uint32_t b0, uint32_t b1)
+    {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi)
+    {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+};
+
+template <>
+struct Mma<__half> {
+    __device__ __forceinline__ static void run(float* d, const uint32_t* a, uint32_t b0, uint32_t b1)
+    {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ __forceinline__ static uint32_t pack(float lo, float hi)
+    {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t* r, uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar,
+                                            uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+constexpr int kTcBoxBytes = 16 * 128;  // 16 rows x 64 16-bit elements
+
+template <int D>
+struct TcCfg {
+    static constexpr int kBoxes = D / 64;                     // boxes per tile
+    static constexpr int kTileBytes = kBoxes * kTcBoxBytes;   // one K (or V) tile
+    static constexpr int kStageBytes = 2 * kTileBytes;        // K then V
+    static constexpr int kKSteps = D / 16;                    // Q.K k-steps
+    static constexpr int kNTiles = D / 8;                     // P.V n-tiles
+    static constexpr int kTilesBytes = kWarps * kStages * kStageBytes;
+    static constexpr int kBarOff = kTilesBytes;
+    static constexpr int kBlkOff = kBarOff + kWarps * kStages * 8;
+    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBlkOff + kPartBlocks * 4;
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+};
+
+// Lane 0 of a warp: fetch the K and V tiles of cache rows [row, row + 16)
+// into the stage at `dst` (K boxes, then V boxes), completing on `bar`.
+template <int D>
+__device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUtensorMap* tm_k,
+                                         const CUtensorMap* tm_v, int row, uint64_t policy)
+{
+    using C = TcCfg<D>;
+    const uint32_t b = pkv::smem_addr(bar);
+    // order this warp's earlier generic reads of the stage before the async writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    pkv::mbar_arrive_expect_tx(bar, C::kStageBytes);
+#pragma unroll
+    for (int bx = 0; bx < C::kBoxes; ++bx) {
+        tma_load_2d(dst + bx * kTcBoxBytes, tm_k, bx * 64, row, b, policy);
+        tma_load_2d(dst + C::kTileBytes + bx * kTcBoxBytes, tm_v, bx * 64, row, b, policy);
+    }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kWarps * 32)
+    decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                               T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
+                               const T* __restrict__ q, const int32_t* __restrict__ block_tables, int32_t mb,
+                               const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t num_blocks, float scale_log2, int32_t max_parts,
+                               int* status)
+{
+    using C = TcCfg<D>;
+    static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
+    if (sr.bad) {
+        if (p == 0) {
+            for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+                pkv::store_out(out + ((int64_t)s * num_q_heads + h * G) * D + i, 0.0f);
+            }
+        }
+        return;
+    }
+    if (p >= sr.nparts) return;
+
+    const int nblk_seq = (sr.ctx + kBlock - 1) / kBlock;
+    const int blk0 = p * kPartBlocks;
+    const int nb = min(kPartBlocks, nblk_seq - blk0);
+    const int last_valid = sr.ctx - (nblk_seq - 1) * kBlock;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
+    int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
+    const uint32_t tiles = pkv::smem_addr(smem + warp * (kStages * C::kStageBytes));
+
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
+        if (b < 0 || b >= num_blocks) {
+            pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
+            b = 0;
+        }
+        s_blk[i] = b;
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) pkv::mbar_init(&bars[st], 1);
+        pkv::fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int nw = nb > warp ? (nb - warp + kWarps - 1) / kWarps : 0;
+    uint64_t policy = 0;
+    if (lane == 0) {
+        policy = pkv::policy_evict_first();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+    }
+
+    if (lane == 0) {
+        for (int k = 0; k < nw && k < kStages; ++k) {
+            tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], &tm_k, &tm_v,
+                        (s_blk[warp + k * kWarps] * num_kv_heads + h) * kBlock, policy);
+        }
+    }
+
+    // ---- Q as A fragments: row g = lane / 4 (zero for g >= G and rows 8..15)
+    const int g_row = lane >> 2;
+    const int qd = 2 * (lane & 3);
+    uint32_t qa[C::kKSteps][4];
+#pragma unroll
+    for (int ks = 0; ks < C::kKSteps; ++ks) {
+        qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
+        if (g_row < G) {
+            const T* qrow = q + ((int64_t)s * num_q_heads + h * G + g_row) * D + 16 * ks + qd;
+            qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
+            qa[ks][2] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+        }
+    }
+
+    // ---- per-lane ldmatrix addressing (128-byte swizzle: chunk c of row r is at c ^ (r % 8))
+    const int mi = lane >> 3, r8 = lane & 7;
+    // K (non-transposed): matrix mi -> tokens (mi / 2) * 8 + r8, 16-byte chunk 2 * ks + (mi % 2)
+    const uint32_t k_row_off = (uint32_t)(((mi >> 1) * 8 + r8) * 128);
+    const uint32_t k_x = (uint32_t)(((mi & 1) ^ r8) << 4);
+    // V (transposed): matrix mi -> tokens (mi % 2) * 8 + r8, chunk 2 * j + (mi / 2)
+    const uint32_t v_row_off = (uint32_t)(((mi & 1) * 8 + r8) * 128);
+    const uint32_t v_x = (uint32_t)(((mi >> 1) ^ r8) << 4);
+
+    float o[C::kNTiles][4];
+#pragma unroll
+    for (int n = 0; n < C::kNTiles; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
+    float m_run = -INFINITY, l_part = 0.0f;
+    bool timed_out = false;
+    int consumed = 0;
+
+    for (int k = 0; k < nw; ++k) {
+        const int st = k % kStages;
+        if (!pkv::mbar_wait(&bars[st], (k / kStages) & 1, kWaitLimitNs)) {
+            timed_out = true;
+            break;
+        }
+        const uint32_t kbase = tiles + st * C::kStageBytes;
+        const uint32_t vbase = kbase + C::kTileBytes;
+        const int valid = (blk0 + warp + k * kWarps == nblk_seq - 1) ? last_valid : kBlock;
+
+        // ---- S = Q K^T for the block's 16 tokens (two 8-token tiles)
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < C::kKSteps; ++ks) {
+            uint32_t b[4];
+            const uint32_t addr = kbase + (ks / 4) * kTcBoxBytes + k_row_off + (((uint32_t)(2 * (ks % 4)) << 4) ^ k_x);
+            ldsm_x4(b, addr);
+            Mma<T>::run(s0, qa[ks], b[0], b[1]);
+            Mma<T>::run(s1, qa[ks], b[2], b[3]);
+        }
+
+        // ---- online softmax on row g_row; this lane holds tokens qd, qd+1, qd+8, qd+9
+        float x[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
+        if (valid < kBlock) {
+            if (qd >= valid) x[0] = -INFINITY;
+            if (qd + 1 >= valid) x[1] = -INFINITY;
+            if (qd + 8 >= valid) x[2] = -INFINITY;
+            if (qd + 9 >= valid) x[3] = -INFINITY;
+        }
+        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m_run, mx);
+        const float alpha = pkv::fast_exp2(m_run - mn);
+        float pr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[i] = pkv::fast_exp2(x[i] - mn);
+        l_part = l_part * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+        if (__any_sync(0xffffffffu, mn != m_run)) {
+#pragma unroll
+            for (int n = 0; n < C::kNTiles; ++n) {
+                o[n][0] *= alpha;
+                o[n][1] *= alpha;
+            }
+        }
+        m_run = mn;
+        const uint32_t pa[4] = {Mma<T>::pack(pr[0], pr[1]), 0u, Mma<T>::pack(pr[2], pr[3]), 0u};
+
+        // ---- O += P V over the head dimension (pairs of 8-wide tiles)
+        uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // V rows qd, qd+1 / qd+8, qd+9
+        if (valid < kBlock) {
+            keep_lo = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
+            keep_hi = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < C::kNTiles / 2; ++j) {
+            uint32_t b[4];
+            const uint32_t addr = vbase + (j / 4) * kTcBoxBytes + v_row_off + (((uint32_t)(2 * (j % 4)) << 4) ^ v_x);
+            ldsm_x4_trans(b, addr);
+            b[0] &= keep_lo;
+            b[1] &= keep_hi;
+            b[2] &= keep_lo;
+            b[3] &= keep_hi;
+            Mma<T>::run(o[2 * j], pa, b[0], b[1]);
+            Mma<T>::run(o[2 * j + 1], pa, b[2], b[3]);
+        }
+        __syncwarp();
+        ++consumed;
+        if (lane == 0 && k + kStages < nw) {
+            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v, (s_blk[warp + (k + kStages) * kWarps] * num_kv_heads + h) * kBlock,
+                        policy);
+        }
+    }
+
+    if (timed_out) {
+        if (lane == 0) pkv::raise_flag(status, PKV_DEV_WAIT_TIMEOUT);
+        for (int k = consumed; k < nw && k < consumed + kStages; ++k) {
+            pkv::mbar_wait(&bars[k % kStages], (k / kStages) & 1, kWaitLimitNs);
+        }
+    }
+
+    // ---- merge the warps: lane (g_row, qd) holds O[g_row][8n + qd .. +1]
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    __syncthreads();
+    float* mg = reinterpret_cast<float*>(smem);  // [kWarps][G][D + 2]: m, l, acc[D]
+    if (g_row < G) {
+        float* rec = mg + (warp * G + g_row) * (D + 2);
+        if ((lane & 3) == 0) {
+            rec[0] = m_run;
+            rec[1] = l_part;
+        }
+#pragma unroll
+        for (int n = 0; n < C::kNTiles; ++n) {
+            rec[2 + 8 * n + qd] = o[n][0];
+            rec[2 + 8 * n + qd + 1] = o[n][1];
+        }
+    }
+    __syncthreads();
+
+    const int hq0 = h * G;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+        const int g = i / D, d = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[(w * G + g) * (D + 2)]);
+        float L = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float* rec = mg + (w * G + g) * (D + 2);
+            const float wgt = exp2f(rec[0] - M);
+            L = fmaf(rec[1], wgt, L);
+            O = fmaf(rec[2 + d], wgt, O);
+        }
+        const int64_t row = (int64_t)s * num_q_heads + hq0 + g;
+        if (sr.nparts == 1) {
+            pkv::store_out(out + row * D + d, O / L);
+        } else {
+            ws_acc[(row * max_parts + p) * D + d] = O;
+            if (d == 0) {
+                ws_ml[(row * max_parts + p) * 2] = M;
+                ws_ml[(row * max_parts + p) * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+}  // namespace

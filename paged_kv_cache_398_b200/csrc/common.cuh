@@ -37,7 +37,37 @@ inline size_t dtype_bytes(int32_t dtype)
     return dtype == PKV_F32 ? 4 : (dtype == PKV_F16 || dtype == PKV_BF16) ? 2 : 0;
 }
 
+// Launch configuration whose kernel may be staged while the previous kernel
+// on the stream finishes (programmatic dependent launch).  The kernel must
+// call grid_dependency_wait() before it reads anything a previous kernel may
+// have written.  After a non-kernel stream operation the launch simply
+// waits, as an ordinary one would.
+inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return cfg;
+}
+
+inline void pdl_attribute(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr)
+{
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg->attrs = attr;
+    cfg->numAttrs = 1;
+}
+
 // ---- device side ---------------------------------------------------------
+
+// Wait until the grids this one depends on have completed and their memory
+// is visible (a no-op when the kernel was not launched as a dependent).
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 __device__ __forceinline__ void raise_flag(int* status, int flag)
 {

@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 {
     using C = Cfg<T, D, G>;
     extern __shared__ __align__(128) uint8_t smem[];
+    pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -438,7 +439,9 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // Merge the partitions of every (sequence, query head) that has more than
 // one: out = sum_p acc_p 2^(m_p - M) / sum_p l_p 2^(m_p - M), M = max_p m_p,
-// in partition order.  One warp per (sequence, query head).
+// in partition order.  One warp per (sequence, query head); each lane owns
+// head_dim / 32 consecutive outputs and issues the vector loads of up to 8
+// partitions before it consumes them.
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
     decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
@@ -447,6 +450,9 @@ __global__ void __launch_bounds__(128)
                          int32_t max_parts)
 {
     constexpr int kPer = D / 32;
+    using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
+    constexpr int kUnroll = 8;
+    pkv::grid_dependency_wait();  // the partition kernel's results are visible after this
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= (int64_t)num_seqs * num_q_heads) return;
@@ -454,7 +460,8 @@ __global__ void __launch_bounds__(128)
     const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, false, nullptr);
     if (sr.bad || sr.nparts <= 1) return;
     const float* ml = ws_ml + row * max_parts * 2;
-    const float* acc = ws_acc + row * max_parts * D;
+    const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
+    constexpr int kStride = D / kPer;  // Vec elements per partition
 
     float M = -INFINITY;
     for (int p0 = 0; p0 < sr.nparts; p0 += 32) {
@@ -476,12 +483,22 @@ __global__ void __launch_bounds__(128)
             lw = ml[pp * 2 + 1] * w;
         }
         const int n = min(32, sr.nparts - p0);
-        for (int j = 0; j < n; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, w, j);
-            L += __shfl_sync(0xffffffffu, lw, j);
-            const float* a = acc + (int64_t)(p0 + j) * D + lane * kPer;
+        for (int j0 = 0; j0 < n; j0 += kUnroll) {
+            Vec a[kUnroll];
 #pragma unroll
-            for (int e = 0; e < kPer; ++e) o[e] = fmaf(a[e], wj, o[e]);
+            for (int u = 0; u < kUnroll; ++u) {
+                if (j0 + u < n) a[u] = acc[(int64_t)(p0 + j0 + u) * kStride];
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (j0 + u < n) {  // warp-uniform
+                    const float wj = __shfl_sync(0xffffffffu, w, j0 + u);
+                    L += __shfl_sync(0xffffffffu, lw, j0 + u);
+                    const float* av = reinterpret_cast<const float*>(&a[u]);
+#pragma unroll
+                    for (int e = 0; e < kPer; ++e) o[e] = fmaf(av[e], wj, o[e]);
+                }
+            }
         }
     }
     const float inv = 1.0f / L;
@@ -572,6 +589,7 @@ int launch(void* out, const void* q, const void* k_cache, const void* v_cache, c
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
     dim3 grid((unsigned)max_parts, (unsigned)Hkv, (unsigned)S);
     int rc;
+    cudaError_t launch_err = cudaSuccess;
     if constexpr (sizeof(T) == 2) {
         // fp16 / bf16: tensor-core kernel fed by tiled TMA
         using C = TcCfg<D>;
@@ -583,24 +601,42 @@ int launch(void* out, const void* q, const void* k_cache, const void* v_cache, c
         CUtensorMap tm_k, tm_v;
         if ((rc = encode_cache_map<T>(&tm_k, k_cache, rows, D)) != PKV_OK) return rc;
         if ((rc = encode_cache_map<T>(&tm_v, v_cache, rows, D)) != PKV_OK) return rc;
-        decode_partition_tc_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
-            tm_k, tm_v, static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), bt, mb, cl, max_ctx, Hq,
-            Hkv, NB, scale_log2, max_parts, status);
+        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, stream);
+        cudaLaunchAttribute attr[1];
+        pkv::pdl_attribute(&cfg, attr);
+        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_tc_kernel<T, D, G>, tm_k, tm_v, static_cast<T*>(out), ws_acc,
+                           ws_ml, static_cast<const T*>(q), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2,
+                           max_parts, status);
     } else {
         // fp32: CUDA-core kernel fed by 1-D bulk copies
         using C = Cfg<T, D, G>;
         static bool configured[64] = {};
         rc = allow_smem(decode_partition_kernel<T, D, G>, C::kSmemBytes, configured);
         if (rc != PKV_OK) return rc;
-        decode_partition_kernel<T, D, G><<<grid, kWarps * 32, C::kSmemBytes, stream>>>(
-            static_cast<T*>(out), ws_acc, ws_ml, static_cast<const T*>(q), static_cast<const T*>(k_cache),
-            static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2, max_parts, status);
+        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, stream);
+        cudaLaunchAttribute attr[1];
+        pkv::pdl_attribute(&cfg, attr);
+        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_kernel<T, D, G>, static_cast<T*>(out), ws_acc, ws_ml,
+                           static_cast<const T*>(q), static_cast<const T*>(k_cache),
+                           static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2,
+                           max_parts, status);
+    }
+    if (launch_err != cudaSuccess) {
+        pkv::record_cuda_error(launch_err);
+        return PKV_ERR_CUDA;
     }
     rc = pkv::check_launch();
     if (rc != PKV_OK || max_parts == 1) return rc;
     const int64_t rows = (int64_t)S * Hq;
-    decode_reduce_kernel<T, D><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(
-        static_cast<T*>(out), ws_acc, ws_ml, cl, S, Hq, mb, max_ctx, max_parts);
+    cudaLaunchConfig_t cfg = pkv::pdl_config(dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream);
+    cudaLaunchAttribute attr[1];
+    pkv::pdl_attribute(&cfg, attr);
+    const cudaError_t reduce_err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<T, D>, static_cast<T*>(out), (const float*)ws_acc,
+                       (const float*)ws_ml, cl, S, Hq, mb, max_ctx, max_parts);
+    if (reduce_err != cudaSuccess) {
+        pkv::record_cuda_error(reduce_err);
+        return PKV_ERR_CUDA;
+    }
     return pkv::check_launch();
 }
 

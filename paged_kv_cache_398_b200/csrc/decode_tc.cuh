@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 

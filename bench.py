@@ -44,6 +44,35 @@ WORKLOAD_NAMES = {2: "7b", 3: "13b", 4: "8b_gqa_prefix", 5: "8b_gqa_sampling"}
 FALLBACK_HBM_GBS = 6650.0
 
 
+DECODE_SOURCES = ("paged_kv_cache_398_b200/csrc/decode.cu", "paged_kv_cache_398_b200/csrc/decode_tc.cuh",
+                  "paged_kv_cache_398_b200/csrc/common.cuh")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def decode_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str, num_seqs: int):
+    """DRAM bytes per decode call from the committed ncu record, or None if
+    there is none for this workload or the decode sources changed since."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != decode_source_hash():
+        return None
+    if rec.get("workload") != workload or rec.get("num_seqs") != num_seqs:
+        return None
+    return rec.get("dram_bytes_per_call")
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -452,7 +481,8 @@ def run_ours(args):
                       "write_and_copy_mean": ms_max / args.steps - dec_mean},
         "roofline": {"kernel": "paged_attention_decode (partition kernel + split-K reduce)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S),
                      "algorithmic_bytes_per_launch": st.decode_bytes},
         "cpu_baseline": ({k: v for k, v in base.items() if k != "seconds"} if base else None),
         "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",

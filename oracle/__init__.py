@@ -64,6 +64,9 @@ def lib():
             L.oracle_paged_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32,
                                               D, ctypes.c_int]
             L.oracle_paged_decode.restype = ctypes.c_int
+            L.oracle_paged_decode_mq.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
+                                                 D, ctypes.c_int]
+            L.oracle_paged_decode_mq.restype = ctypes.c_int
             L.oracle_kv_write.argtypes = [P, P, P, P, P, I32, I32, I32, I32, I32, ctypes.c_int]
             L.oracle_kv_write.restype = ctypes.c_int
             L.oracle_block_copy.argtypes = [P, P, P, I32, I32, I32, I32, I32, ctypes.c_int]
@@ -154,6 +157,30 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float) 
                                    float(scale), _code(q))
     if rc != 0:
         raise OracleError("paged_decode: invalid input")
+    return out
+
+
+def paged_decode_mq(q, k_cache, v_cache, block_tables, context_lens, scale: float) -> np.ndarray:
+    """fp64 multi-query decode: q [S, q_len, Hq, D] -> [S, q_len, Hq, D].
+
+    New token j of sequence s is at position ctx_s - q_len + j and attends
+    to positions 0 .. ctx_s - q_len + j (causal among the new tokens).
+    """
+    _cpu(q), _cpu(k_cache), _cpu(v_cache)
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise OracleError("q and the caches must share one dtype")
+    bt = _cpu(block_tables, torch.int32)
+    cl = _cpu(context_lens, torch.int32)
+    S, QL, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if D2 != D:
+        raise OracleError("head_dim mismatch")
+    out = np.empty((S, QL, Hq, D), np.float64)
+    rc = lib().oracle_paged_decode_mq(out.ctypes.data, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      bt.data_ptr(), bt.shape[1], cl.data_ptr(), S, QL, Hq, Hkv, D, B, NB,
+                                      float(scale), _code(q))
+    if rc != 0:
+        raise OracleError("paged_decode_mq: invalid input")
     return out
 
 

@@ -237,6 +237,49 @@ int oracle_paged_decode(double* out, const void* q, const void* k_cache, const v
 }
 
 /*
+ * Multi-query decode: each sequence brings q_len new tokens (for example
+ * draft tokens to verify), already counted in context_lens.  New token j
+ * (0-based) sits at position ctx - q_len + j and, as in any causal decoder,
+ * attends to every token up to and including its own position, i.e. to the
+ * first ctx - q_len + j + 1 tokens.  q and out are
+ * [num_seqs][q_len][num_q_heads][head_dim].  With q_len = 1 this is
+ * oracle_paged_decode.  (Speculative decoding, "PagedAttention & Continuous
+ * Batching: How vLLM Achieves 24x Serving Throughput", item 7: the target
+ * model checks several proposed tokens in one pass.)
+ * Returns -1 if some ctx < q_len or on any error of the single-query form.
+ */
+int oracle_paged_decode_mq(double* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t q_len,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, double scale, int dtype)
+{
+    size_t eb = elem_bytes(dtype);
+    if (q_len < 1) {
+        return -1;
+    }
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t ctx = context_lens[s];
+        if (ctx < q_len) {
+            return -1;
+        }
+        for (int32_t j = 0; j < q_len; ++j) {
+            int64_t row = (int64_t)s * q_len + j;
+            const char* q_row = (const char*)q + (size_t)row * num_q_heads * head_dim * eb;
+            int rc = oracle_paged_decode_seq(out + row * num_q_heads * head_dim, q_row, k_cache,
+                                             v_cache, block_tables + (int64_t)s * max_blocks_per_seq,
+                                             max_blocks_per_seq, ctx - q_len + j + 1, num_q_heads,
+                                             num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                             dtype);
+            if (rc != 0) {
+                return rc;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
  * Slot write: for token t with slot = slot_mapping[t] >= 0, store its key and
  * value rows (every kv head) at physical block slot / block_size, offset
  * slot % block_size.  A negative slot means "no write" (padding token).

@@ -146,6 +146,52 @@ def test_attention_equals_sdpa_on_contiguous_blocks():
     check_sdpa_contiguous()
 
 
+def check_multi_query_causal_sdpa():
+    for ctx, QL, Hq, Hkv, D, dtype in [(20, 3, 4, 2, 16, torch.float32), (33, 4, 8, 2, 8, torch.bfloat16),
+                                       (5, 5, 2, 1, 8, torch.float16), (48, 1, 4, 4, 16, torch.float32)]:
+        g = torch.Generator().manual_seed(ctx * 7 + QL)
+        q, kc, vc, bt, cl, K, V = _contiguous_case(ctx, Hq, Hkv, D, dtype, seed=ctx + QL)
+        qm = torch.randn(1, QL, Hq, D, generator=g).to(dtype)
+        scale = 0.7 / math.sqrt(D)
+        got = oracle.paged_decode_mq(qm, kc, vc, bt, cl, scale)[0]            # [QL, Hq, D]
+        # query j sits at position ctx - QL + j and may see keys 0..ctx - QL + j
+        allowed = torch.arange(ctx)[None, :] <= (ctx - QL + torch.arange(QL))[:, None]
+        qq = qm.to(torch.float64)[0].permute(1, 0, 2).reshape(1, Hq, QL, D)
+        KK = K.to(torch.float64).permute(1, 0, 2).reshape(1, Hkv, ctx, D)
+        VV = V.to(torch.float64).permute(1, 0, 2).reshape(1, Hkv, ctx, D)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            qq, KK, VV, attn_mask=allowed, scale=scale, enable_gqa=True)[0].permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    # a batch of two sequences in one pool: each row must match its own sequence
+    QL, Hq, Hkv, D = 3, 4, 2, 8
+    g = torch.Generator().manual_seed(5)
+    ctxs, starts = (20, 35), (0, 2)
+    kc = torch.randn(5, Hkv, B, D, generator=g)
+    vc = torch.randn(5, Hkv, B, D, generator=g)
+    bt = torch.tensor([[0, 1, -1], [2, 3, 4]], dtype=torch.int32)
+    cl = torch.tensor(ctxs, dtype=torch.int32)
+    qm = torch.randn(2, QL, Hq, D, generator=g)
+    got = oracle.paged_decode_mq(qm, kc, vc, bt, cl, 0.4)
+    for sq, (ctx, b0) in enumerate(zip(ctxs, starts)):
+        nb = -(-ctx // B)
+        K = kc[b0:b0 + nb].permute(1, 0, 2, 3).reshape(1, Hkv, nb * B, D)[:, :, :ctx].double()
+        V = vc[b0:b0 + nb].permute(1, 0, 2, 3).reshape(1, Hkv, nb * B, D)[:, :, :ctx].double()
+        allowed = torch.arange(ctx)[None, :] <= (ctx - QL + torch.arange(QL))[:, None]
+        qq = qm[sq].double().permute(1, 0, 2).reshape(1, Hq, QL, D)
+        want = torch.nn.functional.scaled_dot_product_attention(
+            qq, K, V, attn_mask=allowed, scale=0.4, enable_gqa=True)[0].permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(got[sq], want, rtol=1e-12, atol=1e-12)
+    # q_len = 1 is the single-query decode, exactly
+    q, kc, vc, bt, cl, K, V = _contiguous_case(30, 4, 2, 16, torch.float32, seed=99)
+    a = oracle.paged_decode(q, kc, vc, bt, cl, 0.3)
+    b = oracle.paged_decode_mq(q.reshape(1, 1, 4, 16).contiguous(), kc, vc, bt, cl, 0.3)
+    np.testing.assert_array_equal(a, b[:, 0])
+
+
+def test_multi_query_decode_equals_causal_sdpa():
+    check_multi_query_causal_sdpa()
+
+
 def check_single_token_is_its_value():
     q, kc, vc, bt, cl, K, V = _contiguous_case(1, 4, 4, 64, torch.float32, seed=1)
     got = oracle.paged_decode(q, kc, vc, bt, cl, 0.125)[0]
@@ -379,7 +425,8 @@ def test_block_copy_rejects_order_dependent_lists():
 # --------------------------------------------------------------------------
 # planted mistakes must be caught
 # --------------------------------------------------------------------------
-QUICK_CHECKS = [check_worked_example_gather, check_sdpa_contiguous, check_single_token_is_its_value,
+QUICK_CHECKS = [check_worked_example_gather, check_sdpa_contiguous, check_multi_query_causal_sdpa,
+                check_single_token_is_its_value,
                 check_uniform_scores_give_mean, check_dominant_key, check_gqa_grouping,
                 check_placement_invariance, check_shared_equals_duplicated,
                 check_write_roundtrip_worked_tables, check_write_touches_only_its_slot,
@@ -397,6 +444,8 @@ MUTANTS = [
     ("for (int32_t i = h * group; rc == 0 && i < (h + 1) * group; ++i)",
      "for (int32_t i = h; rc == 0 && i < num_q_heads; i += num_kv_heads)"),
     ("int64_t off = slot % block_size;", "int64_t off = slot / block_size;"),
+    ("max_blocks_per_seq, ctx - q_len + j + 1, num_q_heads,", "max_blocks_per_seq, ctx - q_len + j, num_q_heads,"),
+    ("int64_t row = (int64_t)s * q_len + j;", "int64_t row = (int64_t)j * num_seqs + s;"),
     ("memcpy((char*)v_cache + (size_t)dst * block_bytes,", "memcpy((char*)v_cache + (size_t)src * block_bytes,"),
     ("v = ldexp((double)(f + 1024), e - 25);", "v = ldexp((double)(f + 1024), e - 24);"),
     ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = (uint32_t)b << 15;"),
@@ -422,8 +471,8 @@ def test_mutants_are_caught(monkeypatch):
             assert src.count(old) == 1, f"mutant {i}: pattern not unique in oracle.c: {old}"
             so = _load_mutant(src.replace(old, new), td, i)
             L = ctypes.CDLL(so)
-            for name in ("oracle_widen", "oracle_gather", "oracle_paged_decode_seq",
-                         "oracle_paged_decode", "oracle_kv_write", "oracle_block_copy"):
+            for name in ("oracle_widen", "oracle_gather", "oracle_paged_decode_seq", "oracle_paged_decode",
+                         "oracle_paged_decode_mq", "oracle_kv_write", "oracle_block_copy"):
                 fn, ref = getattr(L, name), getattr(good, name)
                 fn.argtypes, fn.restype = ref.argtypes, ref.restype
             monkeypatch.setattr(oracle, "_lib", L)

@@ -154,6 +154,51 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * paged_attention_decode_mq -- decode attention for q_len >= 1 new tokens per
+ * sequence, optionally fused with their slot write.  Typical uses are
+ * checking a draft model's proposed tokens in one pass (speculative
+ * decoding: "PagedAttention & Continuous Batching: How vLLM Achieves 24x
+ * Serving Throughput", item 7), and the single-token decode step with its
+ * cache write in the same launch.
+ *
+ * context_lens[s] counts the new tokens.  New token j (0-based) sits at
+ * position ctx - q_len + j and attends causally to positions
+ * 0 .. ctx - q_len + j, so
+ *
+ *   out[s][j][i][:] = sum_{t <= ctx-q_len+j} softmax_t(scale * q[s][j][i] . K_s[t]) * V_s[t]
+ *
+ *  out, q         device, [num_seqs][q_len][num_q_heads][head_dim], dtype
+ *  k_new, v_new   device, [num_seqs][q_len][num_kv_heads][head_dim], or
+ *                 both NULL.  When given, the call first stores the new
+ *                 tokens' rows in their slots, reached through block_tables
+ *                 (the same bytes paged_kv_write would store), and attends
+ *                 to them in the same launch.  When NULL, the caller must
+ *                 already have written them.  The written blocks must not be
+ *                 shared (the allocator's copy-on-write guarantees this).
+ *  k_cache, v_cache  device, cache layout above; written only when k_new is
+ *                 given.
+ *  workspace      >= paged_attention_mq_workspace_bytes(...) bytes, 256-byte
+ *                 aligned, or NULL when that size is 0.
+ *  A context length below q_len raises PKV_DEV_BAD_CONTEXT and zeroes that
+ *  sequence's output rows.  All other arguments and checks are as in
+ *  paged_attention_decode.
+ *  Limits: q_len * (num_q_heads / num_kv_heads) <= 16, because the query
+ *  rows of one kv head fill one 16-row tensor-core operand.  fp32 supports
+ *  only q_len == 1 without a fused write (PKV_ERR_UNSUPPORTED otherwise).
+ * With q_len == 1 and no fused write, the result equals
+ * paged_attention_decode bit for bit.
+ */
+size_t paged_attention_mq_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                          int32_t head_dim, int32_t max_context_len);
+int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const void* v_new,
+                              void* k_cache, void* v_cache, const int32_t* block_tables,
+                              int32_t max_blocks_per_seq, const int32_t* context_lens,
+                              int32_t num_seqs, int32_t q_len, int32_t max_context_len,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * paged_attention_decode_noalloc -- paged_attention_decode without a
  * caller-supplied workspace, for callers that cannot allocate device memory
  * when they decode.  Examples: code that runs while a stream is being

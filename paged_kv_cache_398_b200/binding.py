@@ -111,6 +111,55 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def paged_attention_mq_workspace_bytes(num_seqs: int, q_len: int, num_q_heads: int, head_dim: int,
+                                       max_context_len: int) -> int:
+    return int(lib().paged_attention_mq_workspace_bytes(num_seqs, q_len, num_q_heads, head_dim, max_context_len))
+
+
+def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                              max_context_len: int, k_new=None, v_new=None,
+                              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode for q [S, q_len, Hq, D] new tokens per sequence, causal among them.
+
+    With k_new / v_new [S, q_len, Hkv, D] the new tokens are written to their
+    slots (through the block tables) in the same launch.  Returns `out`
+    [S, q_len, Hq, D].
+    """
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    _cuda("q", q, k_cache.dtype, 4)
+    _cuda("out", out, k_cache.dtype, 4)
+    _cuda("block_tables", block_tables, torch.int32, 2)
+    _cuda("context_lens", context_lens, torch.int32, 1)
+    S, QL, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (S, QL, Hq, D):
+        raise ValueError("q/out must be [S, q_len, Hq, D] with the cache's head_dim")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables/context_lens must have one row per sequence")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    kn = vn = None
+    if k_new is not None:
+        _cuda("k_new", k_new, k_cache.dtype, 4)
+        _cuda("v_new", v_new, k_cache.dtype, 4)
+        if tuple(k_new.shape) != (S, QL, Hkv, D) or tuple(v_new.shape) != (S, QL, Hkv, D):
+            raise ValueError("k_new/v_new must be [S, q_len, Hkv, D]")
+        kn, vn = k_new.data_ptr(), v_new.data_ptr()
+    need = paged_attention_mq_workspace_bytes(S, QL, Hq, D, max_context_len)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = 0, 0
+    if workspace is not None:
+        _cuda("workspace", workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    rc = lib().paged_attention_decode_mq(out.data_ptr(), q.data_ptr(), kn, vn, k_cache.data_ptr(),
+                                         v_cache.data_ptr(), block_tables.data_ptr(), block_tables.shape[1],
+                                         context_lens.data_ptr(), S, QL, int(max_context_len), Hq, Hkv, D, B, NB,
+                                         float(scale), _dtype_code(k_cache), ws_ptr or None, ws_bytes,
+                                         _stream(q.device, stream))
+    check("paged_attention_decode_mq", rc)
+    return out
+
+
 def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
                                    max_context_len: int, stream=None) -> torch.Tensor:
     """paged_attention_decode with the library's fixed scratch array instead

@@ -446,7 +446,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128)
     decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
                          const float* __restrict__ ws_ml, const int32_t* __restrict__ context_lens,
-                         int32_t num_seqs, int32_t num_q_heads, int32_t mb, int32_t max_ctx,
+                         int32_t num_seqs, int32_t q_len, int32_t num_q_heads, int32_t mb, int32_t max_ctx,
                          int32_t max_parts)
 {
     constexpr int kPer = D / 32;
@@ -455,10 +455,10 @@ __global__ void __launch_bounds__(128)
     pkv::grid_dependency_wait();  // the partition kernel's results are visible after this
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (row >= (int64_t)num_seqs * num_q_heads) return;
-    const int s = (int)(row / num_q_heads);
+    if (row >= (int64_t)num_seqs * q_len * num_q_heads) return;   // row = (s * q_len + j) * Hq + i
+    const int s = (int)(row / ((int64_t)q_len * num_q_heads));
     const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, false, nullptr);
-    if (sr.bad || sr.nparts <= 1) return;
+    if (sr.bad || sr.ctx < q_len || sr.nparts <= 1) return;   // zero rows / single partition: written
     const float* ml = ws_ml + row * max_parts * 2;
     const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
     constexpr int kStride = D / kPer;  // Vec elements per partition
@@ -578,48 +578,82 @@ int allow_smem(K kernel, int bytes, bool* configured)
     return PKV_OK;
 }
 
+struct DecodeArgs {
+    void* out;
+    const void* q;
+    const void* k_new;  // fused slot write: [S][q_len][Hkv][D], or null
+    const void* v_new;
+    void* k_cache;
+    void* v_cache;
+    const int32_t* bt;
+    int32_t mb;
+    const int32_t* cl;
+    int32_t S;
+    int32_t q_len;
+    int32_t max_ctx;
+    int32_t Hq;
+    int32_t Hkv;
+    int32_t NB;
+    float scale;
+    void* ws;
+    cudaStream_t stream;
+    int* status;
+};
+
 template <typename T, int D, int G>
-int launch(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* bt,
-           int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
-           int32_t NB, float scale, void* ws, cudaStream_t stream, int* status)
+int launch(const DecodeArgs& a)
 {
-    const int max_parts = (max_ctx + kPartTokens - 1) / kPartTokens;
-    float* ws_acc = static_cast<float*>(ws);
-    float* ws_ml = ws_acc ? ws_acc + (size_t)S * Hq * max_parts * D : nullptr;
-    const float scale_log2 = (float)((double)scale * 1.4426950408889634);
-    dim3 grid((unsigned)max_parts, (unsigned)Hkv, (unsigned)S);
+    const int max_parts = (a.max_ctx + kPartTokens - 1) / kPartTokens;
+    const int64_t qrows = (int64_t)a.S * a.q_len * a.Hq;  // (sequence, new token, query head) rows
+    float* ws_acc = static_cast<float*>(a.ws);
+    float* ws_ml = ws_acc ? ws_acc + (size_t)qrows * max_parts * D : nullptr;
+    const float scale_log2 = (float)((double)a.scale * 1.4426950408889634);
+    dim3 grid((unsigned)max_parts, (unsigned)a.Hkv, (unsigned)a.S);
     int rc;
     cudaError_t launch_err = cudaSuccess;
     if constexpr (sizeof(T) == 2) {
         // fp16 / bf16: tensor-core kernel fed by tiled TMA
         using C = TcCfg<D>;
-        static bool configured[64] = {};
-        rc = allow_smem(decode_partition_tc_kernel<T, D, G>, C::kSmemBytes, configured);
-        if (rc != PKV_OK) return rc;
-        const int64_t rows = (int64_t)NB * Hkv * kBlock;
+        const int64_t rows = (int64_t)a.NB * a.Hkv * kBlock;
         if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
         CUtensorMap tm_k, tm_v;
-        if ((rc = encode_cache_map<T>(&tm_k, k_cache, rows, D)) != PKV_OK) return rc;
-        if ((rc = encode_cache_map<T>(&tm_v, v_cache, rows, D)) != PKV_OK) return rc;
-        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, stream);
+        if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D)) != PKV_OK) return rc;
+        if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D)) != PKV_OK) return rc;
+        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
-        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_tc_kernel<T, D, G>, tm_k, tm_v, static_cast<T*>(out), ws_acc,
-                           ws_ml, static_cast<const T*>(q), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2,
-                           max_parts, status);
+        auto args = [&](auto kernel) {
+            return cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, static_cast<T*>(a.out), ws_acc, ws_ml,
+                                      static_cast<const T*>(a.q), static_cast<const T*>(a.k_new),
+                                      static_cast<const T*>(a.v_new), static_cast<T*>(a.k_cache),
+                                      static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.q_len, a.Hq, a.Hkv,
+                                      a.NB, scale_log2, max_parts, a.status);
+        };
+        if (a.q_len > 1) {
+            static bool configured[64] = {};
+            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, true>, C::kSmemBytes, configured)) != PKV_OK)
+                return rc;
+            launch_err = args(decode_partition_tc_kernel<T, D, G, true>);
+        } else {
+            static bool configured[64] = {};
+            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, false>, C::kSmemBytes, configured)) != PKV_OK)
+                return rc;
+            launch_err = args(decode_partition_tc_kernel<T, D, G, false>);
+        }
     } else {
-        // fp32: CUDA-core kernel fed by 1-D bulk copies
+        // fp32: CUDA-core kernel fed by 1-D bulk copies (one query, no fused write)
+        if (a.q_len != 1 || a.k_new) return PKV_ERR_UNSUPPORTED;
         using C = Cfg<T, D, G>;
         static bool configured[64] = {};
         rc = allow_smem(decode_partition_kernel<T, D, G>, C::kSmemBytes, configured);
         if (rc != PKV_OK) return rc;
-        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, stream);
+        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
-        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_kernel<T, D, G>, static_cast<T*>(out), ws_acc, ws_ml,
-                           static_cast<const T*>(q), static_cast<const T*>(k_cache),
-                           static_cast<const T*>(v_cache), bt, mb, cl, max_ctx, Hq, Hkv, NB, scale_log2,
-                           max_parts, status);
+        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_kernel<T, D, G>, static_cast<T*>(a.out), ws_acc,
+                                        ws_ml, static_cast<const T*>(a.q), static_cast<const T*>(a.k_cache),
+                                        static_cast<const T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.Hq,
+                                        a.Hkv, a.NB, scale_log2, max_parts, a.status);
     }
     if (launch_err != cudaSuccess) {
         pkv::record_cuda_error(launch_err);
@@ -627,12 +661,12 @@ int launch(void* out, const void* q, const void* k_cache, const void* v_cache, c
     }
     rc = pkv::check_launch();
     if (rc != PKV_OK || max_parts == 1) return rc;
-    const int64_t rows = (int64_t)S * Hq;
-    cudaLaunchConfig_t cfg = pkv::pdl_config(dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream);
+    cudaLaunchConfig_t cfg = pkv::pdl_config(dim3((unsigned)((qrows + 3) / 4)), dim3(128), 0, a.stream);
     cudaLaunchAttribute attr[1];
     pkv::pdl_attribute(&cfg, attr);
-    const cudaError_t reduce_err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<T, D>, static_cast<T*>(out), (const float*)ws_acc,
-                       (const float*)ws_ml, cl, S, Hq, mb, max_ctx, max_parts);
+    const cudaError_t reduce_err =
+        cudaLaunchKernelEx(&cfg, decode_reduce_kernel<T, D>, static_cast<T*>(a.out), (const float*)ws_acc,
+                           (const float*)ws_ml, a.cl, a.S, a.q_len, a.Hq, a.mb, a.max_ctx, max_parts);
     if (reduce_err != cudaSuccess) {
         pkv::record_cuda_error(reduce_err);
         return PKV_ERR_CUDA;
@@ -641,38 +675,80 @@ int launch(void* out, const void* q, const void* k_cache, const void* v_cache, c
 }
 
 template <typename T, int D>
-int dispatch_g(int G, void* out, const void* q, const void* kc, const void* vc, const int32_t* bt,
-               int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
-               int32_t NB, float scale, void* ws, cudaStream_t st, int* status)
+int dispatch_g(int G, const DecodeArgs& a)
 {
     switch (G) {
-        case 1: return launch<T, D, 1>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
-        case 2: return launch<T, D, 2>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
-        case 4: return launch<T, D, 4>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
-        case 8: return launch<T, D, 8>(out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+        case 1: return launch<T, D, 1>(a);
+        case 2: return launch<T, D, 2>(a);
+        case 4: return launch<T, D, 4>(a);
+        case 8: return launch<T, D, 8>(a);
         default: return PKV_ERR_UNSUPPORTED;
     }
 }
 
 template <typename T>
-int dispatch_d(int D, int G, void* out, const void* q, const void* kc, const void* vc, const int32_t* bt,
-               int32_t mb, const int32_t* cl, int32_t S, int32_t max_ctx, int32_t Hq, int32_t Hkv,
-               int32_t NB, float scale, void* ws, cudaStream_t st, int* status)
+int dispatch_d(int D, int G, const DecodeArgs& a)
 {
-    if (D == 64) return dispatch_g<T, 64>(G, out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
-    if (D == 128) return dispatch_g<T, 128>(G, out, q, kc, vc, bt, mb, cl, S, max_ctx, Hq, Hkv, NB, scale, ws, st, status);
+    if (D == 64) return dispatch_g<T, 64>(G, a);
+    if (D == 128) return dispatch_g<T, 128>(G, a);
     return PKV_ERR_UNSUPPORTED;
+}
+
+// Host-side checks and dispatch shared by the decode entry points.
+int decode_entry(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                 const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                 int32_t num_seqs, int32_t q_len, int32_t max_context_len, int32_t num_q_heads,
+                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                 int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (pkv::dtype_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        num_blocks < 1 || max_blocks_per_seq < 1 || !isfinite(scale) || (!k_new) != (!v_new))
+        return PKV_ERR_INVALID_ARG;
+    if (block_size != kBlock || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
+    if (q_len * G > 16) return PKV_ERR_UNSUPPORTED;  // the query rows fill one 16-row tensor-core operand
+    if (dtype == PKV_F32 && (q_len != 1 || k_new)) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (max_context_len < 1 || num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+    if (!pkv::aligned16(q) || !pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) ||
+        ((uintptr_t)out % pkv::dtype_bytes(dtype)) || ((uintptr_t)block_tables & 3u) ||
+        ((uintptr_t)context_lens & 3u) || (k_new && (!pkv::aligned16(k_new) || !pkv::aligned16(v_new))))
+        return PKV_ERR_INVALID_ARG;
+    const size_t need =
+        paged_attention_mq_workspace_bytes(num_seqs, q_len, num_q_heads, head_dim, max_context_len);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+        return PKV_ERR_INVALID_ARG;
+    int* status = pkv::status_word_for_current_device();
+    if (!status) return PKV_ERR_CUDA;
+    const DecodeArgs a{out,           q,        k_new,          v_new,        k_cache,      v_cache,
+                       block_tables,  max_blocks_per_seq,       context_lens, num_seqs,     q_len,
+                       max_context_len, num_q_heads, num_kv_heads, num_blocks, scale,       workspace,
+                       (cudaStream_t)stream, status};
+    switch (dtype) {
+        case PKV_F32: return dispatch_d<float>(head_dim, G, a);
+        case PKV_F16: return dispatch_d<__half>(head_dim, G, a);
+        default: return dispatch_d<__nv_bfloat16>(head_dim, G, a);
+    }
 }
 
 }  // namespace
 
+extern "C" size_t paged_attention_mq_workspace_bytes(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                                     int32_t head_dim, int32_t max_context_len)
+{
+    if (num_seqs <= 0 || q_len <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+    const size_t parts = ((size_t)max_context_len + kPartTokens - 1) / kPartTokens;
+    if (parts <= 1) return 0;
+    return (size_t)num_seqs * q_len * num_q_heads * parts * ((size_t)head_dim + 2) * sizeof(float);
+}
+
 extern "C" size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                                   int32_t head_dim, int32_t max_context_len)
 {
-    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
-    const size_t parts = ((size_t)max_context_len + kPartTokens - 1) / kPartTokens;
-    if (parts <= 1) return 0;
-    return (size_t)num_seqs * num_q_heads * parts * ((size_t)head_dim + 2) * sizeof(float);
+    return paged_attention_mq_workspace_bytes(num_seqs, 1, num_q_heads, head_dim, max_context_len);
 }
 
 extern "C" int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -682,41 +758,24 @@ extern "C" int paged_attention_decode(void* out, const void* q, const void* k_ca
                                       int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
                                       int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
-    if (pkv::dtype_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
-    if (num_seqs < 0 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
-        num_blocks < 1 || max_blocks_per_seq < 1 || !isfinite(scale))
-        return PKV_ERR_INVALID_ARG;
-    if (block_size != kBlock || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
-    const int G = num_q_heads / num_kv_heads;
-    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
-    if (num_seqs == 0) return PKV_OK;
-    if (max_context_len < 1 || num_seqs > 65535 || num_kv_heads > 65535) return PKV_ERR_INVALID_ARG;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
-    if (!pkv::aligned16(q) || !pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) ||
-        ((uintptr_t)out % pkv::dtype_bytes(dtype)) || ((uintptr_t)block_tables & 3u) ||
-        ((uintptr_t)context_lens & 3u))
-        return PKV_ERR_INVALID_ARG;
-    const size_t need = paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len);
-    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
-        return PKV_ERR_INVALID_ARG;
-    int* status = pkv::status_word_for_current_device();
-    if (!status) return PKV_ERR_CUDA;
-    cudaStream_t st = (cudaStream_t)stream;
-    switch (dtype) {
-        case PKV_F32:
-            return dispatch_d<float>(head_dim, G, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                     context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
-                                     num_blocks, scale, workspace, st, status);
-        case PKV_F16:
-            return dispatch_d<__half>(head_dim, G, out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                                      context_lens, num_seqs, max_context_len, num_q_heads, num_kv_heads,
-                                      num_blocks, scale, workspace, st, status);
-        default:
-            return dispatch_d<__nv_bfloat16>(head_dim, G, out, q, k_cache, v_cache, block_tables,
-                                             max_blocks_per_seq, context_lens, num_seqs, max_context_len,
-                                             num_q_heads, num_kv_heads, num_blocks, scale, workspace, st,
-                                             status);
-    }
+    // read-only caches: the const is cast away only for the shared launcher
+    return decode_entry(out, q, nullptr, nullptr, const_cast<void*>(k_cache), const_cast<void*>(v_cache),
+                        block_tables, max_blocks_per_seq, context_lens, num_seqs, 1, max_context_len,
+                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype, workspace,
+                        workspace_bytes, stream);
+}
+
+extern "C" int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const void* v_new,
+                                         void* k_cache, void* v_cache, const int32_t* block_tables,
+                                         int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                         int32_t num_seqs, int32_t q_len, int32_t max_context_len,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
+                                         void* workspace, size_t workspace_bytes, void* stream)
+{
+    return decode_entry(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                        num_seqs, q_len, max_context_len, num_q_heads, num_kv_heads, head_dim, block_size,
+                        num_blocks, scale, dtype, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -17,8 +17,10 @@
 //    for P.V (16 head-dim tiles, k = the block's 16 tokens).
 //  * Q stays in registers as MMA fragments (exact 16-bit inputs, scaled
 //    after the product in fp32).  The probabilities go from the score
-//    accumulators straight into the P.V operand (rounded to the input type;
-//    the running sum uses the unrounded fp32 values).
+//    accumulators straight into the P.V operand.  For fp16 they are rounded
+//    to fp16 (11 significant bits).  For bf16 they are split into a bf16
+//    pair hi + lo (about 16 bits) and multiplied by two MMAs, because one
+//    bf16 rounding (8 bits) can cost 5e-3 on a short, cancelling sum.
 //  * In the sequence's last, partial block, the V operand rows of tokens past
 //    the length are zeroed, and their scores are set to -inf, so whatever
 //    the unused slots hold cannot reach the result.
@@ -46,6 +48,14 @@ struct Mma<__nv_bfloat16> {
         __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&v);
     }
+    // bf16 keeps only 8 significant bits, too few for the probabilities of a
+    // short, cancelling sum; P is sent as hi + lo, two bf16 pairs holding
+    // about 16 bits, through two MMAs on the same V fragments.
+    static constexpr bool kSplitP = true;
+    __device__ __forceinline__ static uint32_t residual(float lo, float hi, uint32_t packed)
+    {
+        return pack(lo - __uint_as_float(packed << 16), hi - __uint_as_float(packed & 0xffff0000u));
+    }
 };
 
 template <>
@@ -63,6 +73,9 @@ struct Mma<__half> {
         __half2 v = __floats2half2_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&v);
     }
+    // fp16 keeps 11 significant bits: one MMA per P.V tile is accurate enough
+    static constexpr bool kSplitP = false;
+    __device__ __forceinline__ static uint32_t residual(float, float, uint32_t) { return 0u; }
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr)
@@ -126,38 +139,85 @@ __device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUte
     }
 }
 
-template <typename T, int D, int G>
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Online-softmax update of one score row held by a lane quad.  x: this
+// lane's 4 scores (log2 domain, -inf where masked); m / l: the row's
+// running max and this lane's share of the running sum.  Returns the
+// factor by which earlier partial outputs must be scaled.  A row that has
+// seen no visible token yet keeps m = -inf, and every factor stays finite.
+__device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
+{
+    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mn = fmaxf(m, mx);
+    const float mu = mn == -INFINITY ? 0.0f : mn;
+    const float alpha = pkv::fast_exp2(m - mu);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = pkv::fast_exp2(x[i] - mu);
+    l = l * alpha + ((x[0] + x[1]) + (x[2] + x[3]));
+    m = mn;
+    return alpha;
+}
+
+// One CTA = (partition p, kv head h, sequence s).
+//  kMQ = false: one query per sequence; rows 0..G-1 of the MMA operand are
+//               the G query heads of kv head h (q_len must be 1).
+//  kMQ = true : q_len new tokens per sequence; row r = j * G + g is query
+//               head h*G + g of new token j (q_len * G <= 16).  Token j sits
+//               at position ctx - q_len + j and sees positions up to its own.
+// k_new / v_new non-null: the new tokens' K/V rows [S][q_len][Hkv][D] are
+// written to their slots (through the block table) by the CTA whose
+// partition holds them, and patched into the staged tiles before use.
+template <typename T, int D, int G, bool kMQ>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
-                               const T* __restrict__ q, const int32_t* __restrict__ block_tables, int32_t mb,
-                               const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t num_q_heads,
-                               int32_t num_kv_heads, int32_t num_blocks, float scale_log2, int32_t max_parts,
-                               int* status)
+                               const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
+                               T* __restrict__ k_cache_w, T* __restrict__ v_cache_w,
+                               const int32_t* __restrict__ block_tables, int32_t mb,
+                               const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t q_len,
+                               int32_t num_q_heads, int32_t num_kv_heads, int32_t num_blocks, float scale_log2,
+                               int32_t max_parts, int* status)
 {
     using C = TcCfg<D>;
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
+    constexpr int kRows = kMQ ? 16 : G;  // operand rows that can hold queries
+    constexpr int kChunks = D / 8;       // 16-byte chunks per K or V row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = kMQ ? q_len * G : G;  // live query rows
 
-    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
+    SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
+    if (!sr.bad && sr.ctx < q_len) {
+        if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
+        sr.bad = true;
+    }
     if (sr.bad) {
         if (p == 0) {
-            for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-                pkv::store_out(out + ((int64_t)s * num_q_heads + h * G) * D + i, 0.0f);
+            for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
+                const int r = i / D;
+                const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
+                pkv::store_out(out + orow * D + i % D, 0.0f);
             }
         }
         return;
     }
     if (p >= sr.nparts) return;
 
-    const int nblk_seq = (sr.ctx + kBlock - 1) / kBlock;
+    const int ctx = sr.ctx;
+    const int nblk_seq = (ctx + kBlock - 1) / kBlock;
     const int blk0 = p * kPartBlocks;
     const int nb = min(kPartBlocks, nblk_seq - blk0);
-    const int last_valid = sr.ctx - (nblk_seq - 1) * kBlock;
+    const int first_new = ctx - q_len;   // position of the first new token
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
@@ -167,7 +227,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
         if (b < 0 || b >= num_blocks) {
             pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
-            b = 0;
+            b = -1;  // read block 0 in its place; never write through it
         }
         s_blk[i] = b;
     }
@@ -184,28 +244,37 @@ __global__ void __launch_bounds__(kWarps * 32)
         policy = pkv::policy_evict_first();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
-    }
-
-    if (lane == 0) {
         for (int k = 0; k < nw && k < kStages; ++k) {
             tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], &tm_k, &tm_v,
-                        (s_blk[warp + k * kWarps] * num_kv_heads + h) * kBlock, policy);
+                        (max(s_blk[warp + k * kWarps], 0) * num_kv_heads + h) * kBlock, policy);
         }
     }
 
-    // ---- Q as A fragments: row g = lane / 4 (zero for g >= G and rows 8..15)
-    const int g_row = lane >> 2;
+    // ---- Q as A fragments: rows ra = lane / 4 (a0, a2) and rb = ra + 8 (a1, a3)
+    const int ra = lane >> 2, rb = ra + 8;
     const int qd = 2 * (lane & 3);
+    const bool live_a = ra < rows;
+    const bool live_b = kMQ && rb < rows;
     uint32_t qa[C::kKSteps][4];
 #pragma unroll
     for (int ks = 0; ks < C::kKSteps; ++ks) {
         qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
-        if (g_row < G) {
-            const T* qrow = q + ((int64_t)s * num_q_heads + h * G + g_row) * D + 16 * ks + qd;
+        if (live_a) {
+            const T* qrow = q + (((int64_t)s * q_len + ra / G) * num_q_heads + h * G + ra % G) * D + 16 * ks + qd;
             qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
             qa[ks][2] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
+        if (live_b) {
+            const T* qrow = q + (((int64_t)s * q_len + rb / G) * num_q_heads + h * G + rb % G) * D + 16 * ks + qd;
+            qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow);
+            qa[ks][3] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+        }
     }
+    // positions a row may see: < lim.  Single query: every row (padding rows
+    // included, whose Q is zero) sees the whole context, so each row keeps a
+    // finite maximum.  Multi-query: a row holding no query sees nothing.
+    const int lim_a = kMQ ? (live_a ? first_new + ra / G + 1 : 0) : ctx;
+    const int lim_b = live_b ? first_new + rb / G + 1 : 0;
 
     // ---- per-lane ldmatrix addressing (128-byte swizzle: chunk c of row r is at c ^ (r % 8))
     const int mi = lane >> 3, r8 = lane & 7;
@@ -219,7 +288,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     float o[C::kNTiles][4];
 #pragma unroll
     for (int n = 0; n < C::kNTiles; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
-    float m_run = -INFINITY, l_part = 0.0f;
+    float m_a = -INFINITY, l_a = 0.0f, m_b = -INFINITY, l_b = 0.0f;
     bool timed_out = false;
     int consumed = 0;
 
@@ -231,7 +300,31 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         const uint32_t kbase = tiles + st * C::kStageBytes;
         const uint32_t vbase = kbase + C::kTileBytes;
-        const int valid = (blk0 + warp + k * kWarps == nblk_seq - 1) ? last_valid : kBlock;
+        const int lblk = warp + k * kWarps;
+        const int pos0 = (blk0 + lblk) * kBlock;
+
+        // ---- fused slot write: this block holds new tokens -> store and patch
+        if (k_new != nullptr && pos0 + kBlock > first_new) {
+            const int phys = s_blk[lblk];
+            const int jlo = max(0, pos0 - first_new);
+            const int jhi = min(q_len, pos0 + kBlock - first_new);
+            const int items = (jhi - jlo) * 2 * kChunks;
+            for (int it = lane; it < items; it += 32) {
+                const int c = it % kChunks;
+                const int kv = (it / kChunks) & 1;
+                const int jj = jlo + it / (2 * kChunks);
+                const int t = first_new + jj - pos0;
+                const T* src = (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8;
+                const uint4 val = *reinterpret_cast<const uint4*>(src);
+                st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 + (((c % 8) ^ (t & 7)) << 4),
+                             val);
+                if (phys >= 0) {
+                    T* dst = (kv ? v_cache_w : k_cache_w) + (((int64_t)phys * num_kv_heads + h) * kBlock + t) * D + c * 8;
+                    *reinterpret_cast<uint4*>(dst) = val;
+                }
+            }
+            __syncwarp();
+        }
 
         // ---- S = Q K^T for the block's 16 tokens (two 8-token tiles)
         float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -244,38 +337,78 @@ __global__ void __launch_bounds__(kWarps * 32)
             Mma<T>::run(s1, qa[ks], b[2], b[3]);
         }
 
-        // ---- online softmax on row g_row; this lane holds tokens qd, qd+1, qd+8, qd+9
-        float x[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
-        if (valid < kBlock) {
-            if (qd >= valid) x[0] = -INFINITY;
-            if (qd + 1 >= valid) x[1] = -INFINITY;
-            if (qd + 8 >= valid) x[2] = -INFINITY;
-            if (qd + 9 >= valid) x[3] = -INFINITY;
-        }
-        float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mn = fmaxf(m_run, mx);
-        const float alpha = pkv::fast_exp2(m_run - mn);
-        float pr[4];
+        // ---- online softmax; this lane holds tokens qd, qd+1, qd+8, qd+9 of rows ra (and rb)
+        const bool mask = pos0 + kBlock > first_new + 1;   // some token of this block is not visible to all rows
+        float xa[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
+        const int tp[4] = {pos0 + qd, pos0 + qd + 1, pos0 + qd + 8, pos0 + qd + 9};
+        float alpha_a, alpha_b = 1.0f;
+        uint32_t pa[4], pl[4];  // P (hi) and, for bf16, its residual (lo)
+        if constexpr (!kMQ) {
+            if (mask) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) pr[i] = pkv::fast_exp2(x[i] - mn);
-        l_part = l_part * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-        if (__any_sync(0xffffffffu, mn != m_run)) {
+                for (int i = 0; i < 4; ++i)
+                    if (tp[i] >= lim_a) xa[i] = -INFINITY;
+            }
+            float mx = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mn = fmaxf(m_a, mx);  // every block has a visible token: finite
+            alpha_a = pkv::fast_exp2(m_a - mn);
 #pragma unroll
-            for (int n = 0; n < C::kNTiles; ++n) {
-                o[n][0] *= alpha;
-                o[n][1] *= alpha;
+            for (int i = 0; i < 4; ++i) xa[i] = pkv::fast_exp2(xa[i] - mn);
+            l_a = l_a * alpha_a + ((xa[0] + xa[1]) + (xa[2] + xa[3]));
+            m_a = mn;
+            pa[0] = Mma<T>::pack(xa[0], xa[1]);
+            pa[1] = 0u;
+            pa[2] = Mma<T>::pack(xa[2], xa[3]);
+            pa[3] = 0u;
+            if constexpr (Mma<T>::kSplitP) {
+                pl[0] = Mma<T>::residual(xa[0], xa[1], pa[0]);
+                pl[1] = 0u;
+                pl[2] = Mma<T>::residual(xa[2], xa[3], pa[2]);
+                pl[3] = 0u;
+            }
+        } else {
+            float xb[4] = {s0[2] * scale_log2, s0[3] * scale_log2, s1[2] * scale_log2, s1[3] * scale_log2};
+            if (mask) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (tp[i] >= lim_a) xa[i] = -INFINITY;
+                    if (tp[i] >= lim_b) xb[i] = -INFINITY;
+                }
+            }
+            alpha_a = softmax_row(xa, m_a, l_a);
+            alpha_b = softmax_row(xb, m_b, l_b);
+            pa[0] = Mma<T>::pack(xa[0], xa[1]);
+            pa[1] = Mma<T>::pack(xb[0], xb[1]);
+            pa[2] = Mma<T>::pack(xa[2], xa[3]);
+            pa[3] = Mma<T>::pack(xb[2], xb[3]);
+            if constexpr (Mma<T>::kSplitP) {
+                pl[0] = Mma<T>::residual(xa[0], xa[1], pa[0]);
+                pl[1] = Mma<T>::residual(xb[0], xb[1], pa[1]);
+                pl[2] = Mma<T>::residual(xa[2], xa[3], pa[2]);
+                pl[3] = Mma<T>::residual(xb[2], xb[3], pa[3]);
             }
         }
-        m_run = mn;
-        const uint32_t pa[4] = {Mma<T>::pack(pr[0], pr[1]), 0u, Mma<T>::pack(pr[2], pr[3]), 0u};
+        if (__any_sync(0xffffffffu, alpha_a != 1.0f || alpha_b != 1.0f)) {
+#pragma unroll
+            for (int n = 0; n < C::kNTiles; ++n) {
+                o[n][0] *= alpha_a;
+                o[n][1] *= alpha_a;
+                if constexpr (kMQ) {
+                    o[n][2] *= alpha_b;
+                    o[n][3] *= alpha_b;
+                }
+            }
+        }
 
         // ---- O += P V over the head dimension (pairs of 8-wide tiles)
+        // V rows of tokens at or past the sequence length are zeroed: whatever
+        // the unused slots hold (even NaN) must not reach the result.
         uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // V rows qd, qd+1 / qd+8, qd+9
-        if (valid < kBlock) {
-            keep_lo = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
-            keep_hi = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
+        if (pos0 + kBlock > ctx) {
+            keep_lo = (tp[0] < ctx ? 0x0000ffffu : 0u) | (tp[1] < ctx ? 0xffff0000u : 0u);
+            keep_hi = (tp[2] < ctx ? 0x0000ffffu : 0u) | (tp[3] < ctx ? 0xffff0000u : 0u);
         }
 #pragma unroll
         for (int j = 0; j < C::kNTiles / 2; ++j) {
@@ -288,12 +421,16 @@ __global__ void __launch_bounds__(kWarps * 32)
             b[3] &= keep_hi;
             Mma<T>::run(o[2 * j], pa, b[0], b[1]);
             Mma<T>::run(o[2 * j + 1], pa, b[2], b[3]);
+            if constexpr (Mma<T>::kSplitP) {
+                Mma<T>::run(o[2 * j], pl, b[0], b[1]);
+                Mma<T>::run(o[2 * j + 1], pl, b[2], b[3]);
+            }
         }
         __syncwarp();
         ++consumed;
         if (lane == 0 && k + kStages < nw) {
-            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v, (s_blk[warp + (k + kStages) * kWarps] * num_kv_heads + h) * kBlock,
-                        policy);
+            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v,
+                        (max(s_blk[warp + (k + kStages) * kWarps], 0) * num_kv_heads + h) * kBlock, policy);
         }
     }
 
@@ -304,16 +441,21 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
     }
 
-    // ---- merge the warps: lane (g_row, qd) holds O[g_row][8n + qd .. +1]
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    // ---- merge the warps: lane (ra, qd) holds O[ra][8n + qd .. +1] (and row rb)
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    if constexpr (kMQ) {
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    }
     __syncthreads();
-    float* mg = reinterpret_cast<float*>(smem);  // [kWarps][G][D + 2]: m, l, acc[D]
-    if (g_row < G) {
-        float* rec = mg + (warp * G + g_row) * (D + 2);
+    float* mg = reinterpret_cast<float*>(smem);  // [kWarps][kRows][D + 2]: m, l, acc[D]
+    static_assert(kWarps * kRows * (D + 2) * 4 <= C::kTilesBytes, "merge area must fit in the tile area");
+    if (live_a) {
+        float* rec = mg + (warp * kRows + ra) * (D + 2);
         if ((lane & 3) == 0) {
-            rec[0] = m_run;
-            rec[1] = l_part;
+            rec[0] = m_a;
+            rec[1] = l_a;
         }
 #pragma unroll
         for (int n = 0; n < C::kNTiles; ++n) {
@@ -321,30 +463,44 @@ __global__ void __launch_bounds__(kWarps * 32)
             rec[2 + 8 * n + qd + 1] = o[n][1];
         }
     }
+    if constexpr (kMQ) {
+        if (live_b) {
+            float* rec = mg + (warp * kRows + rb) * (D + 2);
+            if ((lane & 3) == 0) {
+                rec[0] = m_b;
+                rec[1] = l_b;
+            }
+#pragma unroll
+            for (int n = 0; n < C::kNTiles; ++n) {
+                rec[2 + 8 * n + qd] = o[n][2];
+                rec[2 + 8 * n + qd + 1] = o[n][3];
+            }
+        }
+    }
     __syncthreads();
 
-    const int hq0 = h * G;
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-        const int g = i / D, d = i % D;
+    for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
+        const int r = i / D, d = i % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[(w * G + g) * (D + 2)]);
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[(w * kRows + r) * (D + 2)]);
+        const float Mu = M == -INFINITY ? 0.0f : M;  // a row that saw no token here: all weights 0
         float L = 0.0f, O = 0.0f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float* rec = mg + (w * G + g) * (D + 2);
-            const float wgt = exp2f(rec[0] - M);
+            const float* rec = mg + (w * kRows + r) * (D + 2);
+            const float wgt = pkv::fast_exp2(rec[0] - Mu);
             L = fmaf(rec[1], wgt, L);
             O = fmaf(rec[2 + d], wgt, O);
         }
-        const int64_t row = (int64_t)s * num_q_heads + hq0 + g;
+        const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
         if (sr.nparts == 1) {
-            pkv::store_out(out + row * D + d, O / L);
+            pkv::store_out(out + orow * D + d, O / L);
         } else {
-            ws_acc[(row * max_parts + p) * D + d] = O;
+            ws_acc[(orow * max_parts + p) * D + d] = O;
             if (d == 0) {
-                ws_ml[(row * max_parts + p) * 2] = M;
-                ws_ml[(row * max_parts + p) * 2 + 1] = L;
+                ws_ml[(orow * max_parts + p) * 2] = M;
+                ws_ml[(orow * max_parts + p) * 2 + 1] = L;
             }
         }
     }

@@ -250,9 +250,11 @@ def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min
 
 def make_custom(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype,
                 device="cpu", *, seed: int = 1234, spare_blocks: int = 3,
-                max_blocks_per_seq=None, pad_random: bool = False) -> DecodeWorkload:
+                max_blocks_per_seq=None, pad_random: bool = False, q_len=None) -> DecodeWorkload:
     """A batch with the given context lengths and head shape, blocks dealt
-    from a seeded permutation of a pool with `spare_blocks` unused blocks."""
+    from a seeded permutation of a pool with `spare_blocks` unused blocks.
+    With q_len given, q is [S, q_len, Hq, D] and k_new / v_new are
+    [S, q_len, Hkv, D] (several new tokens per sequence)."""
     g = torch.Generator().manual_seed(seed)
     B = BLOCK_SIZE
     ctx = [int(c) for c in context_lens]
@@ -271,11 +273,12 @@ def make_custom(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int
     S, Hq, Hkv, D = len(ctx), num_q_heads, num_kv_heads, head_dim
     dev = torch.device(device)
     gd = g if dev.type == "cpu" else torch.Generator(device=dev).manual_seed(seed)
-    q = _randn((S, Hq, D), dtype, gd, dev)
+    lead = (S,) if q_len is None else (S, q_len)
+    q = _randn(lead + (Hq, D), dtype, gd, dev)
     k_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
     v_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
-    k_new = _randn((S, Hkv, D), dtype, gd, dev)
-    v_new = _randn((S, Hkv, D), dtype, gd, dev)
+    k_new = _randn(lead + (Hkv, D), dtype, gd, dev)
+    v_new = _randn(lead + (Hkv, D), dtype, gd, dev)
     if pad_random:
         junk = torch.randint(0, NB, bt.shape, generator=g, dtype=torch.int32)
         bt = torch.where(bt < 0, junk, bt)

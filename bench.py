@@ -58,7 +58,7 @@ def decode_source_hash() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str, num_seqs: int):
+def recorded_traffic(workload: str, num_seqs: int, path: str):
     """DRAM bytes per decode call from the committed ncu record, or None if
     there is none for this workload or the decode sources changed since."""
     try:
@@ -68,7 +68,7 @@ def recorded_traffic(workload: str, num_seqs: int):
         return None
     if rec.get("source_sha256") != decode_source_hash():
         return None
-    if rec.get("workload") != workload or rec.get("num_seqs") != num_seqs:
+    if rec.get("workload") != workload or rec.get("num_seqs") != num_seqs or rec.get("path") != path:
         return None
     return rec.get("dram_bytes_per_call")
 
@@ -135,6 +135,10 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None):
     st.q, st.k_cache, st.v_cache = w.q, w.k_cache, w.v_cache
     st.k_new, st.v_new = w.k_new, w.v_new
     st.out = torch.empty_like(w.q)
+    # views with one new token per sequence, for the fused path
+    st.q4, st.out4 = st.q.unsqueeze(1), st.out.unsqueeze(1)
+    st.k_new4, st.v_new4 = st.k_new.unsqueeze(1), st.v_new.unsqueeze(1)
+    st.path = "separate"
     st.max_ctx = int(lens.max())
     ws_bytes = pkv.paged_attention_workspace_bytes(S, w.num_q_heads, w.head_dim, st.max_ctx)
     st.workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
@@ -148,19 +152,29 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None):
     st.write_bytes = 2 * 2 * S * w.num_kv_heads * w.head_dim * e + 8 * S
     st.copy_bytes = 2 * 2 * pairs.shape[0] * w.num_kv_heads * w.block_size * w.head_dim * e
     st.max_parts = (st.max_ctx + pkv.PARTITION_TOKENS - 1) // pkv.PARTITION_TOKENS
-    st.launches_per_step = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
+    st.launches_separate = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
+    st.launches_fused = st.launches_separate - 1
     return st
 
 
 def run_step(st, ev=None):
+    """One decode step on the device.  path 'separate': paged_kv_write, then
+    paged_attention_decode.  path 'fused': paged_attention_decode_mq with the
+    new tokens' K/V, which writes them to their slots in the same launch."""
     import paged_kv_cache_398_b200 as pkv
     if st.pairs.shape[0]:
         pkv.block_copy(st.k_cache, st.v_cache, st.pairs)
-    pkv.paged_kv_write(st.k_new, st.v_new, st.k_cache, st.v_cache, st.slots)
+    if st.path == "separate":
+        pkv.paged_kv_write(st.k_new, st.v_new, st.k_cache, st.v_cache, st.slots)
     if ev is not None:
         ev[0].record()
-    pkv.paged_attention_decode(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
-                               st.w.scale, st.max_ctx, workspace=st.workspace)
+    if st.path == "separate":
+        pkv.paged_attention_decode(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                                   st.w.scale, st.max_ctx, workspace=st.workspace)
+    else:
+        pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                                      st.w.scale, st.max_ctx, k_new=st.k_new4, v_new=st.v_new4,
+                                      workspace=st.workspace)
     if ev is not None:
         ev[1].record()
 
@@ -391,6 +405,7 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
 
     st = build_step(args.workload, dev, rank, args.num_seqs)
+    st.path = args.path
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
     # the oracle sample is copied off the device before the first product step
@@ -461,7 +476,9 @@ def run_ours(args):
     S = st.w.num_seqs
     value = kv_total * args.steps / (ms_max / 1e3) / 1e9
     dec_mean = statistics.mean(dec_ms)
-    achieved = st.decode_bytes / (dec_mean / 1e3) / 1e9
+    # the fused call also moves the new tokens' K/V (read and written once)
+    call_bytes = st.decode_bytes + (st.write_bytes if st.path == "fused" else 0)
+    achieved = call_bytes / (dec_mean / 1e3) / 1e9
     clk = clocks.summary(t_wall0, t_wall1)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -479,15 +496,18 @@ def run_ours(args):
         "unique_kv_gbps": uniq_total * args.steps / (ms_max / 1e3) / 1e9,
         "kernel_ms": {"decode_mean": dec_mean, "decode_min": min(dec_ms),
                       "write_and_copy_mean": ms_max / args.steps - dec_mean},
-        "roofline": {"kernel": "paged_attention_decode (partition kernel + split-K reduce)",
+        "roofline": {"kernel": ("paged_attention_decode_mq with fused slot write (partition kernel + split-K reduce)"
+                                if st.path == "fused" else
+                                "paged_attention_decode (partition kernel + split-K reduce)"),
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S),
-                     "algorithmic_bytes_per_launch": st.decode_bytes},
+                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path),
+                     "algorithmic_bytes_per_launch": call_bytes},
         "cpu_baseline": ({k: v for k, v in base.items() if k != "seconds"} if base else None),
         "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_steps},
-        "gpu_launches": st.launches_per_step * args.steps,
+        "gpu_launches": (st.launches_fused if st.path == "fused" else st.launches_separate) * args.steps,
+        "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
         "clocks": clk,
         "wall_s_timed": t_wall1 - t_wall0,
@@ -504,6 +524,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["fused", "separate"], default="fused",
+                    help="fused: slot write inside the decode launch; separate: paged_kv_write then decode")
     ap.add_argument("--reference-seqs", type=int, default=16)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same recipe (profiling); the default is the full workload")

@@ -369,6 +369,42 @@ def run_reference(args):
     return 0
 
 
+def measure_swap(st, dev, nblocks: int = 2048, iters: int = 10):
+    """Preemption traffic: swap_blocks_out / swap_blocks_in of nblocks blocks
+    of this workload's cache (then back into the same blocks, so the cache
+    is unchanged), against a plain pinned copy of the same bytes over the
+    host link.  GB/s counts K and V."""
+    import paged_kv_cache_398_b200 as pkv
+    w = st.w
+    n = min(nblocks, w.num_blocks)
+    ids = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(5))[:n]
+    shape = (n, w.num_kv_heads, w.block_size, w.head_dim)
+    hk = torch.empty(shape, dtype=w.dtype).pin_memory()
+    hv = torch.empty(shape, dtype=w.dtype).pin_memory()
+    dk = torch.empty(shape, dtype=w.dtype, device=dev)
+    nbytes = 2 * hk.numel() * hk.element_size()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        return nbytes * iters / (a.elapsed_time(b) / 1e3) / 1e9
+
+    out_gbps = timed(lambda: pkv.swap_blocks_out(st.k_cache, st.v_cache, ids, hk, hv))
+    in_gbps = timed(lambda: pkv.swap_blocks_in(st.k_cache, st.v_cache, ids, hk, hv))
+    d2h = timed(lambda: (hk.copy_(dk, non_blocking=True), hv.copy_(dk, non_blocking=True)))
+    h2d = timed(lambda: (dk.copy_(hk, non_blocking=True), dk.copy_(hv, non_blocking=True)))
+    return {"blocks": n, "bytes_per_call": nbytes, "out_gbps": out_gbps, "in_gbps": in_gbps,
+            "link_d2h_gbps": d2h, "link_h2d_gbps": h2d,
+            "note": "one gather/scatter kernel over pinned host memory vs a contiguous pinned copy of the same size"}
+
+
 def reduce_over_ranks(dist, device, times_ms, amounts):
     """Max over ranks of each time, sum over ranks of each amount (timing and
     byte counts only; the decode path itself exchanges nothing)."""
@@ -463,6 +499,7 @@ def run_ours(args):
     t_wall2 = time.monotonic()
     e2e_ms = e0.elapsed_time(e1)
     clocks.stop()
+    swap = measure_swap(st, dev) if not args.no_swap else None
 
     ms_max, e2e_max, kv_total, uniq_total = reduce_over_ranks(
         dist, dev, [ms, e2e_ms], [float(st.kv_bytes), float(st.kv_unique_bytes)])
@@ -510,6 +547,7 @@ def run_ours(args):
         "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
         "clocks": clk,
+        "swap": swap,
         "wall_s_timed": t_wall1 - t_wall0,
     }
     print(json.dumps(line), flush=True)
@@ -524,6 +562,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-swap", action="store_true", help="skip the swap-out / swap-in measurement")
     ap.add_argument("--path", choices=["fused", "separate"], default="fused",
                     help="fused: slot write inside the decode launch; separate: paged_kv_write then decode")
     ap.add_argument("--reference-seqs", type=int, default=16)

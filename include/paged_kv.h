@@ -258,6 +258,32 @@ int block_copy(void* k_cache, void* v_cache, const int64_t* pairs, int32_t num_p
                int32_t dtype, void* stream);
 
 /*
+ * swap_blocks_out / swap_blocks_in -- move whole blocks (keys and values of
+ * every kv head) between the device cache and host memory, so a preempted
+ * sequence can give its device blocks back and later resume where it stopped.
+ * ("vLLM Architecture": the scheduler preempts low-priority requests by
+ * swapping their blocks to CPU memory.)
+ *
+ *  block_ids      HOST, int64 [n], each in [0, num_blocks).  For swap-in,
+ *                 no id may appear twice (PKV_ERR_INVALID_ARG).
+ *  host_k, host_v HOST memory, pinned (page-locked) and mapped into the
+ *                 device's address space (cudaHostAlloc / cudaMallocHost, or
+ *                 torch pin_memory()); each [n][num_kv_heads][block_size]
+ *                 [head_dim] of dtype.  Slot i holds block block_ids[i].
+ *                 Pageable memory returns PKV_ERR_INVALID_ARG.
+ *  swap_blocks_out copies device -> host; swap_blocks_in host -> device.
+ *  One kernel launch per 1024 blocks moves the data over the host link.
+ *  The call is asynchronous on `stream`; the host buffers must stay alive
+ *  and untouched until the stream reaches this point.  The copy is bit-exact.
+ */
+int swap_blocks_out(const void* k_cache, const void* v_cache, const int64_t* block_ids, int32_t n,
+                    void* host_k, void* host_v, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, int32_t dtype, void* stream);
+int swap_blocks_in(void* k_cache, void* v_cache, const int64_t* block_ids, int32_t n,
+                   const void* host_k, const void* host_v, int32_t num_kv_heads, int32_t head_dim,
+                   int32_t block_size, int32_t num_blocks, int32_t dtype, void* stream);
+
+/*
  * pkv_slot_mapping -- HOST helper: slots_out[s] = slot of token position
  * positions[s] of sequence s, given its block-table row (host int32
  * [num_seqs][max_blocks_per_seq]).  Returns PKV_ERR_INVALID_ARG for a
@@ -367,6 +393,19 @@ int pkv_seq_num_tokens(const pkv_allocator* a, int64_t seq, int32_t* out);
 int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
                      int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
                      int32_t* context_lens_out);
+
+/* Preemption.  pkv_seq_swap_out lists the sequence's blocks in logical
+ * order in blocks_out (HOST int32 [cap]; *n_out = count), for
+ * swap_blocks_out.  It then releases them like pkv_seq_free, but the
+ * sequence stays registered, swapped out, with its token count.
+ * pkv_seq_swap_in takes fresh blocks for a swapped-out sequence in one
+ * all-or-nothing step (PKV_ERR_OUT_OF_BLOCKS changes nothing) and lists
+ * them in logical order, the destinations for swap_blocks_in.  While a
+ * sequence is swapped out, append, fork, share_prefix and
+ * pkv_batch_tables refuse it (PKV_ERR_INVALID_ARG); pkv_seq_free drops it. */
+int pkv_seq_swap_out(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t cap, int32_t* n_out);
+int pkv_seq_swap_in(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t cap, int32_t* n_out);
+int pkv_seq_is_swapped(const pkv_allocator* a, int64_t seq, int32_t* out);
 
 int32_t pkv_num_free(const pkv_allocator* a);
 /* The free blocks in the order they will be handed out (HOST int32 [cap]). */

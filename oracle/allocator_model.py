@@ -32,6 +32,12 @@ Policy choices the pages leave open (the product follows the same ones):
   last holder (count == 1) writes in place.
 * An operation that cannot get every block it needs fails with
   ``OutOfBlocks`` and changes nothing.
+* Swapping a sequence out ("vLLM Architecture": the scheduler preempts
+  low-priority requests by swapping their blocks to CPU memory) reports its
+  blocks in logical order, then releases them like ``free``.  The sequence
+  keeps its token count.  Swapping it back in takes fresh blocks in one
+  all-or-nothing step.  A swapped-out sequence accepts no other operation
+  except ``free``.
 """
 
 from __future__ import annotations
@@ -83,7 +89,7 @@ class AllocatorModel:
         return self._seq(seq)["ntok"]
 
     def stats(self) -> dict:
-        frag = sum(len(s["blocks"]) * self.block_size - s["ntok"] for s in self._seqs.values())
+        frag = sum(len(s["blocks"]) * self.block_size - s["ntok"] for s in self._seqs.values() if not s["swapped"])
         return {
             "num_blocks": self.num_blocks,
             "free_blocks": len(self._free),
@@ -136,13 +142,48 @@ class AllocatorModel:
     def add(self, seq: int) -> None:
         if seq in self._seqs:
             raise InvalidArgument(f"sequence {seq} exists")
-        self._seqs[seq] = {"blocks": [], "ntok": 0}
+        self._seqs[seq] = {"blocks": [], "ntok": 0, "swapped": False, "nswap": 0}
+
+    def _live(self, seq: int) -> dict:
+        s = self._seq(seq)
+        if s["swapped"]:
+            raise InvalidArgument(f"sequence {seq} is swapped out")
+        return s
+
+    def is_swapped(self, seq: int) -> bool:
+        return self._seq(seq)["swapped"]
+
+    def swap_out(self, seq: int) -> list[int]:
+        """Blocks to copy to host memory (logical order); they are released."""
+        s = self._live(seq)
+        blocks = list(s["blocks"])
+        for b in reversed(blocks):
+            self._ref[b] -= 1
+            if self._ref[b] == 0:
+                self._free.append(b)
+        s["blocks"] = []
+        s["swapped"] = True
+        s["nswap"] = len(blocks)
+        return blocks
+
+    def swap_in(self, seq: int) -> list[int]:
+        """Fresh blocks for a swapped-out sequence, in logical order."""
+        s = self._seq(seq)
+        if not s["swapped"]:
+            raise InvalidArgument(f"sequence {seq} is not swapped out")
+        n = s["nswap"]
+        if n > len(self._free):
+            raise OutOfBlocks()
+        s["blocks"] = [self._pop() for _ in range(n)]
+        s["swapped"] = False
+        s["nswap"] = 0
+        return list(s["blocks"])
 
     def append_tokens(self, seq: int, n: int):
         """Reserve slots for n new tokens; returns (slots, cow_pair_or_None)."""
         if n < 0:
             raise InvalidArgument("negative token count")
-        s = self._seq(seq)
+        s = self._live(seq)
         if self._needs(s, n) > len(self._free):
             raise OutOfBlocks()
         return self._append(s, n)
@@ -151,7 +192,7 @@ class AllocatorModel:
         """One new token for each sequence, in order: (slots, cow_pairs)."""
         if len(set(seqs)) != len(seqs):
             raise InvalidArgument("a sequence is named twice")
-        recs = [self._seq(q) for q in seqs]
+        recs = [self._live(q) for q in seqs]
         if sum(self._needs(r, 1) for r in recs) > len(self._free):
             raise OutOfBlocks()
         slots, pairs = [], []
@@ -171,16 +212,16 @@ class AllocatorModel:
         del self._seqs[seq]
 
     def fork(self, parent: int, child: int) -> None:
-        p = self._seq(parent)
+        p = self._live(parent)
         if child in self._seqs:
             raise InvalidArgument(f"sequence {child} exists")
         for b in p["blocks"]:
             self._ref[b] += 1
-        self._seqs[child] = {"blocks": list(p["blocks"]), "ntok": p["ntok"]}
+        self._seqs[child] = {"blocks": list(p["blocks"]), "ntok": p["ntok"], "swapped": False, "nswap": 0}
 
     def share_prefix(self, seq: int, blocks, num_tokens: int) -> None:
         """Point an empty sequence at existing (allocated) blocks holding num_tokens tokens."""
-        s = self._seq(seq)
+        s = self._live(seq)
         blocks = [int(b) for b in blocks]
         B = self.block_size
         if s["blocks"] or s["ntok"]:

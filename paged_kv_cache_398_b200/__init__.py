@@ -8,6 +8,7 @@ C ABI of ``include/paged_kv.h``:
 * ``paged_kv_write``          -- slot write of the new tokens' K/V
 * ``paged_attention_decode``  -- decode attention through the block tables
 * ``block_copy``              -- copy-on-write block copy
+* ``swap_blocks_out`` / ``swap_blocks_in`` -- preemption: blocks to / from host memory
 * ``BlockAllocator``          -- host block allocator (free list, refcounts, CoW)
 
 The native library ``libpaged_kv.so`` is built in-tree by
@@ -19,11 +20,11 @@ from .allocator import BlockAllocator, OutOfBlocks
 from .binding import (BLOCK_SIZE, PARTITION_TOKENS, block_copy, paged_attention_decode,
                       paged_attention_decode_mq, paged_attention_decode_noalloc,
                       paged_attention_mq_workspace_bytes, paged_attention_workspace_bytes, paged_kv_write,
-                      pkv_device_status, pkv_slot_mapping)
+                      pkv_device_status, pkv_slot_mapping, swap_blocks_in, swap_blocks_out)
 
 __all__ = [
     "BLOCK_SIZE", "PARTITION_TOKENS", "BlockAllocator", "LibraryMissing", "OutOfBlocks",
     "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_decode_mq",
     "paged_attention_decode_noalloc", "paged_attention_mq_workspace_bytes", "paged_attention_workspace_bytes",
-    "paged_kv_write", "pkv_device_status", "pkv_slot_mapping",
+    "paged_kv_write", "pkv_device_status", "pkv_slot_mapping", "swap_blocks_in", "swap_blocks_out",
 ]

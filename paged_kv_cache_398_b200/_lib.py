@@ -49,6 +49,11 @@ _SIGS = {
     "paged_attention_decode_noalloc": ([P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
                                         ctypes.c_float, I32, P], ctypes.c_int),
     "block_copy": ([P, P, P, I32, I32, I32, I32, I32, I32, P], ctypes.c_int),
+    "swap_blocks_out": ([P, P, P, I32, P, P, I32, I32, I32, I32, I32, P], ctypes.c_int),
+    "swap_blocks_in": ([P, P, P, I32, P, P, I32, I32, I32, I32, I32, P], ctypes.c_int),
+    "pkv_seq_swap_out": ([P, I64, P, I32, P], ctypes.c_int),
+    "pkv_seq_swap_in": ([P, I64, P, I32, P], ctypes.c_int),
+    "pkv_seq_is_swapped": ([P, I64, P], ctypes.c_int),
     "pkv_slot_mapping": ([P, I32, P, I32, I32, P], ctypes.c_int),
     "pkv_device_status": ([I32, P, I32], ctypes.c_int),
     "pkv_last_cuda_error": ([], ctypes.c_int),

@@ -120,6 +120,30 @@ class BlockAllocator:
             self._h, ids.data_ptr(), S, tables.data_ptr(), max_blocks_per_seq, pad, lens.data_ptr()))
         return tables[:S], lens[:S]
 
+    def swap_out(self, seq: int) -> list:
+        """Release a sequence's blocks for preemption; returns them (logical
+        order) so their contents can be copied out with swap_blocks_out."""
+        n = ctypes.c_int32(0)
+        cap = len(self.block_table(seq))
+        out = torch.empty(max(cap, 1), dtype=torch.int32)
+        _check("pkv_seq_swap_out", self._L.pkv_seq_swap_out(self._h, seq, out.data_ptr(), out.numel(),
+                                                            ctypes.byref(n)))
+        return out[:n.value].tolist()
+
+    def swap_in(self, seq: int) -> list:
+        """Fresh blocks for a swapped-out sequence (logical order), the
+        destinations for swap_blocks_in."""
+        n = ctypes.c_int32(0)
+        out = torch.empty(max(self.num_blocks, 1), dtype=torch.int32)
+        _check("pkv_seq_swap_in", self._L.pkv_seq_swap_in(self._h, seq, out.data_ptr(), out.numel(),
+                                                          ctypes.byref(n)))
+        return out[:n.value].tolist()
+
+    def is_swapped(self, seq: int) -> bool:
+        v = ctypes.c_int32(0)
+        _check("pkv_seq_is_swapped", self._L.pkv_seq_is_swapped(self._h, seq, ctypes.byref(v)))
+        return bool(v.value)
+
     def num_free(self) -> int:
         return int(self._L.pkv_num_free(self._h))
 

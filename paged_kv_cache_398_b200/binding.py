@@ -194,6 +194,31 @@ def block_copy(k_cache, v_cache, pairs, stream=None) -> None:
     check("block_copy", rc)
 
 
+def _swap(name, k_cache, v_cache, block_ids, host_k, host_v, stream):
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    ids = torch.as_tensor(block_ids, dtype=torch.int64, device="cpu").reshape(-1).contiguous()
+    n = ids.numel()
+    for nm, t in (("host_k", host_k), ("host_v", host_v)):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous host tensor")
+        if t.dtype != k_cache.dtype or tuple(t.shape) != (n, Hkv, B, D):
+            raise ValueError(f"{nm} must be {k_cache.dtype} [n, Hkv, B, D] with n = len(block_ids)")
+    rc = getattr(lib(), name)(k_cache.data_ptr(), v_cache.data_ptr(), ids.data_ptr(), n, host_k.data_ptr(),
+                              host_v.data_ptr(), Hkv, D, B, NB, _dtype_code(k_cache), _stream(k_cache.device, stream))
+    check(name, rc)
+
+
+def swap_blocks_out(k_cache, v_cache, block_ids, host_k, host_v, stream=None) -> None:
+    """Copy device blocks block_ids[i] into slot i of the pinned host buffers
+    host_k / host_v [n, Hkv, B, D] (asynchronous on the stream)."""
+    _swap("swap_blocks_out", k_cache, v_cache, block_ids, host_k, host_v, stream)
+
+
+def swap_blocks_in(k_cache, v_cache, block_ids, host_k, host_v, stream=None) -> None:
+    """Copy slot i of the pinned host buffers into device block block_ids[i]."""
+    _swap("swap_blocks_in", k_cache, v_cache, block_ids, host_k, host_v, stream)
+
+
 def pkv_slot_mapping(block_tables: torch.Tensor, positions: torch.Tensor, block_size: int = BLOCK_SIZE):
     """Host helper: slot of positions[s] in sequence s given host tables [S, MB]."""
     bt = torch.as_tensor(block_tables, dtype=torch.int32).contiguous()

@@ -25,6 +25,8 @@ namespace {
 struct Seq {
     std::vector<int32_t> blocks;
     int64_t ntok = 0;
+    bool swapped = false;  // blocks live in host memory (swap_blocks_out)
+    int32_t nswap = 0;     // how many
 };
 
 }  // namespace
@@ -94,6 +96,12 @@ struct pkv_allocator {
         auto it = seqs.find(id);
         return it == seqs.end() ? nullptr : &it->second;
     }
+    // a sequence whose blocks are on the device
+    Seq* live(int64_t id)
+    {
+        Seq* s = find(id);
+        return (s && !s->swapped) ? s : nullptr;
+    }
     const Seq* find(int64_t id) const
     {
         auto it = seqs.find(id);
@@ -145,7 +153,7 @@ int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slo
                           int64_t* cow_pair_out, int32_t* cow_out)
 {
     if (!a || n < 0) return PKV_ERR_INVALID_ARG;
-    Seq* s = a->find(seq);
+    Seq* s = a->live(seq);
     if (!s) return PKV_ERR_INVALID_ARG;
     if (a->needs(*s, n) > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
     a->append(*s, n, slots_out, cow_pair_out, cow_out);
@@ -159,7 +167,7 @@ int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
     std::vector<Seq*> recs(n_seqs);
     int64_t need = 0;
     for (int32_t i = 0; i < n_seqs; ++i) {
-        recs[i] = a->find(seqs[i]);
+        recs[i] = a->live(seqs[i]);
         if (!recs[i]) return PKV_ERR_INVALID_ARG;
         need += a->needs(*recs[i], 1);
     }
@@ -199,7 +207,7 @@ int pkv_seq_free(pkv_allocator* a, int64_t seq)
 int pkv_seq_fork(pkv_allocator* a, int64_t parent, int64_t child)
 {
     if (!a) return PKV_ERR_INVALID_ARG;
-    const Seq* p = a->find(parent);
+    const Seq* p = a->live(parent);
     if (!p || a->find(child)) return PKV_ERR_INVALID_ARG;
     Seq c = *p;
     for (int32_t b : c.blocks) a->incref(b);
@@ -211,7 +219,7 @@ int pkv_seq_share_prefix(pkv_allocator* a, int64_t seq, const int32_t* blocks, i
                          int32_t n_tokens)
 {
     if (!a || n_blocks < 0 || n_tokens < 0 || (n_blocks > 0 && !blocks)) return PKV_ERR_INVALID_ARG;
-    Seq* s = a->find(seq);
+    Seq* s = a->live(seq);
     if (!s || !s->blocks.empty() || s->ntok != 0) return PKV_ERR_INVALID_ARG;
     if ((int64_t)(n_tokens + a->block_size - 1) / a->block_size != n_blocks) return PKV_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_blocks; ++i) {
@@ -253,7 +261,7 @@ int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs
         return PKV_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n_seqs; ++i) {
         const Seq* s = a->find(seqs[i]);
-        if (!s || (int64_t)s->blocks.size() > max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
+        if (!s || s->swapped || (int64_t)s->blocks.size() > max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
     }
     for (int32_t i = 0; i < n_seqs; ++i) {
         const Seq* s = a->find(seqs[i]);
@@ -295,10 +303,51 @@ int pkv_alloc_get_stats(const pkv_allocator* a, pkv_alloc_stats* out)
     int64_t tok = 0, frag = 0;
     for (const auto& kv : a->seqs) {
         tok += kv.second.ntok;
-        frag += (int64_t)kv.second.blocks.size() * a->block_size - kv.second.ntok;
+        if (!kv.second.swapped) frag += (int64_t)kv.second.blocks.size() * a->block_size - kv.second.ntok;
     }
     out->num_tokens = tok;
     out->fragmentation_tokens = frag;
+    return PKV_OK;
+}
+
+int pkv_seq_swap_out(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t cap, int32_t* n_out)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->live(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    const int32_t n = (int32_t)s->blocks.size();
+    if (n_out) *n_out = n;
+    if (n > cap || (n > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
+    if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
+    for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
+    s->blocks.clear();
+    s->swapped = true;
+    s->nswap = n;
+    return PKV_OK;
+}
+
+int pkv_seq_swap_in(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t cap, int32_t* n_out)
+{
+    if (!a) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->find(seq);
+    if (!s || !s->swapped) return PKV_ERR_INVALID_ARG;
+    const int32_t n = s->nswap;
+    if (n_out) *n_out = n;
+    if (n > cap || (n > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
+    if (n > (int32_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    for (int32_t i = 0; i < n; ++i) s->blocks.push_back(a->pop());
+    if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
+    s->swapped = false;
+    s->nswap = 0;
+    return PKV_OK;
+}
+
+int pkv_seq_is_swapped(const pkv_allocator* a, int64_t seq, int32_t* out)
+{
+    if (!a || !out) return PKV_ERR_INVALID_ARG;
+    const Seq* s = a->find(seq);
+    if (!s) return PKV_ERR_INVALID_ARG;
+    *out = s->swapped ? 1 : 0;
     return PKV_OK;
 }
 

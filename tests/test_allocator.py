@@ -8,6 +8,7 @@ worked examples run through the native allocator as well.
 import random
 
 import pytest
+import torch
 
 import paged_kv_cache_398_b200 as pkv
 from oracle.allocator_model import AllocatorModel, InvalidArgument, OutOfBlocks
@@ -119,6 +120,8 @@ def test_random_operations_match_model(seed):
                 next_id += 1
             elif op < 0.55:
                 s = rng.choice(live)
+                if m.is_swapped(s):
+                    continue
                 n = rng.choice([0, 1, 1, 1, 3, 15, 16, 17, 40])
                 try:
                     want = m.append_tokens(s, n)
@@ -129,7 +132,9 @@ def test_random_operations_match_model(seed):
                     got = a.append_tokens(s, n)
                     assert got == (want[0], want[1])
             elif op < 0.65:
-                batch = rng.sample(live, k=min(len(live), rng.randint(1, 6)))
+                batch = [q for q in rng.sample(live, k=min(len(live), rng.randint(1, 6))) if not m.is_swapped(q)]
+                if not batch:
+                    continue
                 try:
                     ws, wp = m.append_one_batch(batch)
                 except OutOfBlocks:
@@ -140,17 +145,32 @@ def test_random_operations_match_model(seed):
                     assert gs.tolist() == ws and [tuple(p) for p in gp.tolist()] == wp
             elif op < 0.8:
                 s = rng.choice(live)
+                if m.is_swapped(s):
+                    continue
                 m.fork(s, next_id)
                 a.fork(s, next_id)
                 live.append(next_id)
                 next_id += 1
+            elif op < 0.83 and live:
+                s = rng.choice(live)
+                if m.is_swapped(s):
+                    try:
+                        want = m.swap_in(s)
+                    except OutOfBlocks:
+                        with pytest.raises(pkv.OutOfBlocks):
+                            a.swap_in(s)
+                    else:
+                        assert a.swap_in(s) == want
+                else:
+                    assert a.swap_out(s) == m.swap_out(s)
+                assert a.is_swapped(s) == m.is_swapped(s)
             elif op < 0.87 and live:
                 s = rng.choice(live)
-                if m.num_tokens(s) == 0:
+                if m.num_tokens(s) == 0 and not m.is_swapped(s):
                     src = rng.choice(live)
                     blocks = m.block_table(src)
                     full = len(blocks) * 16
-                    if blocks and m.num_tokens(src) == full:
+                    if blocks and m.num_tokens(src) == full and not m.is_swapped(src):
                         m.share_prefix(s, blocks, full)
                         a.share_prefix(s, blocks, full)
             else:
@@ -193,3 +213,62 @@ def test_batch_tables_pad():
     t, lens = a.batch_tables([1, 0], 4, pad=-1)
     assert t.tolist() == [[1, 2, 3, -1], [0, -1, -1, -1]]
     assert lens.tolist() == [33, 5]
+
+
+def test_swap_out_and_in_native():
+    """Preemption: a swapped-out sequence gives its blocks back, keeps its
+    token count, and resumes in fresh blocks; shared blocks stay with the
+    other holders."""
+    a = pkv.BlockAllocator(12, 16)
+    m = AllocatorModel(12, 16)
+    for x in (a, m):
+        x.add(0)
+        x.append_tokens(0, 40)            # blocks 0, 1, 2
+        x.fork(0, 1)                      # 1 shares them
+        x.append_tokens(1, 30)            # CoW of block 2 (-> 3), then new blocks 4 and 5
+    assert a.block_table(1) == m.block_table(1)
+    out_a, out_m = a.swap_out(1), m.swap_out(1)
+    assert out_a == out_m == [0, 1, 3, 4, 5]
+    assert a.is_swapped(1) and a.num_tokens(1) == 70
+    assert a.refcount(0) == 1 and a.refcount(3) == 0       # shared kept, private freed
+    for bad in (lambda: a.append_tokens(1, 1), lambda: a.fork(1, 9), lambda: a.batch_tables([1], 8),
+                lambda: a.swap_out(1)):
+        with pytest.raises(pkv.PagedKVError):
+            bad()
+    # another request takes the freed blocks; the swapped one comes back elsewhere
+    for x in (a, m):
+        x.add(2)
+        x.append_tokens(2, 32)
+    assert a.block_table(2) == m.block_table(2)
+    back_a, back_m = a.swap_in(1), m.swap_in(1)
+    assert back_a == back_m and len(back_a) == 5
+    assert not a.is_swapped(1) and a.block_table(1) == back_a
+    assert a.stats() == m.stats()
+    with pytest.raises(pkv.PagedKVError):
+        a.swap_in(1)
+
+
+def test_swap_in_is_all_or_nothing():
+    a = pkv.BlockAllocator(4, 16)
+    a.add(0)
+    a.append_tokens(0, 48)                # 3 blocks
+    a.swap_out(0)
+    a.add(1)
+    a.append_tokens(1, 40)                # takes 3 of the 4 blocks
+    with pytest.raises(pkv.OutOfBlocks):
+        a.swap_in(0)
+    assert a.is_swapped(0) and a.num_free() == 1
+    a.free(1)
+    assert len(a.swap_in(0)) == 3
+
+
+def test_swap_kernels_reject_bad_lists_on_host():
+    from paged_kv_cache_398_b200._lib import C, lib
+    import ctypes
+    L = lib()
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 16
+    for ids, fn in (([0, 9], "swap_blocks_out"), ([-1], "swap_blocks_in"), ([2, 2], "swap_blocks_in")):
+        t = torch.tensor(ids, dtype=torch.int64)
+        rc = getattr(L, fn)(p, p, t.data_ptr(), t.numel(), p, p, 2, 64, 16, 8, C["PKV_F16"], None)
+        assert rc == C["PKV_ERR_INVALID_ARG"], (ids, fn)

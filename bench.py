@@ -102,25 +102,33 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None):
     st = Step()
     st.w = w
     st.host_alloc_us = None
+    st.prefix = None
+    st.admit_us_per_request = None
     if number == 5:
         # parallel sampling: the generator's tables already hold the shared
         # prompt blocks; the step's copy-on-write pairs come with them
         tables, lens, pairs = w.block_tables, w.context_lens, w.copy_pairs
         slots = pkv.pkv_slot_mapping(tables, lens - 1)
     else:
-        perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(seed + 7))
+        gen = torch.Generator().manual_seed(seed + 7)
+        perm = torch.randperm(w.num_blocks, generator=gen)
         alloc = pkv.BlockAllocator(w.num_blocks, w.block_size, initial_order=perm)
-        prefix_tokens = 64 if number == 4 else 0
-        prefix = []
-        if prefix_tokens:
-            alloc.add(-1)
-            alloc.append_tokens(-1, prefix_tokens)
-            prefix = alloc.block_table(-1)
-        for s in range(S):
-            alloc.add(s)
-            if prefix:
-                alloc.share_prefix(s, prefix, prefix_tokens)
-            alloc.append_tokens(s, int(w.context_lens[s]) - 1 - prefix_tokens)
+        if number == 4:
+            # every request starts with the same 64-token system prompt; the
+            # prefix cache finds its 4 blocks instead of being told about them
+            system = torch.randint(0, 128000, (64,), generator=gen)
+            t0 = time.perf_counter()
+            for s in range(S):
+                own = torch.randint(0, 128000, (int(w.context_lens[s]) - 1 - 64,), generator=gen)
+                alloc.add(s)
+                alloc.append_prompt(s, torch.cat([system, own]))
+            st.admit_us_per_request = (time.perf_counter() - t0) * 1e6 / S
+            st.prefix = alloc.prefix_stats()
+            assert st.prefix["hit_tokens"] == 64 * (S - 1)
+        else:
+            for s in range(S):
+                alloc.add(s)
+                alloc.append_tokens(s, int(w.context_lens[s]) - 1)
         seqs = list(range(S))
         t0 = time.perf_counter()
         slots, pairs = alloc.append_one_batch(seqs)          # this step's slots (+ CoW pairs)
@@ -546,6 +554,10 @@ def run_ours(args):
         "gpu_launches": (st.launches_fused if st.path == "fused" else st.launches_separate) * args.steps,
         "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
+        "prefix_cache": (None if st.prefix is None else
+                         {"admit_us_per_request": st.admit_us_per_request, "hit_tokens": st.prefix["hit_tokens"],
+                          "blocks_shared": st.prefix["hit_tokens"] // st.w.block_size,
+                          "cached_blocks": st.prefix["cached_blocks"]}),
         "clocks": clk,
         "swap": swap,
         "wall_s_timed": t_wall1 - t_wall0,

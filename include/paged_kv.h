@@ -394,6 +394,34 @@ int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs
                      int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
                      int32_t* context_lens_out);
 
+/* Prefix cache ("Prefix Caching": a system prompt identical across
+ * requests is stored once; "PagedAttention & Continuous Batching…",
+ * item 5).  pkv_seq_append_prompt gives an empty sequence its prompt
+ * (token_ids: HOST int32 [n]).  It walks the prompt's full blocks in order
+ * and reuses every leading block whose content is already cached.  A
+ * block's identity is the block before it, that block's generation and its
+ * own block_size token ids, compared exactly.  From the first miss on it
+ * takes fresh blocks and makes each new full block findable.  slots_out
+ * (HOST int64 [n], may be NULL) receives -1 for the cached tokens (their
+ * K/V is already in place) and the slot of every other token.
+ * *n_cached_out receives the number of cached tokens, a multiple of
+ * block_size.  A cached block that no sequence uses any more stays
+ * findable.  It is handed out again (evicted, least recently released
+ * first) only when no never-cached block is free; pkv_num_free and
+ * pkv_free_list count it as free.  All-or-nothing:
+ * PKV_ERR_OUT_OF_BLOCKS changes nothing. */
+typedef struct pkv_prefix_stats {
+    int32_t cached_blocks;      /* blocks findable by content                 */
+    int32_t evictable_blocks;   /* of those, used by no sequence              */
+    int64_t prompts;            /* pkv_seq_append_prompt calls with a full block */
+    int64_t prompts_with_hits;  /* of those, calls that reused >= 1 block     */
+    int64_t hit_tokens;         /* prompt tokens served from the cache        */
+    int64_t evictions;          /* cached blocks reclaimed for new content    */
+} pkv_prefix_stats;
+int pkv_seq_append_prompt(pkv_allocator* a, int64_t seq, const int32_t* token_ids, int32_t n,
+                          int64_t* slots_out, int32_t* n_cached_out);
+int pkv_prefix_cache_stats(const pkv_allocator* a, pkv_prefix_stats* out);
+
 /* Preemption.  pkv_seq_swap_out lists the sequence's blocks in logical
  * order in blocks_out (HOST int32 [cap]; *n_out = count), for
  * swap_blocks_out.  It then releases them like pkv_seq_free, but the

@@ -32,6 +32,15 @@ Policy choices the pages leave open (the product follows the same ones):
   last holder (count == 1) writes in place.
 * An operation that cannot get every block it needs fails with
   ``OutOfBlocks`` and changes nothing.
+* Prefix cache ("Prefix Caching": a system prompt shared by many requests
+  is stored once; "PagedAttention & Continuous Batching...", item 5).
+  ``append_prompt`` walks a new request's full prompt blocks in order and
+  reuses every leading block whose identity -- (block before it, that
+  block's generation, its own token ids) -- is cached; from the first miss
+  on it takes fresh blocks and caches each new full block.  A cached block
+  whose count drops to zero stays findable; it is handed out again, least
+  recently released first, only when no never-cached block is free.  The
+  generation of a block grows each time it is handed out.
 * Swapping a sequence out ("vLLM Architecture": the scheduler preempts
   low-priority requests by swapping their blocks to CPU memory) reports its
   blocks in logical order, then releases them like ``free``.  The sequence
@@ -41,6 +50,8 @@ Policy choices the pages leave open (the product follows the same ones):
 """
 
 from __future__ import annotations
+
+from collections import OrderedDict
 
 
 def slot_for_position(block_table, position: int, block_size: int) -> int:
@@ -70,14 +81,23 @@ class AllocatorModel:
         self._free = list(reversed(order))
         self._ref = [0] * num_blocks
         self._seqs: dict[int, dict] = {}
+        self._cache: dict = {}          # (parent, parent_gen, tokens) -> block
+        self._key_of: dict = {}         # block -> its key
+        self._gen = [0] * num_blocks
+        self._lru: OrderedDict = OrderedDict()   # cached, unused blocks; first = evicted first
+        self._counts = {"prompts": 0, "prompts_with_hits": 0, "hit_tokens": 0, "evictions": 0}
 
     # --- queries -------------------------------------------------------
     def num_free(self) -> int:
-        return len(self._free)
+        return len(self._free) + len(self._lru)
 
     def free_list(self) -> list[int]:
-        """Free blocks in the order they will be handed out."""
-        return list(reversed(self._free))
+        """Free blocks in the order they will be handed out (never-cached
+        blocks first, then cached unused blocks, least recently released first)."""
+        return list(reversed(self._free)) + list(self._lru)
+
+    def prefix_stats(self) -> dict:
+        return {"cached_blocks": len(self._cache), "evictable_blocks": len(self._lru), **self._counts}
 
     def refcount(self, block: int) -> int:
         return self._ref[block]
@@ -92,8 +112,8 @@ class AllocatorModel:
         frag = sum(len(s["blocks"]) * self.block_size - s["ntok"] for s in self._seqs.values() if not s["swapped"])
         return {
             "num_blocks": self.num_blocks,
-            "free_blocks": len(self._free),
-            "used_blocks": self.num_blocks - len(self._free),
+            "free_blocks": self.num_free(),
+            "used_blocks": self.num_blocks - self.num_free(),
             "shared_blocks": sum(1 for r in self._ref if r > 1),
             "num_seqs": len(self._seqs),
             "num_tokens": sum(s["ntok"] for s in self._seqs.values()),
@@ -107,9 +127,23 @@ class AllocatorModel:
         return self._seqs[seq]
 
     def _pop(self) -> int:
-        b = self._free.pop()
+        if self._free:
+            b = self._free.pop()
+        else:                                   # evict the least recently released cached block
+            b, _ = self._lru.popitem(last=False)
+            del self._cache[self._key_of.pop(b)]
+            self._counts["evictions"] += 1
+        self._gen[b] += 1
         self._ref[b] = 1
         return b
+
+    def _decref(self, b: int) -> None:
+        self._ref[b] -= 1
+        if self._ref[b] == 0:
+            if b in self._key_of:
+                self._lru[b] = None             # keep its contents findable
+            else:
+                self._free.append(b)
 
     def _needs(self, seq: dict, n: int) -> int:
         """Blocks an append of n tokens takes from the free list."""
@@ -127,7 +161,7 @@ class AllocatorModel:
         if n > 0 and ntok % B != 0 and self._ref[blocks[-1]] > 1:
             src = blocks[-1]
             dst = self._pop()
-            self._ref[src] -= 1
+            self._decref(src)
             blocks[-1] = dst
             cow = (src, dst)
         slots = []
@@ -158,9 +192,7 @@ class AllocatorModel:
         s = self._live(seq)
         blocks = list(s["blocks"])
         for b in reversed(blocks):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
+            self._decref(b)
         s["blocks"] = []
         s["swapped"] = True
         s["nswap"] = len(blocks)
@@ -172,7 +204,7 @@ class AllocatorModel:
         if not s["swapped"]:
             raise InvalidArgument(f"sequence {seq} is not swapped out")
         n = s["nswap"]
-        if n > len(self._free):
+        if n > self.num_free():
             raise OutOfBlocks()
         s["blocks"] = [self._pop() for _ in range(n)]
         s["swapped"] = False
@@ -184,16 +216,55 @@ class AllocatorModel:
         if n < 0:
             raise InvalidArgument("negative token count")
         s = self._live(seq)
-        if self._needs(s, n) > len(self._free):
+        if self._needs(s, n) > self.num_free():
             raise OutOfBlocks()
         return self._append(s, n)
+
+    def append_prompt(self, seq: int, tokens):
+        """Prompt of a new request: (slots with -1 for cached tokens, n_cached)."""
+        tokens = [int(t) for t in tokens]
+        s = self._live(seq)
+        if s["blocks"] or s["ntok"]:
+            raise InvalidArgument("append_prompt needs an empty sequence")
+        B, n = self.block_size, len(tokens)
+        nfull = n // B
+        hit, parent, pgen = [], -1, 0
+        for k in range(nfull):
+            key = (parent, pgen, tuple(tokens[k * B:(k + 1) * B]))
+            if key not in self._cache:
+                break
+            b = self._cache[key]
+            hit.append(b)
+            parent, pgen = b, self._gen[b]
+        revived = sum(1 for b in hit if self._ref[b] == 0)
+        if -(-n // B) - len(hit) > self.num_free() - revived:
+            raise OutOfBlocks()
+        if nfull:
+            self._counts["prompts"] += 1
+            self._counts["prompts_with_hits"] += 1 if hit else 0
+        for b in hit:
+            if self._ref[b] == 0:
+                del self._lru[b]
+            self._ref[b] += 1
+        s["blocks"] = list(hit)
+        cached = len(hit) * B
+        self._counts["hit_tokens"] += cached
+        s["ntok"] = cached
+        slots, _ = self._append(s, n - cached)
+        for k in range(len(hit), nfull):
+            b = s["blocks"][k]
+            par = s["blocks"][k - 1] if k else -1
+            key = (par, self._gen[par] if par >= 0 else 0, tuple(tokens[k * B:(k + 1) * B]))
+            self._cache[key] = b
+            self._key_of[b] = key
+        return [-1] * cached + slots, cached
 
     def append_one_batch(self, seqs):
         """One new token for each sequence, in order: (slots, cow_pairs)."""
         if len(set(seqs)) != len(seqs):
             raise InvalidArgument("a sequence is named twice")
         recs = [self._live(q) for q in seqs]
-        if sum(self._needs(r, 1) for r in recs) > len(self._free):
+        if sum(self._needs(r, 1) for r in recs) > self.num_free():
             raise OutOfBlocks()
         slots, pairs = [], []
         for r in recs:
@@ -206,9 +277,7 @@ class AllocatorModel:
     def free(self, seq: int) -> None:
         s = self._seq(seq)
         for b in reversed(s["blocks"]):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
+            self._decref(b)
         del self._seqs[seq]
 
     def fork(self, parent: int, child: int) -> None:

@@ -51,6 +51,8 @@ _SIGS = {
     "block_copy": ([P, P, P, I32, I32, I32, I32, I32, I32, P], ctypes.c_int),
     "swap_blocks_out": ([P, P, P, I32, P, P, I32, I32, I32, I32, I32, P], ctypes.c_int),
     "swap_blocks_in": ([P, P, P, I32, P, P, I32, I32, I32, I32, I32, P], ctypes.c_int),
+    "pkv_seq_append_prompt": ([P, I64, P, I32, P, P], ctypes.c_int),
+    "pkv_prefix_cache_stats": ([P, P], ctypes.c_int),
     "pkv_seq_swap_out": ([P, I64, P, I32, P], ctypes.c_int),
     "pkv_seq_swap_in": ([P, I64, P, I32, P], ctypes.c_int),
     "pkv_seq_is_swapped": ([P, I64, P], ctypes.c_int),

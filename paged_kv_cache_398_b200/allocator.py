@@ -20,6 +20,12 @@ class AllocStats(ctypes.Structure):
                 ("fragmentation_tokens", ctypes.c_int64)]
 
 
+class PrefixStats(ctypes.Structure):
+    _fields_ = [("cached_blocks", ctypes.c_int32), ("evictable_blocks", ctypes.c_int32),
+                ("prompts", ctypes.c_int64), ("prompts_with_hits", ctypes.c_int64),
+                ("hit_tokens", ctypes.c_int64), ("evictions", ctypes.c_int64)]
+
+
 class OutOfBlocks(PagedKVError):
     pass
 
@@ -119,6 +125,22 @@ class BlockAllocator:
         _check("pkv_batch_tables", self._L.pkv_batch_tables(
             self._h, ids.data_ptr(), S, tables.data_ptr(), max_blocks_per_seq, pad, lens.data_ptr()))
         return tables[:S], lens[:S]
+
+    def append_prompt(self, seq: int, tokens):
+        """Prompt of a new (empty) sequence, reusing cached prefix blocks.
+        Returns (slots int64 tensor with -1 for cached tokens, n_cached)."""
+        t = torch.as_tensor(tokens, dtype=torch.int32).reshape(-1).contiguous()
+        n = t.numel()
+        slots = torch.empty(max(n, 1), dtype=torch.int64)
+        cached = ctypes.c_int32(0)
+        _check("pkv_seq_append_prompt", self._L.pkv_seq_append_prompt(
+            self._h, seq, t.data_ptr() if n else None, n, slots.data_ptr(), ctypes.byref(cached)))
+        return slots[:n], int(cached.value)
+
+    def prefix_stats(self) -> dict:
+        st = PrefixStats()
+        _check("pkv_prefix_cache_stats", self._L.pkv_prefix_cache_stats(self._h, ctypes.byref(st)))
+        return {name: int(getattr(st, name)) for name, _ in PrefixStats._fields_}
 
     def swap_out(self, seq: int) -> list:
         """Release a sequence's blocks for preemption; returns them (logical

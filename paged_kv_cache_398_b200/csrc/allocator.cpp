@@ -14,6 +14,7 @@
 // The policy choices the pages leave open are stated in include/paged_kv.h.
 #include <algorithm>
 #include <cstring>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -29,6 +30,27 @@ struct Seq {
     int32_t nswap = 0;     // how many
 };
 
+// Identity of a cached full block: the block it follows (and that block's
+// generation, so a reused id never matches stale children) plus its tokens.
+// Equal keys mean equal prefixes, compared exactly.
+struct BlockKey {
+    int32_t parent;    // -1 for the first block of a prompt
+    uint32_t pgen;
+    std::vector<int32_t> toks;
+    bool operator==(const BlockKey& o) const { return parent == o.parent && pgen == o.pgen && toks == o.toks; }
+};
+
+struct BlockKeyHash {
+    size_t operator()(const BlockKey& k) const
+    {
+        uint64_t h = 0x9e3779b97f4a7c15ull ^ (uint64_t)(uint32_t)k.parent ^ ((uint64_t)k.pgen << 32);
+        for (int32_t t : k.toks) {
+            h ^= (uint64_t)(uint32_t)t + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+        }
+        return (size_t)h;
+    }
+};
+
 }  // namespace
 
 struct pkv_allocator {
@@ -38,24 +60,53 @@ struct pkv_allocator {
     std::vector<int32_t> ref;         // reference count per block
     std::unordered_map<int64_t, Seq> seqs;
     int32_t shared = 0;               // blocks with ref > 1
+    // prefix cache: full prompt blocks findable by content
+    std::unordered_map<BlockKey, int32_t, BlockKeyHash> cache;
+    std::vector<BlockKey> key_of;     // per block; toks empty = not cached
+    std::vector<uint32_t> gen;        // per block; +1 each time it is handed out
+    std::list<int32_t> lru;           // cached blocks with ref 0, least recently released first
+    std::vector<std::list<int32_t>::iterator> lru_pos;
+    std::vector<char> in_lru;
+    int64_t lookups = 0, hits = 0, hit_tokens = 0, evictions = 0;
 
+    int64_t available() const { return (int64_t)free_stack.size() + (int64_t)lru.size(); }
     int32_t pop()
     {
-        int32_t b = free_stack.back();
-        free_stack.pop_back();
+        int32_t b;
+        if (!free_stack.empty()) {
+            b = free_stack.back();
+            free_stack.pop_back();
+        } else {  // evict the least recently released cached block
+            b = lru.front();
+            lru.pop_front();
+            in_lru[b] = 0;
+            cache.erase(key_of[b]);
+            key_of[b].toks.clear();
+            ++evictions;
+        }
+        ++gen[b];
         ref[b] = 1;
         return b;
     }
     void incref(int32_t b)
     {
+        if (ref[b] == 0 && in_lru[b]) {  // a cached block comes back into use
+            lru.erase(lru_pos[b]);
+            in_lru[b] = 0;
+        }
         if (++ref[b] == 2) ++shared;
     }
-    // returns true when the block became free
+    // returns true when the block stopped being used
     bool decref(int32_t b)
     {
         if (ref[b]-- == 2) --shared;
         if (ref[b] == 0) {
-            free_stack.push_back(b);
+            if (!key_of[b].toks.empty()) {  // keep its contents findable until evicted
+                lru_pos[b] = lru.insert(lru.end(), b);
+                in_lru[b] = 1;
+            } else {
+                free_stack.push_back(b);
+            }
             return true;
         }
         return false;
@@ -121,6 +172,10 @@ int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* init
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->ref.assign(num_blocks, 0);
+    a->key_of.assign(num_blocks, BlockKey{-1, 0, {}});
+    a->gen.assign(num_blocks, 0);
+    a->lru_pos.resize(num_blocks);
+    a->in_lru.assign(num_blocks, 0);
     a->free_stack.resize(num_blocks);
     if (initial_order) {
         std::vector<char> seen(num_blocks, 0);
@@ -155,7 +210,7 @@ int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slo
     if (!a || n < 0) return PKV_ERR_INVALID_ARG;
     Seq* s = a->live(seq);
     if (!s) return PKV_ERR_INVALID_ARG;
-    if (a->needs(*s, n) > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (a->needs(*s, n) > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
     a->append(*s, n, slots_out, cow_pair_out, cow_out);
     return PKV_OK;
 }
@@ -176,7 +231,7 @@ int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
         std::sort(ids.begin(), ids.end());
         if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PKV_ERR_INVALID_ARG;
     }
-    if (need > (int64_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (need > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
     int32_t ncow = 0;
     for (int32_t i = 0; i < n_seqs; ++i) {
         int64_t pair[2];
@@ -274,15 +329,18 @@ int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs
     return PKV_OK;
 }
 
-int32_t pkv_num_free(const pkv_allocator* a) { return a ? (int32_t)a->free_stack.size() : -1; }
+int32_t pkv_num_free(const pkv_allocator* a) { return a ? (int32_t)a->available() : -1; }
 
 int pkv_free_list(const pkv_allocator* a, int32_t* out, int32_t cap, int32_t* n_out)
 {
     if (!a) return PKV_ERR_INVALID_ARG;
-    int32_t n = (int32_t)a->free_stack.size();
+    const int32_t ns = (int32_t)a->free_stack.size();
+    const int32_t n = (int32_t)a->available();
     if (n_out) *n_out = n;
     if (n > cap || (n > 0 && !out)) return PKV_ERR_INVALID_ARG;
-    for (int32_t i = 0; i < n; ++i) out[i] = a->free_stack[n - 1 - i];
+    for (int32_t i = 0; i < ns; ++i) out[i] = a->free_stack[ns - 1 - i];
+    int32_t i = ns;
+    for (int32_t b : a->lru) out[i++] = b;  // then the cached blocks, in eviction order
     return PKV_OK;
 }
 
@@ -296,7 +354,7 @@ int pkv_alloc_get_stats(const pkv_allocator* a, pkv_alloc_stats* out)
 {
     if (!a || !out) return PKV_ERR_INVALID_ARG;
     out->num_blocks = a->num_blocks;
-    out->free_blocks = (int32_t)a->free_stack.size();
+    out->free_blocks = (int32_t)a->available();
     out->used_blocks = a->num_blocks - out->free_blocks;
     out->shared_blocks = a->shared;
     out->num_seqs = (int64_t)a->seqs.size();
@@ -307,6 +365,66 @@ int pkv_alloc_get_stats(const pkv_allocator* a, pkv_alloc_stats* out)
     }
     out->num_tokens = tok;
     out->fragmentation_tokens = frag;
+    return PKV_OK;
+}
+
+int pkv_seq_append_prompt(pkv_allocator* a, int64_t seq, const int32_t* token_ids, int32_t n,
+                          int64_t* slots_out, int32_t* n_cached_out)
+{
+    if (!a || n < 0 || (n > 0 && !token_ids)) return PKV_ERR_INVALID_ARG;
+    Seq* s = a->live(seq);
+    if (!s || !s->blocks.empty() || s->ntok != 0) return PKV_ERR_INVALID_ARG;
+    const int32_t B = a->block_size;
+    const int32_t nfull = n / B;
+    // leading full blocks already cached, walked in order
+    std::vector<int32_t> hit;
+    int32_t parent = -1;
+    uint32_t pgen = 0;
+    int32_t revived = 0;  // hits now resting in the LRU list (not available to others)
+    for (int32_t k = 0; k < nfull; ++k) {
+        BlockKey key{parent, pgen, std::vector<int32_t>(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B)};
+        auto it = a->cache.find(key);
+        if (it == a->cache.end()) break;
+        hit.push_back(it->second);
+        if (a->ref[it->second] == 0) ++revived;
+        parent = it->second;
+        pgen = a->gen[parent];
+    }
+    const int64_t fresh = (int64_t)(n + B - 1) / B - (int64_t)hit.size();
+    if (fresh > a->available() - revived) return PKV_ERR_OUT_OF_BLOCKS;
+    a->lookups += nfull > 0 ? 1 : 0;
+    a->hits += hit.empty() ? 0 : 1;
+    for (int32_t b : hit) {
+        a->incref(b);
+        s->blocks.push_back(b);
+    }
+    const int32_t cached = (int32_t)hit.size() * B;
+    a->hit_tokens += cached;
+    s->ntok = cached;
+    for (int32_t i = 0; i < cached && slots_out; ++i) slots_out[i] = -1;
+    a->append(*s, n - cached, slots_out ? slots_out + cached : nullptr, nullptr, nullptr);
+    // make this prompt's new full blocks findable by the next request
+    for (int32_t k = (int32_t)hit.size(); k < nfull; ++k) {
+        const int32_t b = s->blocks[k];
+        const int32_t par = k == 0 ? -1 : s->blocks[k - 1];
+        BlockKey key{par, par < 0 ? 0u : a->gen[par],
+                     std::vector<int32_t>(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B)};
+        a->key_of[b] = key;
+        a->cache.emplace(std::move(key), b);
+    }
+    if (n_cached_out) *n_cached_out = cached;
+    return PKV_OK;
+}
+
+int pkv_prefix_cache_stats(const pkv_allocator* a, pkv_prefix_stats* out)
+{
+    if (!a || !out) return PKV_ERR_INVALID_ARG;
+    out->cached_blocks = (int32_t)a->cache.size();
+    out->evictable_blocks = (int32_t)a->lru.size();
+    out->prompts = a->lookups;
+    out->prompts_with_hits = a->hits;
+    out->hit_tokens = a->hit_tokens;
+    out->evictions = a->evictions;
     return PKV_OK;
 }
 
@@ -334,7 +452,7 @@ int pkv_seq_swap_in(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t 
     const int32_t n = s->nswap;
     if (n_out) *n_out = n;
     if (n > cap || (n > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
-    if (n > (int32_t)a->free_stack.size()) return PKV_ERR_OUT_OF_BLOCKS;
+    if (n > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
     for (int32_t i = 0; i < n; ++i) s->blocks.push_back(a->pop());
     if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
     s->swapped = false;

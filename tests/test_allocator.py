@@ -32,6 +32,7 @@ def _same(a: pkv.BlockAllocator, m: AllocatorModel, seqs):
     st, sm = a.stats(), m.stats()
     for k in sm:
         assert st[k] == sm[k], k
+    assert a.prefix_stats() == m.prefix_stats()
 
 
 def test_worked_examples_native():
@@ -272,3 +273,71 @@ def test_swap_kernels_reject_bad_lists_on_host():
         t = torch.tensor(ids, dtype=torch.int64)
         rc = getattr(L, fn)(p, p, t.data_ptr(), t.numel(), p, p, 2, 64, 16, 8, C["PKV_F16"], None)
         assert rc == C["PKV_ERR_INVALID_ARG"], (ids, fn)
+
+
+def test_prefix_cache_golden_native():
+    gold = load_golden("prefix_sharing.json")
+    B = gold["block_size"]
+    system = list(range(1000, 1000 + len(gold["prefix_blocks"]) * B))
+    a = pkv.BlockAllocator(5000, B)
+    for u in range(gold["users"]):
+        a.add(u)
+        slots, cached = a.append_prompt(u, system + [7, u % 97, u // 97, 3])
+        assert cached == (0 if u == 0 else len(system))
+        assert (slots[:cached] == -1).all()
+    pre = a.block_table(0)[:len(gold["prefix_blocks"])]
+    assert all(a.refcount(b) == gold["users"] for b in pre)
+    assert a.stats()["used_blocks"] == gold["blocks_with_sharing"] + gold["users"]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_prefix_cache_random_prompts_match_model(seed):
+    """Prompts drawn from a few shared system prompts, in a pool small
+    enough to force evictions; every step compared with the model."""
+    rng = random.Random(100 + seed)
+    B, NB = 16, 60
+    a = pkv.BlockAllocator(NB, B)
+    m = AllocatorModel(NB, B)
+    systems = [[rng.randrange(50) for _ in range(rng.choice([16, 32, 40, 64]))] for _ in range(3)]
+    live, sid = [], 0
+    for step in range(300):
+        r = rng.random()
+        if r < 0.45 or not live:
+            toks = list(rng.choice(systems)) + [rng.randrange(50) for _ in range(rng.randrange(0, 40))]
+            m.add(sid)
+            a.add(sid)
+            try:
+                want = m.append_prompt(sid, toks)
+            except OutOfBlocks:
+                with pytest.raises(pkv.OutOfBlocks):
+                    a.append_prompt(sid, toks)
+                m.free(sid)
+                a.free(sid)
+            else:
+                slots, cached = a.append_prompt(sid, toks)
+                assert (slots.tolist(), cached) == want
+                live.append(sid)
+            sid += 1
+        elif r < 0.75:
+            s = rng.choice(live)
+            m.free(s)
+            a.free(s)
+            live.remove(s)
+        elif r < 0.9:
+            s = rng.choice(live)
+            n = rng.choice([1, 5, 17])
+            try:
+                want = m.append_tokens(s, n)
+            except OutOfBlocks:
+                with pytest.raises(pkv.OutOfBlocks):
+                    a.append_tokens(s, n)
+            else:
+                assert a.append_tokens(s, n) == (want[0], want[1])
+        else:
+            s = rng.choice(live)
+            m.fork(s, sid)
+            a.fork(s, sid)
+            live.append(sid)
+            sid += 1
+        _same(a, m, live)
+    assert m.prefix_stats()["evictions"] > 0 and m.prefix_stats()["hit_tokens"] > 0

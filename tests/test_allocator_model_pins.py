@@ -156,3 +156,50 @@ def test_out_of_blocks_changes_nothing():
         m.add(0)
     with pytest.raises(InvalidArgument):
         m.free(7)
+
+
+def test_prefix_cache_found_by_lookup():
+    """The page's prefix example, with the sharing found by content: every
+    request brings the same 64-token system prompt and its own question."""
+    gold = load_golden("prefix_sharing.json")
+    B = gold["block_size"]
+    system = list(range(1000, 1000 + len(gold["prefix_blocks"]) * B))
+    m = AllocatorModel(5000, B)
+    for u in range(gold["users"]):
+        m.add(u)
+        question = [7, u % 97, u // 97, 3]
+        slots, cached = m.append_prompt(u, system + question)
+        assert cached == (0 if u == 0 else len(system))
+        assert slots[:cached] == [-1] * cached
+    pre = m.block_table(0)[:len(gold["prefix_blocks"])]
+    assert all(m.refcount(b) == gold["users"] for b in pre)
+    assert all(m.block_table(u)[:len(pre)] == pre for u in range(gold["users"]))
+    # each user: 4 shared system blocks + 1 private block for the question
+    assert m.stats()["used_blocks"] == gold["blocks_with_sharing"] + gold["users"]
+    assert m.prefix_stats()["hit_tokens"] == (gold["users"] - 1) * len(system)
+
+
+def test_prefix_cache_keeps_released_blocks_and_evicts_lru():
+    B = 16
+    m = AllocatorModel(6, B)                   # hands out 0, 1, 2, ...
+    p1 = list(range(48))                       # 3 full blocks
+    m.add(0)
+    m.append_prompt(0, p1)                     # blocks 0, 1, 2, all cached
+    m.free(0)                                  # released 2, 1, 0: all stay findable
+    assert m.num_free() == 6 and m.prefix_stats()["evictable_blocks"] == 3
+    assert m.free_list() == [3, 4, 5, 2, 1, 0]  # never-cached first, then least recently released
+    m.add(1)
+    _, cached = m.append_prompt(1, p1[:32] + [99] * 16)   # blocks 0, 1 hit; third differs -> block 3
+    assert cached == 32 and m.block_table(1) == [0, 1, 3]
+    assert m.prefix_stats()["evictable_blocks"] == 1       # block 2 still findable
+    m.add(2)
+    m.append_tokens(2, 32)                     # blocks 4, 5: the last never-cached ones
+    assert m.prefix_stats()["evictions"] == 0
+    m.add(3)
+    m.append_tokens(3, 1)                      # nothing else free: block 2 is evicted
+    assert m.block_table(3) == [2] and m.prefix_stats()["evictions"] == 1
+    m.free(2)
+    m.add(4)
+    _, cached = m.append_prompt(4, p1)
+    assert cached == 32                        # the evicted third block no longer matches
+    assert m.block_table(4)[:2] == [0, 1]

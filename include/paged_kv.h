@@ -301,6 +301,16 @@ int pkv_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
  */
 int pkv_device_status(int32_t device, int32_t* flags_out, int32_t clear);
 
+/*
+ * pkv_debug_wait_timeout -- test hook for failure detection.  It launches
+ * one warp that waits, through the same bounded wait the decode kernels
+ * use, on an mbarrier that nothing arrives on.  After limit_ns nanoseconds
+ * (at most 1 s) the wait gives up and sets PKV_DEV_WAIT_TIMEOUT in the
+ * status word.  The kernel then exits normally and the context stays
+ * usable.  It never hangs and never faults.
+ */
+int pkv_debug_wait_timeout(int64_t limit_ns, void* stream);
+
 /* The last cudaError_t seen by any call in this thread, as an int. */
 int pkv_last_cuda_error(void);
 

@@ -59,6 +59,7 @@ _SIGS = {
     "pkv_slot_mapping": ([P, I32, P, I32, I32, P], ctypes.c_int),
     "pkv_device_status": ([I32, P, I32], ctypes.c_int),
     "pkv_last_cuda_error": ([], ctypes.c_int),
+    "pkv_debug_wait_timeout": ([I64, P], ctypes.c_int),
     "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "pkv_alloc_create": ([I32, I32, P, P], ctypes.c_int),
     "pkv_alloc_destroy": ([P], None),

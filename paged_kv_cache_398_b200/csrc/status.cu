@@ -43,7 +43,41 @@ int* status_word_for_current_device()
 
 }  // namespace pkv
 
+namespace {
+
+// One warp waits, with the kernels' own bounded wait, on an mbarrier that
+// nothing ever arrives on.  The wait gives up after limit_ns and records
+// PKV_DEV_WAIT_TIMEOUT, exactly as a decode kernel would if its copies
+// never landed.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int* status, int* gave_up)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        pkv::mbar_init(&bar, 1);
+        pkv::fence_mbar_init();
+    }
+    __syncwarp();
+    if (!pkv::mbar_wait(&bar, 0, limit_ns)) {
+        if (threadIdx.x == 0) {
+            pkv::raise_flag(status, PKV_DEV_WAIT_TIMEOUT);
+            if (gave_up) *gave_up = 1;
+        }
+    }
+}
+
+}  // namespace
+
 extern "C" {
+
+int pkv_debug_wait_timeout(int64_t limit_ns, void* stream)
+{
+    if (limit_ns < 0 || limit_ns > 1000000000ll) return PKV_ERR_INVALID_ARG;
+    int* status = pkv::status_word_for_current_device();
+    if (!status) return PKV_ERR_CUDA;
+    wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_ns, status, nullptr);
+    return pkv::check_launch();
+}
+
 
 int pkv_device_status(int32_t device, int32_t* flags_out, int32_t clear)
 {

@@ -348,3 +348,17 @@ def test_many_copy_pairs_span_launches():
     torch.cuda.synchronize()
     assert torch.equal(kc[1300:], k0[:1300]) and torch.equal(vc[1300:], v0[:1300])
     assert torch.equal(kc[:1300], k0[:1300])
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait on a barrier nothing arrives on gives up after its limit and
+    reports PKV_DEV_WAIT_TIMEOUT; the GPU keeps working afterwards."""
+    import ctypes
+    L = pkv._lib.lib()
+    t0 = __import__("time").perf_counter()
+    assert L.pkv_debug_wait_timeout(20_000_000, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    flags = pkv.pkv_device_status(0)
+    waited = __import__("time").perf_counter() - t0
+    assert flags & pkv._lib.C["PKV_DEV_WAIT_TIMEOUT"]
+    assert 0.015 < waited < 5.0
+    _run_full_parity(make_workload(1))

@@ -58,7 +58,7 @@ def decode_source_hash() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str, num_seqs: int, path: str):
+def recorded_traffic(workload: str, num_seqs: int, path: str, block_size: int):
     """DRAM bytes per decode call from the committed ncu record, or None if
     there is none for this workload or the decode sources changed since."""
     try:
@@ -68,7 +68,8 @@ def recorded_traffic(workload: str, num_seqs: int, path: str):
         return None
     if rec.get("source_sha256") != decode_source_hash():
         return None
-    if rec.get("workload") != workload or rec.get("num_seqs") != num_seqs or rec.get("path") != path:
+    if (rec.get("workload"), rec.get("num_seqs"), rec.get("path"), rec.get("block_size")) != \
+            (workload, num_seqs, path, block_size):
         return None
     return rec.get("dram_bytes_per_call")
 
@@ -89,7 +90,7 @@ class Step:
     """Everything one decode step needs, resident on the GPU."""
 
 
-def build_step(number: int, device, rank: int = 0, num_seqs=None):
+def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16):
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 
@@ -97,7 +98,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None):
     kw = {}
     if num_seqs:
         kw = {"num_prompts": max(1, num_seqs // 4)} if number == 5 else {"num_seqs": num_seqs}
-    w = make_workload(number, device=device, seed=seed, **kw)   # lengths on host, values on the GPU
+    w = make_workload(number, device=device, seed=seed, block_size=block_size, **kw)   # lengths on host, values on the GPU
     S = w.num_seqs
     st = Step()
     st.w = w
@@ -124,7 +125,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None):
                 alloc.append_prompt(s, torch.cat([system, own]))
             st.admit_us_per_request = (time.perf_counter() - t0) * 1e6 / S
             st.prefix = alloc.prefix_stats()
-            assert st.prefix["hit_tokens"] == 64 * (S - 1)
+            assert st.prefix["hit_tokens"] == 64 * (S - 1)     # every request found the system prompt
         else:
             for s in range(S):
                 alloc.add(s)
@@ -377,6 +378,30 @@ def run_reference(args):
     return 0
 
 
+def fragmentation_report(lens, max_len: int = 8192):
+    """Internal fragmentation of the batch's contexts under paged allocation
+    with block sizes 8, 16 and 32 (the native allocator's own count: empty
+    slots in each sequence's last block), against one contiguous
+    reservation of max_len tokens per request."""
+    import paged_kv_cache_398_b200 as pkv
+    lens = [int(n) for n in lens]
+    total = sum(lens)
+    rep = {}
+    for bs in (8, 16, 32):
+        need = sum(-(-n // bs) for n in lens)
+        a = pkv.BlockAllocator(need, bs)
+        for i, n in enumerate(lens):
+            a.add(i)
+            a.append_tokens(i, n)
+        st = a.stats()
+        held = st["used_blocks"] * bs
+        rep[f"block_{bs}"] = {"waste_tokens": st["fragmentation_tokens"],
+                              "waste_pct": 100.0 * st["fragmentation_tokens"] / held,
+                              "max_waste_per_seq": bs - 1}
+    rep["contiguous_max_len"] = {"max_len": max_len, "waste_pct": 100.0 * (1 - total / (max_len * len(lens)))}
+    return rep
+
+
 def measure_swap(st, dev, nblocks: int = 2048, iters: int = 10):
     """Preemption traffic: swap_blocks_out / swap_blocks_in of nblocks blocks
     of this workload's cache (then back into the same blocks, so the cache
@@ -448,7 +473,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    st = build_step(args.workload, dev, rank, args.num_seqs)
+    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size)
     st.path = args.path
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
@@ -546,7 +571,7 @@ def run_ours(args):
                                 "paged_attention_decode (partition kernel + split-K reduce)"),
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path),
+                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path, st.w.block_size),
                      "algorithmic_bytes_per_launch": call_bytes},
         "cpu_baseline": ({k: v for k, v in base.items() if k != "seconds"} if base else None),
         "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
@@ -560,6 +585,7 @@ def run_ours(args):
                           "cached_blocks": st.prefix["cached_blocks"]}),
         "clocks": clk,
         "swap": swap,
+        "fragmentation": fragmentation_report(st.lens_host),
         "wall_s_timed": t_wall1 - t_wall0,
     }
     print(json.dumps(line), flush=True)
@@ -575,6 +601,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-swap", action="store_true", help="skip the swap-out / swap-in measurement")
+    ap.add_argument("--block-size", type=int, default=16, choices=[8, 16, 32],
+                    help="tokens per block (the pages use 16)")
     ap.add_argument("--path", choices=["fused", "separate"], default="fused",
                     help="fused: slot write inside the decode launch; separate: paged_kv_write then decode")
     ap.add_argument("--reference-seqs", type=int, default=16)

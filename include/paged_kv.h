@@ -36,10 +36,11 @@
  *    the kernels.  A kernel never reads or writes outside the buffers
  *    described here: it skips the bad item and sets a flag in a sticky
  *    per-device status word, which pkv_device_status reads.
- *  - Supported decode shapes: block_size 16, head_dim 64 or 128,
- *    num_q_heads / num_kv_heads in {1, 2, 4, 8}.  Element type fp32, fp16
- *    or bf16, with fp32 accumulation.  Other shapes return
- *    PKV_ERR_UNSUPPORTED.
+ *  - Supported decode shapes: block_size 8, 16 or 32 (16 is the pages'
+ *    choice), head_dim 64 or 128, num_q_heads / num_kv_heads in
+ *    {1, 2, 4, 8}.  Element type fp32, fp16 or bf16, with fp32
+ *    accumulation.  Other shapes return PKV_ERR_UNSUPPORTED.  The slot
+ *    write, block copy, swap and allocator take any block size.
  */
 #ifndef PAGED_KV_H
 #define PAGED_KV_H

@@ -40,9 +40,10 @@
 
 namespace {
 
-constexpr int kBlock = 16;
+constexpr int kTile = 16;                          // tokens per compute tile
 constexpr int kPartTokens = PKV_PARTITION_TOKENS;
-constexpr int kPartBlocks = kPartTokens / kBlock;
+constexpr int kPartTiles = kPartTokens / kTile;    // tiles per partition
+constexpr int kMaxPartBlocks = kPartTokens / 8;    // blocks per partition at the smallest block size
 constexpr int kWarps = 4;
 constexpr int kStages = 2;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
@@ -52,10 +53,10 @@ struct Cfg {
     static constexpr int kVec = 16 / (int)sizeof(T);   // elements per 16 bytes
     static constexpr int kLpt = D / kVec;              // lanes per token row
     static constexpr int kTpi = 32 / kLpt;             // tokens per warp iteration
-    static constexpr int kIters = kBlock / kTpi;       // iterations per block
-    static constexpr int kTileBytes = kBlock * D * (int)sizeof(T);
-    static constexpr int kNv = kIters * G;             // partial dots per lane per block
-    static constexpr int kItems = kBlock * G;          // scores per block
+    static constexpr int kIters = kTile / kTpi;        // iterations per tile
+    static constexpr int kTileBytes = kTile * D * (int)sizeof(T);
+    static constexpr int kNv = kIters * G;             // partial dots per lane per tile
+    static constexpr int kItems = kTile * G;           // scores per tile
     static constexpr int kItemsPerLane = (kItems + 31) / 32;
     static_assert(kLpt >= 1 && kLpt <= 32 && 32 % kLpt == 0, "bad row split");
     static_assert(32 % G == 0, "G must divide the warp");
@@ -64,7 +65,7 @@ struct Cfg {
     static constexpr int kBarOff = kTilesBytes;
     static constexpr int kScoreOff = kBarOff + kWarps * kStages * 8;
     static constexpr int kBlkOff = kScoreOff + kWarps * kItems * 4;
-    static constexpr int kSmemBytes = kBlkOff + kPartBlocks * 4;
+    static constexpr int kSmemBytes = kBlkOff + kMaxPartBlocks * 4;
     // the cross-warp merge reuses the tile area
     static constexpr int kMergeBytes = kWarps * G * (D + 2) * 4;
     static_assert(kMergeBytes <= kTilesBytes, "merge area does not fit");
@@ -119,17 +120,52 @@ __host__ __device__ constexpr int treduce_dup_mask()
     }
 }
 
-// Lane 0 of a warp: fetch the K and V tiles at element offset `off` into the
-// tile pair at `dst` (K then V), completing on `bar`.
+// A compute tile is 16 consecutive token positions of a sequence.  With
+// block size B it is one block (B = 16), half of one (B = 32) or two
+// consecutive ones (B = 8).  tile_rows gives the cache rows, in units of
+// one token of one kv head (row = (block * Hkv + h) * B + offset), where the
+// tile's first and second 8 tokens start.  For B = 16 and 32 the second half
+// follows the first (r1 = r0 + 8).  nbp is the number of blocks this
+// partition has, and a missing second block of a B = 8 tile reads the last
+// one again (those positions are past the length and masked).
+template <int B>
+__device__ __forceinline__ void tile_rows(const int32_t* s_blk, int nbp, int tile, int num_kv_heads, int h,
+                                          int& r0, int& r1)
+{
+    static_assert(B == 8 || B == 16 || B == 32, "block size 8, 16 or 32");
+    if constexpr (B == 16) {
+        r0 = (max(s_blk[tile], 0) * num_kv_heads + h) * 16;
+        r1 = r0 + 8;
+    } else if constexpr (B == 32) {
+        r0 = (max(s_blk[tile / 2], 0) * num_kv_heads + h) * 32 + (tile % 2) * 16;
+        r1 = r0 + 8;
+    } else {
+        const int bb = min(2 * tile + 1, nbp - 1);
+        r0 = (max(s_blk[2 * tile], 0) * num_kv_heads + h) * 8;
+        r1 = (max(s_blk[bb], 0) * num_kv_heads + h) * 8;
+    }
+}
+
+// Lane 0 of a warp: fetch the K and V rows of one tile (16 tokens x D) into
+// the tile pair at `dst` (K then V), completing on `bar`.
 template <int kTileBytes, typename T>
 __device__ __forceinline__ void issue_tile_pair(uint8_t* dst, uint64_t* bar, const T* k_cache,
-                                                const T* v_cache, int64_t off, uint64_t policy)
+                                                const T* v_cache, int64_t row0, int64_t row1, bool split,
+                                                int D, uint64_t policy)
 {
     // order this warp's earlier generic reads of the tiles before the async writes
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     pkv::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-    pkv::bulk_load(dst, k_cache + off, kTileBytes, bar, policy);
-    pkv::bulk_load(dst + kTileBytes, v_cache + off, kTileBytes, bar, policy);
+    if (!split) {
+        pkv::bulk_load(dst, k_cache + row0 * D, kTileBytes, bar, policy);
+        pkv::bulk_load(dst + kTileBytes, v_cache + row0 * D, kTileBytes, bar, policy);
+    } else {
+        constexpr int kHalf = kTileBytes / 2;
+        pkv::bulk_load(dst, k_cache + row0 * D, kHalf, bar, policy);
+        pkv::bulk_load(dst + kHalf, k_cache + row1 * D, kHalf, bar, policy);
+        pkv::bulk_load(dst + kTileBytes, v_cache + row0 * D, kHalf, bar, policy);
+        pkv::bulk_load(dst + kTileBytes + kHalf, v_cache + row1 * D, kHalf, bar, policy);
+    }
 }
 
 struct SeqRange {
@@ -138,8 +174,8 @@ struct SeqRange {
     bool bad;      // context length < 1
 };
 
-__device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int max_ctx,
-                                              bool report, int* status)
+__device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int block_size,
+                                              int max_ctx, bool report, int* status)
 {
     SeqRange r;
     int ctx = __ldg(context_lens + s);
@@ -148,9 +184,9 @@ __device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s
         flag = 1;
         ctx = 0;
     }
-    if (ctx > mb * kBlock) {
+    if ((int64_t)ctx > (int64_t)mb * block_size) {
         flag = 1;
-        ctx = mb * kBlock;
+        ctx = mb * block_size;
     }
     if (ctx > max_ctx) {
         flag = 1;
@@ -163,7 +199,7 @@ __device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s
     return r;
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int B>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_partition_kernel(T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
                             const T* __restrict__ q, const T* __restrict__ k_cache,
@@ -178,7 +214,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0,
+    const SeqRange sr = seq_range(context_lens, s, mb, B, max_ctx, p == 0 && h == 0 && threadIdx.x == 0,
                                   status);
     if (sr.bad) {
         // nothing to attend to: a zero row (flagged above)
@@ -191,17 +227,18 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     if (p >= sr.nparts) return;
 
-    const int nblk_seq = (sr.ctx + kBlock - 1) / kBlock;
+    constexpr int kPartBlocks = kPartTokens / B;
+    const int nblk_seq = (sr.ctx + B - 1) / B;
     const int blk0 = p * kPartBlocks;
-    const int nb = min(kPartBlocks, nblk_seq - blk0);
-    const int last_valid = sr.ctx - (nblk_seq - 1) * kBlock;
+    const int nbp = min(kPartBlocks, nblk_seq - blk0);                 // blocks of this partition
+    const int nb = min(kPartTiles, (sr.ctx - p * kPartTokens + kTile - 1) / kTile);  // its tiles
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
     float* s_sc = reinterpret_cast<float*>(smem + C::kScoreOff) + warp * C::kItems;
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
     uint8_t* my_tiles = smem + warp * (kStages * 2 * C::kTileBytes);
 
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    for (int i = threadIdx.x; i < nbp; i += blockDim.x) {
         int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
         if (b < 0 || b >= num_blocks) {
             pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
@@ -216,18 +253,17 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     __syncthreads();
 
-    // this warp's blocks: j = warp + k * kWarps, k < nw
+    // this warp's tiles: warp + k * kWarps, k < nw
     const int nw = nb > warp ? (nb - warp + kWarps - 1) / kWarps : 0;
-    const int64_t tile_elems = (int64_t)kBlock * D;
     uint64_t policy = 0;
     if (lane == 0) policy = pkv::policy_evict_first();
 
     if (lane == 0) {
         for (int k = 0; k < nw && k < kStages; ++k) {
+            int r0, r1;
+            tile_rows<B>(s_blk, nbp, warp + k * kWarps, num_kv_heads, h, r0, r1);
             issue_tile_pair<C::kTileBytes>(my_tiles + (k % kStages) * 2 * C::kTileBytes, &bars[k % kStages],
-                                           k_cache, v_cache,
-                                           ((int64_t)s_blk[warp + k * kWarps] * num_kv_heads + h) * tile_elems,
-                                           policy);
+                                           k_cache, v_cache, r0, r1, B == 8, D, policy);
         }
     }
 
@@ -271,7 +307,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         const T* sk = reinterpret_cast<const T*>(my_tiles + st * 2 * C::kTileBytes);
         const T* sv = reinterpret_cast<const T*>(my_tiles + st * 2 * C::kTileBytes + C::kTileBytes);
-        const int valid = (blk0 + warp + k * kWarps == nblk_seq - 1) ? last_valid : kBlock;
+        const int valid = min(kTile, sr.ctx - (p * kPartTokens + (warp + k * kWarps) * kTile));
 
         // ---- Q.K for the block's 16 tokens -----------------------------
         float part[C::kNv];
@@ -367,10 +403,10 @@ __global__ void __launch_bounds__(kWarps * 32)
         __syncwarp();
         ++consumed;
         if (lane == 0 && k + kStages < nw) {
-            const int kn = k + kStages;
-            issue_tile_pair<C::kTileBytes>(my_tiles + st * 2 * C::kTileBytes, &bars[st], k_cache, v_cache,
-                                           ((int64_t)s_blk[warp + kn * kWarps] * num_kv_heads + h) * tile_elems,
-                                           policy);
+            int r0, r1;
+            tile_rows<B>(s_blk, nbp, warp + (k + kStages) * kWarps, num_kv_heads, h, r0, r1);
+            issue_tile_pair<C::kTileBytes>(my_tiles + st * 2 * C::kTileBytes, &bars[st], k_cache, v_cache, r0, r1,
+                                           B == 8, D, policy);
         }
     }
 
@@ -446,8 +482,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128)
     decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
                          const float* __restrict__ ws_ml, const int32_t* __restrict__ context_lens,
-                         int32_t num_seqs, int32_t q_len, int32_t num_q_heads, int32_t mb, int32_t max_ctx,
-                         int32_t max_parts)
+                         int32_t num_seqs, int32_t q_len, int32_t num_q_heads, int32_t mb, int32_t block_size,
+                         int32_t max_ctx, int32_t max_parts)
 {
     constexpr int kPer = D / 32;
     using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
@@ -457,7 +493,7 @@ __global__ void __launch_bounds__(128)
     const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= (int64_t)num_seqs * q_len * num_q_heads) return;   // row = (s * q_len + j) * Hq + i
     const int s = (int)(row / ((int64_t)q_len * num_q_heads));
-    const SeqRange sr = seq_range(context_lens, s, mb, max_ctx, false, nullptr);
+    const SeqRange sr = seq_range(context_lens, s, mb, block_size, max_ctx, false, nullptr);
     if (sr.bad || sr.ctx < q_len || sr.nparts <= 1) return;   // zero rows / single partition: written
     const float* ml = ws_ml + row * max_parts * 2;
     const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
@@ -529,10 +565,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// Tensor map over a cache viewed as [num_blocks * Hkv * 16 rows][D] 16-bit
-// elements, in boxes of 16 rows x 64 elements with the 128-byte swizzle.
+// Tensor map over a cache viewed as [num_blocks * Hkv * block_size rows][D]
+// 16-bit elements, in boxes of box_rows x 64 elements with the 128-byte
+// swizzle (box_rows 16, or 8 for block size 8).
 template <typename T>
-int encode_cache_map(CUtensorMap* map, const void* cache, int64_t rows, int D)
+int encode_cache_map(CUtensorMap* map, const void* cache, int64_t rows, int D, int box_rows)
 {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) {
@@ -541,7 +578,7 @@ int encode_cache_map(CUtensorMap* map, const void* cache, int64_t rows, int D)
     }
     const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)D * sizeof(T)};
-    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t estride[2] = {1, 1};
     const CUtensorMapDataType ty =
         sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -594,13 +631,14 @@ struct DecodeArgs {
     int32_t Hq;
     int32_t Hkv;
     int32_t NB;
+    int32_t block_size;
     float scale;
     void* ws;
     cudaStream_t stream;
     int* status;
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int B>
 int launch(const DecodeArgs& a)
 {
     const int max_parts = (a.max_ctx + kPartTokens - 1) / kPartTokens;
@@ -614,11 +652,11 @@ int launch(const DecodeArgs& a)
     if constexpr (sizeof(T) == 2) {
         // fp16 / bf16: tensor-core kernel fed by tiled TMA
         using C = TcCfg<D>;
-        const int64_t rows = (int64_t)a.NB * a.Hkv * kBlock;
+        const int64_t rows = (int64_t)a.NB * a.Hkv * B;
         if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
         CUtensorMap tm_k, tm_v;
-        if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D)) != PKV_OK) return rc;
-        if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D)) != PKV_OK) return rc;
+        if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
+        if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
         cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
@@ -631,26 +669,26 @@ int launch(const DecodeArgs& a)
         };
         if (a.q_len > 1) {
             static bool configured[64] = {};
-            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, true>, C::kSmemBytes, configured)) != PKV_OK)
+            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, true, B>, C::kSmemBytes, configured)) != PKV_OK)
                 return rc;
-            launch_err = args(decode_partition_tc_kernel<T, D, G, true>);
+            launch_err = args(decode_partition_tc_kernel<T, D, G, true, B>);
         } else {
             static bool configured[64] = {};
-            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, false>, C::kSmemBytes, configured)) != PKV_OK)
+            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, false, B>, C::kSmemBytes, configured)) != PKV_OK)
                 return rc;
-            launch_err = args(decode_partition_tc_kernel<T, D, G, false>);
+            launch_err = args(decode_partition_tc_kernel<T, D, G, false, B>);
         }
     } else {
         // fp32: CUDA-core kernel fed by 1-D bulk copies (one query, no fused write)
         if (a.q_len != 1 || a.k_new) return PKV_ERR_UNSUPPORTED;
         using C = Cfg<T, D, G>;
         static bool configured[64] = {};
-        rc = allow_smem(decode_partition_kernel<T, D, G>, C::kSmemBytes, configured);
+        rc = allow_smem(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured);
         if (rc != PKV_OK) return rc;
         cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
-        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_kernel<T, D, G>, static_cast<T*>(a.out), ws_acc,
+        launch_err = cudaLaunchKernelEx(&cfg, decode_partition_kernel<T, D, G, B>, static_cast<T*>(a.out), ws_acc,
                                         ws_ml, static_cast<const T*>(a.q), static_cast<const T*>(a.k_cache),
                                         static_cast<const T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.Hq,
                                         a.Hkv, a.NB, scale_log2, max_parts, a.status);
@@ -666,7 +704,7 @@ int launch(const DecodeArgs& a)
     pkv::pdl_attribute(&cfg, attr);
     const cudaError_t reduce_err =
         cudaLaunchKernelEx(&cfg, decode_reduce_kernel<T, D>, static_cast<T*>(a.out), (const float*)ws_acc,
-                           (const float*)ws_ml, a.cl, a.S, a.q_len, a.Hq, a.mb, a.max_ctx, max_parts);
+                           (const float*)ws_ml, a.cl, a.S, a.q_len, a.Hq, a.mb, B, a.max_ctx, max_parts);
     if (reduce_err != cudaSuccess) {
         pkv::record_cuda_error(reduce_err);
         return PKV_ERR_CUDA;
@@ -674,14 +712,25 @@ int launch(const DecodeArgs& a)
     return pkv::check_launch();
 }
 
+template <typename T, int D, int G>
+int dispatch_b(const DecodeArgs& a)
+{
+    switch (a.block_size) {
+        case 8: return launch<T, D, G, 8>(a);
+        case 16: return launch<T, D, G, 16>(a);
+        case 32: return launch<T, D, G, 32>(a);
+        default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
 template <typename T, int D>
 int dispatch_g(int G, const DecodeArgs& a)
 {
     switch (G) {
-        case 1: return launch<T, D, 1>(a);
-        case 2: return launch<T, D, 2>(a);
-        case 4: return launch<T, D, 4>(a);
-        case 8: return launch<T, D, 8>(a);
+        case 1: return dispatch_b<T, D, 1>(a);
+        case 2: return dispatch_b<T, D, 2>(a);
+        case 4: return dispatch_b<T, D, 4>(a);
+        case 8: return dispatch_b<T, D, 8>(a);
         default: return PKV_ERR_UNSUPPORTED;
     }
 }
@@ -705,7 +754,8 @@ int decode_entry(void* out, const void* q, const void* k_new, const void* v_new,
     if (num_seqs < 0 || q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
         num_blocks < 1 || max_blocks_per_seq < 1 || !isfinite(scale) || (!k_new) != (!v_new))
         return PKV_ERR_INVALID_ARG;
-    if (block_size != kBlock || (head_dim != 64 && head_dim != 128)) return PKV_ERR_UNSUPPORTED;
+    if ((block_size != 8 && block_size != 16 && block_size != 32) || (head_dim != 64 && head_dim != 128))
+        return PKV_ERR_UNSUPPORTED;
     const int G = num_q_heads / num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
     if (q_len * G > 16) return PKV_ERR_UNSUPPORTED;  // the query rows fill one 16-row tensor-core operand
@@ -725,7 +775,7 @@ int decode_entry(void* out, const void* q, const void* k_new, const void* v_new,
     if (!status) return PKV_ERR_CUDA;
     const DecodeArgs a{out,           q,        k_new,          v_new,        k_cache,      v_cache,
                        block_tables,  max_blocks_per_seq,       context_lens, num_seqs,     q_len,
-                       max_context_len, num_q_heads, num_kv_heads, num_blocks, scale,       workspace,
+                       max_context_len, num_q_heads, num_kv_heads, num_blocks, block_size, scale, workspace,
                        (cudaStream_t)stream, status};
     switch (dtype) {
         case PKV_F32: return dispatch_d<float>(head_dim, G, a);

@@ -117,15 +117,19 @@ struct TcCfg {
     static constexpr int kTilesBytes = kWarps * kStages * kStageBytes;
     static constexpr int kBarOff = kTilesBytes;
     static constexpr int kBlkOff = kBarOff + kWarps * kStages * 8;
-    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBlkOff + kPartBlocks * 4;
+    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBlkOff + kMaxPartBlocks * 4;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
 };
 
-// Lane 0 of a warp: fetch the K and V tiles of cache rows [row, row + 16)
-// into the stage at `dst` (K boxes, then V boxes), completing on `bar`.
+// Lane 0 of a warp: fetch the K and V rows of one 16-token tile into the
+// stage at `dst` (K boxes, then V boxes), completing on `bar`.  Unsplit:
+// cache rows [r0, r0 + 16) as 16-row boxes.  Split (block size 8): rows
+// [r0, r0 + 8) and [r1, r1 + 8) as 8-row boxes into the two 1 KiB halves of
+// each 16-row box, which gives the same swizzled layout, since the 128-byte
+// swizzle repeats every 8 rows.
 template <int D>
 __device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUtensorMap* tm_k,
-                                         const CUtensorMap* tm_v, int row, uint64_t policy)
+                                         const CUtensorMap* tm_v, int r0, int r1, bool split, uint64_t policy)
 {
     using C = TcCfg<D>;
     const uint32_t b = pkv::smem_addr(bar);
@@ -134,8 +138,13 @@ __device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUte
     pkv::mbar_arrive_expect_tx(bar, C::kStageBytes);
 #pragma unroll
     for (int bx = 0; bx < C::kBoxes; ++bx) {
-        tma_load_2d(dst + bx * kTcBoxBytes, tm_k, bx * 64, row, b, policy);
-        tma_load_2d(dst + C::kTileBytes + bx * kTcBoxBytes, tm_v, bx * 64, row, b, policy);
+        const uint32_t kd = dst + bx * kTcBoxBytes, vd = dst + C::kTileBytes + bx * kTcBoxBytes;
+        tma_load_2d(kd, tm_k, bx * 64, r0, b, policy);
+        tma_load_2d(vd, tm_v, bx * 64, r0, b, policy);
+        if (split) {
+            tma_load_2d(kd + kTcBoxBytes / 2, tm_k, bx * 64, r1, b, policy);
+            tma_load_2d(vd + kTcBoxBytes / 2, tm_v, bx * 64, r1, b, policy);
+        }
     }
 }
 
@@ -174,7 +183,7 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 // k_new / v_new non-null: the new tokens' K/V rows [S][q_len][Hkv][D] are
 // written to their slots (through the block table) by the CTA whose
 // partition holds them, and patched into the staged tiles before use.
-template <typename T, int D, int G, bool kMQ>
+template <typename T, int D, int G, bool kMQ, int B>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = kMQ ? q_len * G : G;  // live query rows
 
-    SeqRange sr = seq_range(context_lens, s, mb, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
+    SeqRange sr = seq_range(context_lens, s, mb, B, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
     if (!sr.bad && sr.ctx < q_len) {
         if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
         sr.bad = true;
@@ -214,16 +223,18 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (p >= sr.nparts) return;
 
     const int ctx = sr.ctx;
-    const int nblk_seq = (ctx + kBlock - 1) / kBlock;
+    constexpr int kPartBlocks = kPartTokens / B;
+    const int nblk_seq = (ctx + B - 1) / B;
     const int blk0 = p * kPartBlocks;
-    const int nb = min(kPartBlocks, nblk_seq - blk0);
+    const int nbp = min(kPartBlocks, nblk_seq - blk0);                          // blocks of this partition
+    const int nb = min(kPartTiles, (ctx - p * kPartTokens + kTile - 1) / kTile);  // its 16-token tiles
     const int first_new = ctx - q_len;   // position of the first new token
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
     const uint32_t tiles = pkv::smem_addr(smem + warp * (kStages * C::kStageBytes));
 
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    for (int i = threadIdx.x; i < nbp; i += blockDim.x) {
         int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
         if (b < 0 || b >= num_blocks) {
             pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
@@ -245,8 +256,10 @@ __global__ void __launch_bounds__(kWarps * 32)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
         for (int k = 0; k < nw && k < kStages; ++k) {
-            tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], &tm_k, &tm_v,
-                        (max(s_blk[warp + k * kWarps], 0) * num_kv_heads + h) * kBlock, policy);
+            int r0, r1;
+            tile_rows<B>(s_blk, nbp, warp + k * kWarps, num_kv_heads, h, r0, r1);
+            tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], &tm_k, &tm_v, r0, r1, B == 8,
+                        policy);
         }
     }
 
@@ -300,26 +313,28 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         const uint32_t kbase = tiles + st * C::kStageBytes;
         const uint32_t vbase = kbase + C::kTileBytes;
-        const int lblk = warp + k * kWarps;
-        const int pos0 = (blk0 + lblk) * kBlock;
+        const int tile = warp + k * kWarps;
+        const int pos0 = p * kPartTokens + tile * kTile;
 
-        // ---- fused slot write: this block holds new tokens -> store and patch
-        if (k_new != nullptr && pos0 + kBlock > first_new) {
-            const int phys = s_blk[lblk];
+        // ---- fused slot write: this tile holds new tokens -> store and patch
+        if (k_new != nullptr && pos0 + kTile > first_new) {
             const int jlo = max(0, pos0 - first_new);
-            const int jhi = min(q_len, pos0 + kBlock - first_new);
+            const int jhi = min(q_len, pos0 + kTile - first_new);
             const int items = (jhi - jlo) * 2 * kChunks;
             for (int it = lane; it < items; it += 32) {
                 const int c = it % kChunks;
                 const int kv = (it / kChunks) & 1;
                 const int jj = jlo + it / (2 * kChunks);
-                const int t = first_new + jj - pos0;
+                const int t = first_new + jj - pos0;                  // row in the tile
+                const int pos = first_new + jj;                          // position in the sequence
+                const int phys = s_blk[(pos - p * kPartTokens) / B];
                 const T* src = (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8;
                 const uint4 val = *reinterpret_cast<const uint4*>(src);
                 st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 + (((c % 8) ^ (t & 7)) << 4),
                              val);
                 if (phys >= 0) {
-                    T* dst = (kv ? v_cache_w : k_cache_w) + (((int64_t)phys * num_kv_heads + h) * kBlock + t) * D + c * 8;
+                    T* dst = (kv ? v_cache_w : k_cache_w) +
+                             (((int64_t)phys * num_kv_heads + h) * B + pos % B) * D + c * 8;
                     *reinterpret_cast<uint4*>(dst) = val;
                 }
             }
@@ -338,7 +353,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
 
         // ---- online softmax; this lane holds tokens qd, qd+1, qd+8, qd+9 of rows ra (and rb)
-        const bool mask = pos0 + kBlock > first_new + 1;   // some token of this block is not visible to all rows
+        const bool mask = pos0 + kTile > first_new + 1;   // some token of this tile is not visible to all rows
         float xa[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
         const int tp[4] = {pos0 + qd, pos0 + qd + 1, pos0 + qd + 8, pos0 + qd + 9};
         float alpha_a, alpha_b = 1.0f;
@@ -406,7 +421,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         // V rows of tokens at or past the sequence length are zeroed: whatever
         // the unused slots hold (even NaN) must not reach the result.
         uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // V rows qd, qd+1 / qd+8, qd+9
-        if (pos0 + kBlock > ctx) {
+        if (pos0 + kTile > ctx) {
             keep_lo = (tp[0] < ctx ? 0x0000ffffu : 0u) | (tp[1] < ctx ? 0xffff0000u : 0u);
             keep_hi = (tp[2] < ctx ? 0x0000ffffu : 0u) | (tp[3] < ctx ? 0xffff0000u : 0u);
         }
@@ -429,8 +444,9 @@ __global__ void __launch_bounds__(kWarps * 32)
         __syncwarp();
         ++consumed;
         if (lane == 0 && k + kStages < nw) {
-            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v,
-                        (max(s_blk[warp + (k + kStages) * kWarps], 0) * num_kv_heads + h) * kBlock, policy);
+            int r0, r1;
+            tile_rows<B>(s_blk, nbp, warp + (k + kStages) * kWarps, num_kv_heads, h, r0, r1);
+            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v, r0, r1, B == 8, policy);
         }
     }
 

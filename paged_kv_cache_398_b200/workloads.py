@@ -120,7 +120,7 @@ def _lognormal(n: int, mean: float, sigma: float, gen) -> torch.Tensor:
 
 def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min_ctx=None,
                   num_prompts=None, max_prompt=None, max_output=None, seed=None,
-                  pad_random: bool = False) -> DecodeWorkload:
+                  pad_random: bool = False, block_size: int = BLOCK_SIZE) -> DecodeWorkload:
     """Build workload `number` (1..5).  Keyword overrides shrink it for tests.
 
     Lengths, the pool permutation and the block tables are always drawn on the
@@ -131,7 +131,7 @@ def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min
     name = WORKLOADS[number]
     seed = 398000 + number if seed is None else seed
     g = torch.Generator().manual_seed(seed)
-    B = BLOCK_SIZE
+    B = block_size
     copy_pairs = []
     meta = {"workload": name}
 
@@ -164,7 +164,7 @@ def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min
             ctx = torch.clamp(p + o, lo, hi).to(torch.int64).tolist()
         else:
             ctx = torch.randint(lo, hi + 1, (S,), generator=g).tolist()
-        prefix = 4 if number == 4 else 0
+        prefix = 64 // B if number == 4 else 0      # the 64-token system prompt
         need = prefix + sum(_nblk(c, B) - prefix for c in ctx)
         NB = need + _nblk(need, 8)
         perm = torch.randperm(NB, generator=g).tolist()
@@ -250,13 +250,14 @@ def make_workload(number: int, device="cpu", *, num_seqs=None, max_ctx=None, min
 
 def make_custom(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype,
                 device="cpu", *, seed: int = 1234, spare_blocks: int = 3,
-                max_blocks_per_seq=None, pad_random: bool = False, q_len=None) -> DecodeWorkload:
+                max_blocks_per_seq=None, pad_random: bool = False, q_len=None,
+                block_size: int = BLOCK_SIZE) -> DecodeWorkload:
     """A batch with the given context lengths and head shape, blocks dealt
     from a seeded permutation of a pool with `spare_blocks` unused blocks.
     With q_len given, q is [S, q_len, Hq, D] and k_new / v_new are
     [S, q_len, Hkv, D] (several new tokens per sequence)."""
     g = torch.Generator().manual_seed(seed)
-    B = BLOCK_SIZE
+    B = block_size
     ctx = [int(c) for c in context_lens]
     need = sum(_nblk(max(c, 1), B) for c in ctx)
     NB = need + spare_blocks

@@ -59,7 +59,7 @@ def test_host_side_rejections(L):
     assert L.paged_kv_write(None, None, None, None, None, 0, 8, 128, 16, 10, 2, None) == C["PKV_OK"]
     assert L.paged_attention_decode(None, None, None, None, None, 4, None, 2, 100, 32, 8, 96, 16, 10,
                                     ctypes.c_float(0.1), 2, None, 0, None) == UNS
-    assert L.paged_attention_decode(None, None, None, None, None, 4, None, 2, 100, 32, 8, 128, 32, 10,
+    assert L.paged_attention_decode(None, None, None, None, None, 4, None, 2, 100, 32, 8, 128, 24, 10,
                                     ctypes.c_float(0.1), 2, None, 0, None) == UNS
     assert L.paged_attention_decode(None, None, None, None, None, 4, None, 2, 100, 24, 8, 128, 16, 10,
                                     ctypes.c_float(0.1), 2, None, 0, None) == UNS

@@ -35,7 +35,7 @@ def oracle_slots_mq(w, q_len):
     for s in range(w.num_seqs):
         ctx = int(w.context_lens[s])
         row = w.block_tables[s].tolist()
-        out += [slot_for_position(row, ctx - q_len + j, B) for j in range(q_len)]
+        out += [slot_for_position(row, ctx - q_len + j, w.block_size) for j in range(q_len)]
     return torch.tensor(out, dtype=torch.int64)
 
 
@@ -57,9 +57,10 @@ def _clean_status(cuda_device):
 def _both_paths(w, q_len):
     """(separate write + decode_mq, fused decode_mq) outputs and caches on the GPU."""
     S, Hkv, D = w.num_seqs, w.num_kv_heads, w.head_dim
-    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - q_len + j, B)
+    Bs = w.block_size
+    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - q_len + j, Bs)
                           for s in range(S) for j in range(q_len)], dtype=torch.int64)
-    prod_slots = torch.cat([pkv.pkv_slot_mapping(w.block_tables, w.context_lens - q_len + j)[:, None]
+    prod_slots = torch.cat([pkv.pkv_slot_mapping(w.block_tables, w.context_lens - q_len + j, Bs)[:, None]
                             for j in range(q_len)], dim=1).reshape(-1)
     assert torch.equal(prod_slots, slots)
     a = w.to("cuda")
@@ -145,3 +146,18 @@ def test_unsupported_combinations_are_rejected():
     with pytest.raises(pkv.PagedKVError):
         pkv.paged_attention_decode_mq(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale,
                                       w.max_context_len)
+
+
+@pytest.mark.parametrize("block_size", [8, 32])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("G,q_len", [(1, 1), (4, 3), (2, 8)])
+def test_multi_query_fused_block_sizes_8_and_32(block_size, dtype, G, q_len):
+    lens = [max(n, q_len) for n in (5, 8, 9, 17, 33, 510, 514, 1031)]
+    w = make_custom(lens, 2 * G, 2, 128, dtype, seed=7 * block_size + G + q_len, q_len=q_len,
+                    block_size=block_size)
+    ref, k_ref, v_ref = oracle_mq(w, q_len)
+    (oa, ka, va), (ob, kb, vb) = _both_paths(w, q_len)
+    for k_, v_ in ((ka, va), (kb, vb)):
+        assert torch.equal(k_.cpu(), k_ref) and torch.equal(v_.cpu(), v_ref)
+    assert_close(oa, ref, "write then decode")
+    assert torch.equal(oa, ob)

@@ -35,7 +35,7 @@ def assert_close(got: torch.Tensor, ref: np.ndarray, what=""):
 
 def oracle_slots(w):
     """Slots of each sequence's new token (its last position), by the oracle."""
-    return torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - 1, B)
+    return torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - 1, w.block_size)
                          for s in range(w.num_seqs)], dtype=torch.int64)
 
 
@@ -70,7 +70,7 @@ def _clean_status(cuda_device):
 def _run_full_parity(w):
     slots = oracle_slots(w)
     # the product computes its own slot mapping (host helper) and must agree
-    prod_slots = pkv.pkv_slot_mapping(w.block_tables, w.context_lens - 1)
+    prod_slots = pkv.pkv_slot_mapping(w.block_tables, w.context_lens - 1, w.block_size)
     assert torch.equal(prod_slots, slots)
     g = w.to("cuda")
     out = product_step(g, prod_slots.cuda())
@@ -362,3 +362,15 @@ def test_bounded_wait_times_out_and_context_survives():
     assert flags & pkv._lib.C["PKV_DEV_WAIT_TIMEOUT"]
     assert 0.015 < waited < 5.0
     _run_full_parity(make_workload(1))
+
+
+# ---------------------------------------------------------------------------
+# block sizes 8 and 32 (a compute tile is 16 tokens: two blocks or half of one)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("block_size", [8, 32])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("D,G", [(64, 1), (128, 4), (128, 8)])
+def test_block_sizes_8_and_32(block_size, dtype, D, G):
+    lens = [1, 7, 8, 9, 15, 16, 17, 31, 33, 511, 512, 513, 520, 1000, 4100]
+    w = make_custom(lens, 2 * G, 2, D, dtype, seed=block_size * 100 + G + D, block_size=block_size)
+    _run_full_parity(w)

@@ -52,8 +52,20 @@ inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStr
     return cfg;
 }
 
+// Under stream capture (CUDA graphs) the attribute is left out: capture
+// does not accept it here, and an ordinary launch is always correct.
 inline void pdl_attribute(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr)
 {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(cfg->stream, &cs) != cudaSuccess) {
+        cudaGetLastError();  // clear; fall back to an ordinary launch
+        cs = cudaStreamCaptureStatusActive;
+    }
+    if (cs != cudaStreamCaptureStatusNone) {
+        cfg->attrs = nullptr;
+        cfg->numAttrs = 0;
+        return;
+    }
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg->attrs = attr;

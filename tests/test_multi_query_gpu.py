@@ -161,3 +161,37 @@ def test_multi_query_fused_block_sizes_8_and_32(block_size, dtype, G, q_len):
         assert torch.equal(k_.cpu(), k_ref) and torch.equal(v_.cpu(), v_ref)
     assert_close(oa, ref, "write then decode")
     assert torch.equal(oa, ob)
+
+
+def test_fused_decode_step_replays_from_a_cuda_graph():
+    """The step (fused slot write + decode) captured once and replayed gives
+    the same bits as eager calls, also after the inputs change in place."""
+    host = make_workload(4, num_seqs=16, max_ctx=3000)
+    w = host.to("cuda")
+    S, max_ctx = w.num_seqs, host.max_context_len      # a host int: nothing is read back under capture
+    q4, kn4, vn4 = w.q[:, None].contiguous(), w.k_new[:, None].contiguous(), w.v_new[:, None].contiguous()
+    ws = torch.empty(max(1, pkv.paged_attention_mq_workspace_bytes(S, 1, w.num_q_heads, w.head_dim, max_ctx)),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q4)
+
+    def step():
+        pkv.paged_attention_decode_mq(out, q4, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale,
+                                      max_ctx, k_new=kn4, v_new=vn4, workspace=ws)
+
+    step()                                  # first call on the device: set-up outside capture
+    torch.cuda.synchronize()
+    eager = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    q4.copy_(torch.randn(q4.shape, generator=torch.Generator(device="cuda").manual_seed(3), device="cuda").to(q4.dtype))
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = out.clone()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(replayed, out) and not torch.equal(replayed, eager)

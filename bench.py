@@ -283,8 +283,10 @@ def sub_workload(w, tables, lens, pairs, seqs):
         k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(), scale=w.scale, seed=w.seed)
 
 
-def oracle_step_timed(sub, threads: int) -> float:
-    """Run the oracle's copy + write + decode on `sub`; returns wall seconds."""
+def oracle_step_timed(sub, threads: int, keep=None):
+    """Run the oracle's copy + write + decode on `sub`; returns wall seconds.
+    With `keep` (a list), the fp64 outputs [Hq, D] of the sequences are
+    appended to it."""
     import concurrent.futures as cf
 
     import oracle
@@ -298,9 +300,12 @@ def oracle_step_timed(sub, threads: int) -> float:
         oracle.block_copy(k, v, sub.copy_pairs)
     oracle.kv_write(k, v, sub.k_new, sub.v_new, slots)
     with cf.ThreadPoolExecutor(max_workers=threads) as ex:
-        list(ex.map(lambda s: oracle.paged_decode_seq(s, sub.q, k, v, sub.block_tables, sub.context_lens,
-                                                      sub.scale), range(sub.num_seqs)))
-    return time.perf_counter() - t0
+        outs = list(ex.map(lambda s: oracle.paged_decode_seq(s, sub.q, k, v, sub.block_tables, sub.context_lens,
+                                                             sub.scale), range(sub.num_seqs)))
+    t = time.perf_counter() - t0
+    if keep is not None:
+        keep.extend(outs)
+    return t
 
 
 def sample_kv_bytes(sub) -> int:
@@ -332,11 +337,27 @@ def cpu_baseline(st, threads: int):
     per_tok = t1 / max(1, int(lens[0]))
     seqs = pick_sample(lens, 30.0, per_tok)
     sub = sub_workload(st.w, tables, lens, pairs, seqs)
-    t = oracle_step_timed(sub, threads)
+    refs = []
+    t = oracle_step_timed(sub, threads, keep=refs)
     return {"value": sample_kv_bytes(sub) / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": (f"{len(seqs)} of {len(lens)} sequences (all {sub.num_q_heads} query heads): "
                        f"copy + slot write + decode by the fp64 C oracle, {t:.2f} s wall on {threads} threads"),
-            "seconds": t}
+            "seconds": t, "seqs": seqs, "refs": refs}
+
+
+def parity_on_sample(st, base, atol: float = 2e-3, rtol: float = 1e-2):
+    """The timed steps' output of the sampled sequences against the oracle's
+    fp64 output of the same step (repeating a step leaves the cache as one
+    step leaves it, so the last step's output is the one to compare)."""
+    import numpy as np
+    got = st.out[torch.tensor(base["seqs"], device=st.out.device)].double().cpu().numpy()
+    ref = np.stack(base["refs"])
+    err = np.abs(got - ref)
+    big = np.abs(ref) > 1e-3
+    return {"max_abs_err": float(err.max()), "max_rel_err": float((err[big] / np.abs(ref[big])).max()),
+            "out_of_tolerance": int((err > atol + rtol * np.abs(ref)).sum()), "elements": int(err.size),
+            "tolerance": f"|gpu - oracle| <= {atol:g} + {rtol:g} |oracle| per element",
+            "sample": f"{len(base['seqs'])} sequences x {ref.shape[1]} query heads x {ref.shape[2]}"}
 
 
 # ----------------------------------------------------------------------------
@@ -573,7 +594,9 @@ def run_ours(args):
                      "unit": "GB/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path, st.w.block_size),
                      "algorithmic_bytes_per_launch": call_bytes},
-        "cpu_baseline": ({k: v for k, v in base.items() if k != "seconds"} if base else None),
+        "cpu_baseline": ({k: v for k, v in base.items() if k in ("value", "unit", "cores", "kind", "sample")}
+                         if base else None),
+        "parity": parity_on_sample(st, base) if base else None,
         "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_steps},
         "gpu_launches": (st.launches_fused if st.path == "fused" else st.launches_separate) * args.steps,

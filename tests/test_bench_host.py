@@ -1,0 +1,52 @@
+"""Host-side pieces of bench.py (CPU only): the relabelled sample of the
+batch that the oracle baseline times, and the parity summary the bench
+prints for the sampled sequences."""
+
+import types
+
+import numpy as np
+import torch
+
+import bench
+import oracle
+from oracle.allocator_model import slot_for_position
+from paged_kv_cache_398_b200.workloads import make_workload
+
+
+def _full_oracle_step(w):
+    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - 1, w.block_size)
+                          for s in range(w.num_seqs)], dtype=torch.int64)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    if w.copy_pairs.numel():
+        oracle.block_copy(k, v, w.copy_pairs)
+    oracle.kv_write(k, v, w.k_new, w.v_new, slots)
+    return oracle.paged_decode(w.q, k, v, w.block_tables, w.context_lens, w.scale)
+
+
+def test_sample_gives_the_same_outputs_as_the_whole_batch():
+    """Sampled sequences, their blocks gathered and relabelled (copy-on-write
+    sources included), decode to exactly the whole batch's rows."""
+    w = make_workload(5, device="cpu", num_prompts=3, max_prompt=400, max_output=200)
+    seqs = [1, 4, 6]
+    sub = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs)
+    assert sub.num_blocks < w.num_blocks
+    refs = []
+    bench.oracle_step_timed(sub, 2, keep=refs)
+    whole = _full_oracle_step(w)
+    assert np.array_equal(np.stack(refs), whole[seqs])
+
+
+def test_parity_summary_counts_out_of_tolerance_elements():
+    w = make_workload(1, device="cpu")
+    seqs = list(range(w.num_seqs))
+    sub = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs)
+    refs = []
+    bench.oracle_step_timed(sub, 2, keep=refs)
+    st = types.SimpleNamespace(out=torch.tensor(np.stack(refs)).to(w.dtype))
+    base = {"seqs": seqs, "refs": refs}
+    rep = bench.parity_on_sample(st, base)
+    assert rep["out_of_tolerance"] == 0 and rep["max_abs_err"] < 1e-6
+    assert rep["elements"] == w.num_seqs * w.num_q_heads * w.head_dim
+    st.out[1, 2, 3] += 0.5
+    rep = bench.parity_on_sample(st, base)
+    assert rep["out_of_tolerance"] == 1 and rep["max_abs_err"] > 0.49

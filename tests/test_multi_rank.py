@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_like_the_bench():
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:    # no fork of a threaded process
         out = mgr.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)

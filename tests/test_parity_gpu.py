@@ -350,6 +350,39 @@ def test_many_copy_pairs_span_launches():
     assert torch.equal(kc[:1300], k0[:1300])
 
 
+# ---------------------------------------------------------------------------
+# split-K: one workspace serves every batch shape, and the longest contexts
+# (hundreds of partitions per sequence) merge correctly
+# ---------------------------------------------------------------------------
+def test_one_workspace_serves_batches_of_any_shape():
+    """One workspace, reused without clearing by batches of other shapes (the
+    previous call's records stay in it), gives every batch its own result."""
+    shapes = [make_custom([5000, 2000, 700], 32, 8, 128, torch.bfloat16, seed=34),
+              make_custom([600, 1100, 40, 3000, 900, 1500, 2600], 8, 2, 64, torch.float16, seed=35),
+              make_custom([9000], 16, 2, 128, torch.bfloat16, seed=36)]
+    need = max(pkv.paged_attention_workspace_bytes(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len)
+               for w in shapes)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for w in shapes + shapes[::-1]:
+        ref = oracle.paged_decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale)
+        g = w.to("cuda")
+        out = torch.full_like(g.q, float("nan"))
+        pkv.paged_attention_decode(out, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale,
+                                   g.max_context_len, workspace=ws)
+        torch.cuda.synchronize()
+        assert_close(out, ref)
+        assert pkv.pkv_device_status(0) == 0
+
+
+@pytest.mark.parametrize("dtype,lens,G,D", [
+    (torch.bfloat16, [131072, 70001, 1, 512], 4, 128),   # 256 partitions merged by one CTA
+    (torch.float32, [40000, 3], 4, 64),
+])
+def test_longest_contexts(dtype, lens, G, D):
+    w = make_custom(lens, 2 * G, 2, D, dtype, seed=33)
+    _run_full_parity(w)
+
+
 def test_bounded_wait_times_out_and_context_survives():
     """A wait on a barrier nothing arrives on gives up after its limit and
     reports PKV_DEV_WAIT_TIMEOUT; the GPU keeps working afterwards."""

@@ -81,6 +81,16 @@ __device__ __forceinline__ void grid_dependency_wait()
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// A read-only 32-bit global load kept where it is written (volatile asm): a
+// kernel issues it ahead of the branches that decide whether the value is
+// used, so independent loads travel together.
+__device__ __forceinline__ int32_t ld_early(const int32_t* p)
+{
+    int32_t v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ void raise_flag(int* status, int flag)
 {
     if (status) atomicOr(status, flag);

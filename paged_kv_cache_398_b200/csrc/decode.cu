@@ -174,11 +174,11 @@ struct SeqRange {
     bool bad;      // context length < 1
 };
 
-__device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int block_size,
-                                              int max_ctx, bool report, int* status)
+// Checks and clamps a sequence's context length (ctx as loaded).
+__device__ __forceinline__ SeqRange seq_range_of(int ctx, int mb, int block_size, int max_ctx, bool report,
+                                                 int* status)
 {
     SeqRange r;
-    int ctx = __ldg(context_lens + s);
     int flag = 0;
     if (ctx < 1) {
         flag = 1;
@@ -197,6 +197,12 @@ __device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s
     r.nparts = (ctx + kPartTokens - 1) / kPartTokens;
     r.bad = ctx < 1;
     return r;
+}
+
+__device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int block_size,
+                                              int max_ctx, bool report, int* status)
+{
+    return seq_range_of(__ldg(context_lens + s), mb, block_size, max_ctx, report, status);
 }
 
 template <typename T, int D, int G, int B>

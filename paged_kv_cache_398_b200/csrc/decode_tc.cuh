@@ -205,7 +205,19 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = kMQ ? q_len * G : G;  // live query rows
 
-    SeqRange sr = seq_range(context_lens, s, mb, B, max_ctx, p == 0 && h == 0 && threadIdx.x == 0, status);
+    // The context length and this thread's entry of the partition's table
+    // slice are loaded together: the entry depends only on (s, p), so the
+    // slice does not wait for the length (one memory round trip before the
+    // first tile copies instead of two).  Entries past the sequence's own
+    // blocks are loaded but never used.
+    constexpr int kPartBlocks = kPartTokens / B;
+    static_assert(kPartBlocks <= kWarps * 32, "one table entry per thread");
+    const int blk0 = p * kPartBlocks;
+    int32_t blk_raw = -1;
+    if ((int)threadIdx.x < kPartBlocks && blk0 + (int)threadIdx.x < mb)
+        blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+    SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx,
+                               p == 0 && h == 0 && threadIdx.x == 0, status);
     if (!sr.bad && sr.ctx < q_len) {
         if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
         sr.bad = true;
@@ -223,9 +235,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (p >= sr.nparts) return;
 
     const int ctx = sr.ctx;
-    constexpr int kPartBlocks = kPartTokens / B;
     const int nblk_seq = (ctx + B - 1) / B;
-    const int blk0 = p * kPartBlocks;
     const int nbp = min(kPartBlocks, nblk_seq - blk0);                          // blocks of this partition
     const int nb = min(kPartTiles, (ctx - p * kPartTokens + kTile - 1) / kTile);  // its 16-token tiles
     const int first_new = ctx - q_len;   // position of the first new token
@@ -234,13 +244,13 @@ __global__ void __launch_bounds__(kWarps * 32)
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
     const uint32_t tiles = pkv::smem_addr(smem + warp * (kStages * C::kStageBytes));
 
-    for (int i = threadIdx.x; i < nbp; i += blockDim.x) {
-        int b = __ldg(block_tables + (int64_t)s * mb + blk0 + i);
+    if ((int)threadIdx.x < nbp) {  // nbp <= kPartBlocks, and blk0 + nbp <= mb
+        int b = blk_raw;
         if (b < 0 || b >= num_blocks) {
             pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
             b = -1;  // read block 0 in its place; never write through it
         }
-        s_blk[i] = b;
+        s_blk[threadIdx.x] = b;
     }
     if (lane == 0) {
 #pragma unroll

@@ -139,6 +139,21 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
+// Keep-in-L2 policy for data the next kernel reads back soon (split-K
+// records), so the cache stream of the partition kernel does not push them
+// out to DRAM first.
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void st_global_hint(float* ptr, float v, uint64_t policy)
+{
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(ptr), "f"(v), "l"(policy) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;

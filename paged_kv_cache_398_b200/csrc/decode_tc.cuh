@@ -523,10 +523,12 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (sr.nparts == 1) {
             pkv::store_out(out + orow * D + d, O / L);
         } else {
-            ws_acc[(orow * max_parts + p) * D + d] = O;
+            // the reduce reads these right after this kernel: keep them in L2
+            const uint64_t keep = pkv::policy_evict_last();
+            pkv::st_global_hint(ws_acc + (orow * max_parts + p) * D + d, O, keep);
             if (d == 0) {
-                ws_ml[(orow * max_parts + p) * 2] = M;
-                ws_ml[(orow * max_parts + p) * 2 + 1] = L;
+                pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2, M, keep);
+                pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2 + 1, L, keep);
             }
         }
     }

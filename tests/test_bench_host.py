@@ -50,3 +50,15 @@ def test_parity_summary_counts_out_of_tolerance_elements():
     st.out[1, 2, 3] += 0.5
     rep = bench.parity_on_sample(st, base)
     assert rep["out_of_tolerance"] == 1 and rep["max_abs_err"] > 0.49
+
+
+def test_event_brackets_are_few_and_spread():
+    for steps in (1, 3, 20, 59, 60, 61, 119, 600, 1500):
+        idx = bench.sampled_steps(steps)
+        assert idx == sorted(set(idx)) and all(0 <= i < steps for i in idx)
+        assert 1 <= len(idx) <= 60
+        if steps <= 60:
+            assert len(idx) == steps            # short runs bracket every step
+    idx = bench.sampled_steps(1500)
+    gaps = {b - a for a, b in zip(idx, idx[1:])}
+    assert gaps == {25} and len(idx) == 60

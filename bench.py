@@ -160,7 +160,8 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.decode_bytes = (st.kv_bytes + 2 * S * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S)
     st.write_bytes = 2 * 2 * S * w.num_kv_heads * w.head_dim * e + 8 * S
     st.copy_bytes = 2 * 2 * pairs.shape[0] * w.num_kv_heads * w.block_size * w.head_dim * e
-    st.max_parts = (st.max_ctx + pkv.PARTITION_TOKENS - 1) // pkv.PARTITION_TOKENS
+    st.part_tokens = pkv.paged_attention_partition_tokens(S, w.num_kv_heads, st.max_ctx, w.dtype)
+    st.max_parts = (st.max_ctx + st.part_tokens - 1) // st.part_tokens
     st.launches_separate = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
     st.launches_fused = st.launches_separate - 1
     return st
@@ -598,6 +599,7 @@ def run_ours(args):
                    "num_q_heads": st.w.num_q_heads, "num_kv_heads": st.w.num_kv_heads,
                    "head_dim": st.w.head_dim, "block_size": st.w.block_size,
                    "context_tokens": int(st.lens_host.sum()), "max_context_len": st.max_ctx,
+                   "partition_tokens": st.part_tokens,
                    "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB of K/V per step), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": 100.0 * value / peak,

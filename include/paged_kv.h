@@ -98,13 +98,39 @@ int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_
                    void* stream);
 
 /*
+ * Split-K partitions.  Decode splits each sequence into partitions of
+ * PKV_PARTITION_TOKENS tokens, one thread block each, and merges them.  A
+ * launch uses PKV_PARTITION_TOKENS_LONG instead when it is fp16 / bf16,
+ * max_context_len >= PKV_LONG_MIN_CONTEXT, and num_seqs * num_kv_heads >=
+ * PKV_LONG_MIN_PAIRS_PER_SM x the device's multiprocessor count.  Such a
+ * batch fills the GPU with (sequence, kv head) pairs alone, and halving its
+ * thread-block count saves more fixed per-block cost than the longer
+ * blocks add to the tail.  The choice depends only on these launch values,
+ * so calls with the same shape always split the same way.
+ */
+#define PKV_PARTITION_TOKENS 512
+#define PKV_PARTITION_TOKENS_LONG 1024
+#define PKV_LONG_MIN_CONTEXT 4096
+#define PKV_LONG_MIN_PAIRS_PER_SM 12
+
+/*
+ * paged_attention_partition_tokens -- the partition size, in tokens, that
+ * paged_attention_decode and paged_attention_decode_mq use for this launch
+ * shape on the current device (rule above).  Returns PKV_PARTITION_TOKENS,
+ * PKV_PARTITION_TOKENS_LONG, or a negative PKV_ERR_* code (no CUDA device:
+ * PKV_ERR_CUDA).
+ */
+int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,
+                                         int32_t dtype);
+
+/*
  * paged_attention_workspace_bytes -- size of the workspace that
  * paged_attention_decode needs for this batch shape.  The value is 0 when
  * max_context_len fits in one partition (PKV_PARTITION_TOKENS tokens).
  * Otherwise the workspace holds, per (sequence, query head, partition), an
- * fp32 running max, an fp32 sum and head_dim fp32 partial outputs.
+ * fp32 running max, an fp32 sum and head_dim fp32 partial outputs.  It is
+ * sized for PKV_PARTITION_TOKENS partitions, which covers the long ones too.
  */
-#define PKV_PARTITION_TOKENS 512
 size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                        int32_t max_context_len);
 

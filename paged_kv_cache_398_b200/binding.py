@@ -19,6 +19,7 @@ from ._lib import C, PagedKVError, check, lib
 _DTYPE = {torch.float32: C["PKV_F32"], torch.float16: C["PKV_F16"], torch.bfloat16: C["PKV_BF16"]}
 BLOCK_SIZE = 16
 PARTITION_TOKENS = C["PKV_PARTITION_TOKENS"]
+PARTITION_TOKENS_LONG = C["PKV_PARTITION_TOKENS_LONG"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -72,6 +73,17 @@ def paged_kv_write(k_new, v_new, k_cache, v_cache, slot_mapping, stream=None) ->
 def paged_attention_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
                                     max_context_len: int) -> int:
     return int(lib().paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
+
+
+def paged_attention_partition_tokens(num_seqs: int, num_kv_heads: int, max_context_len: int,
+                                     dtype: torch.dtype) -> int:
+    """Split-K partition size (tokens) a decode launch of this shape uses on
+    the current CUDA device: PARTITION_TOKENS or PARTITION_TOKENS_LONG."""
+    if dtype not in _DTYPE:
+        raise PagedKVError("dtype", C["PKV_ERR_UNSUPPORTED"])
+    rc = int(lib().paged_attention_partition_tokens(num_seqs, num_kv_heads, max_context_len, _DTYPE[dtype]))
+    check("paged_attention_partition_tokens", min(rc, 0))
+    return rc
 
 
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,

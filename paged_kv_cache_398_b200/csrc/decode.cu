@@ -41,9 +41,10 @@
 namespace {
 
 constexpr int kTile = 16;                          // tokens per compute tile
-constexpr int kPartTokens = PKV_PARTITION_TOKENS;
-constexpr int kPartTiles = kPartTokens / kTile;    // tiles per partition
-constexpr int kMaxPartBlocks = kPartTokens / 8;    // blocks per partition at the smallest block size
+constexpr int kPartTokens = PKV_PARTITION_TOKENS;          // partition of an ordinary launch
+constexpr int kLongPartTokens = PKV_PARTITION_TOKENS_LONG;  // large batches of long contexts (fp16 / bf16)
+constexpr int kPartTiles = kPartTokens / kTile;             // tiles per ordinary partition
+constexpr int kMaxPartBlocks = kLongPartTokens / 8;         // blocks per partition, at most
 constexpr int kWarps = 4;
 constexpr int kStages = 2;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
@@ -174,9 +175,10 @@ struct SeqRange {
     bool bad;      // context length < 1
 };
 
-// Checks and clamps a sequence's context length (ctx as loaded).
-__device__ __forceinline__ SeqRange seq_range_of(int ctx, int mb, int block_size, int max_ctx, bool report,
-                                                 int* status)
+// Checks and clamps a sequence's context length (ctx as loaded); the
+// sequence splits into partitions of part_tokens tokens.
+__device__ __forceinline__ SeqRange seq_range_of(int ctx, int mb, int block_size, int max_ctx, int part_tokens,
+                                                 bool report, int* status)
 {
     SeqRange r;
     int flag = 0;
@@ -194,15 +196,15 @@ __device__ __forceinline__ SeqRange seq_range_of(int ctx, int mb, int block_size
     }
     if (flag && report) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
     r.ctx = ctx;
-    r.nparts = (ctx + kPartTokens - 1) / kPartTokens;
+    r.nparts = (ctx + part_tokens - 1) / part_tokens;
     r.bad = ctx < 1;
     return r;
 }
 
 __device__ __forceinline__ SeqRange seq_range(const int32_t* context_lens, int s, int mb, int block_size,
-                                              int max_ctx, bool report, int* status)
+                                              int max_ctx, int part_tokens, bool report, int* status)
 {
-    return seq_range_of(__ldg(context_lens + s), mb, block_size, max_ctx, report, status);
+    return seq_range_of(__ldg(context_lens + s), mb, block_size, max_ctx, part_tokens, report, status);
 }
 
 template <typename T, int D, int G, int B>
@@ -220,8 +222,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const SeqRange sr = seq_range(context_lens, s, mb, B, max_ctx, p == 0 && h == 0 && threadIdx.x == 0,
-                                  status);
+    const SeqRange sr =
+        seq_range(context_lens, s, mb, B, max_ctx, kPartTokens, p == 0 && h == 0 && threadIdx.x == 0, status);
     if (sr.bad) {
         // nothing to attend to: a zero row (flagged above)
         if (p == 0) {
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(128)
     decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
                          const float* __restrict__ ws_ml, const int32_t* __restrict__ context_lens,
                          int32_t num_seqs, int32_t q_len, int32_t num_q_heads, int32_t mb, int32_t block_size,
-                         int32_t max_ctx, int32_t max_parts)
+                         int32_t max_ctx, int32_t part_tokens, int32_t max_parts)
 {
     constexpr int kPer = D / 32;
     using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
@@ -499,7 +501,7 @@ __global__ void __launch_bounds__(128)
     const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= (int64_t)num_seqs * q_len * num_q_heads) return;   // row = (s * q_len + j) * Hq + i
     const int s = (int)(row / ((int64_t)q_len * num_q_heads));
-    const SeqRange sr = seq_range(context_lens, s, mb, block_size, max_ctx, false, nullptr);
+    const SeqRange sr = seq_range(context_lens, s, mb, block_size, max_ctx, part_tokens, false, nullptr);
     if (sr.bad || sr.ctx < q_len || sr.nparts <= 1) return;   // zero rows / single partition: written
     const float* ml = ws_ml + row * max_parts * 2;
     const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
@@ -638,16 +640,61 @@ struct DecodeArgs {
     int32_t Hkv;
     int32_t NB;
     int32_t block_size;
+    int32_t part_tokens;  // kPartTokens or kLongPartTokens (part_tokens_for)
     float scale;
     void* ws;
     cudaStream_t stream;
     int* status;
 };
 
+// Multiprocessor count of the current device, read once per device.
+int sm_count(int* out)
+{
+    static int cached[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+        return PKV_ERR_CUDA;
+    }
+    if (cached[dev] == 0) {
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess || n < 1) {
+            pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidValue : e);
+            return PKV_ERR_CUDA;
+        }
+        cached[dev] = n;
+    }
+    *out = cached[dev];
+    return PKV_OK;
+}
+
+// Partition size of a launch.  A partition CTA has a fixed cost besides its
+// stream of tiles: the prologue, the merge of its warps, its split-K record,
+// and the CTAs past a shorter sequence's end that start only to exit.  On a
+// large batch of long contexts, partitions of kLongPartTokens halve the CTA
+// count and that cost; a batch of (sequence, kv head) pairs that alone fills
+// every SM several times over keeps the GPU busy, and contexts of at least
+// PKV_LONG_MIN_CONTEXT tokens still split into several partitions.  Smaller
+// or shorter batches keep kPartTokens for parallelism and a short tail.
+// The choice depends only on the launch shape, so it is the same for every
+// call with that shape (bitwise-repeatable results).  fp32 keeps kPartTokens.
+int part_tokens_for(int32_t dtype, int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int* out)
+{
+    *out = kPartTokens;
+    if (dtype == PKV_F32 || max_context_len < PKV_LONG_MIN_CONTEXT) return PKV_OK;
+    int sms = 0;
+    const int rc = sm_count(&sms);
+    if (rc != PKV_OK) return rc;
+    if ((int64_t)num_seqs * num_kv_heads >= (int64_t)PKV_LONG_MIN_PAIRS_PER_SM * sms) *out = kLongPartTokens;
+    return PKV_OK;
+}
+
 template <typename T, int D, int G, int B>
 int launch(const DecodeArgs& a)
 {
-    const int max_parts = (a.max_ctx + kPartTokens - 1) / kPartTokens;
+    const int max_parts = (a.max_ctx + a.part_tokens - 1) / a.part_tokens;
     const int64_t qrows = (int64_t)a.S * a.q_len * a.Hq;  // (sequence, new token, query head) rows
     float* ws_acc = static_cast<float*>(a.ws);
     float* ws_ml = ws_acc ? ws_acc + (size_t)qrows * max_parts * D : nullptr;
@@ -673,20 +720,23 @@ int launch(const DecodeArgs& a)
                                       static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.q_len, a.Hq, a.Hkv,
                                       a.NB, scale_log2, max_parts, a.status);
         };
-        if (a.q_len > 1) {
-            static bool configured[64] = {};
-            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, true, B>, C::kSmemBytes, configured)) != PKV_OK)
-                return rc;
-            launch_err = args(decode_partition_tc_kernel<T, D, G, true, B>);
-        } else {
-            static bool configured[64] = {};
-            if ((rc = allow_smem(decode_partition_tc_kernel<T, D, G, false, B>, C::kSmemBytes, configured)) != PKV_OK)
-                return rc;
-            launch_err = args(decode_partition_tc_kernel<T, D, G, false, B>);
-        }
+        // one instantiation per (multi-query, partition size); each sets its
+        // shared-memory limit once per device
+        auto run = [&](auto kernel, bool* configured) {
+            const int r = allow_smem(kernel, C::kSmemBytes, configured);
+            if (r == PKV_OK) launch_err = args(kernel);
+            return r;
+        };
+        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
+        static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
+        if (!mq && !wide) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
+        else if (!mq) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);
+        else if (!wide) rc = run(decode_partition_tc_kernel<T, D, G, true, B, kPartTokens>, cfg_m);
+        else rc = run(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens>, cfg_mw);
+        if (rc != PKV_OK) return rc;
     } else {
         // fp32: CUDA-core kernel fed by 1-D bulk copies (one query, no fused write)
-        if (a.q_len != 1 || a.k_new) return PKV_ERR_UNSUPPORTED;
+        if (a.q_len != 1 || a.k_new || a.part_tokens != kPartTokens) return PKV_ERR_UNSUPPORTED;
         using C = Cfg<T, D, G>;
         static bool configured[64] = {};
         rc = allow_smem(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured);
@@ -710,7 +760,8 @@ int launch(const DecodeArgs& a)
     pkv::pdl_attribute(&cfg, attr);
     const cudaError_t reduce_err =
         cudaLaunchKernelEx(&cfg, decode_reduce_kernel<T, D>, static_cast<T*>(a.out), (const float*)ws_acc,
-                           (const float*)ws_ml, a.cl, a.S, a.q_len, a.Hq, a.mb, B, a.max_ctx, max_parts);
+                           (const float*)ws_ml, a.cl, a.S, a.q_len, a.Hq, a.mb, B, a.max_ctx, a.part_tokens,
+                           max_parts);
     if (reduce_err != cudaSuccess) {
         pkv::record_cuda_error(reduce_err);
         return PKV_ERR_CUDA;
@@ -779,10 +830,13 @@ int decode_entry(void* out, const void* q, const void* k_new, const void* v_new,
         return PKV_ERR_INVALID_ARG;
     int* status = pkv::status_word_for_current_device();
     if (!status) return PKV_ERR_CUDA;
+    int part_tokens = kPartTokens;
+    const int rc = part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, &part_tokens);
+    if (rc != PKV_OK) return rc;
     const DecodeArgs a{out,           q,        k_new,          v_new,        k_cache,      v_cache,
                        block_tables,  max_blocks_per_seq,       context_lens, num_seqs,     q_len,
-                       max_context_len, num_q_heads, num_kv_heads, num_blocks, block_size, scale, workspace,
-                       (cudaStream_t)stream, status};
+                       max_context_len, num_q_heads, num_kv_heads, num_blocks, block_size, part_tokens, scale,
+                       workspace,     (cudaStream_t)stream,     status};
     switch (dtype) {
         case PKV_F32: return dispatch_d<float>(head_dim, G, a);
         case PKV_F16: return dispatch_d<__half>(head_dim, G, a);
@@ -799,6 +853,16 @@ extern "C" size_t paged_attention_mq_workspace_bytes(int32_t num_seqs, int32_t q
     const size_t parts = ((size_t)max_context_len + kPartTokens - 1) / kPartTokens;
     if (parts <= 1) return 0;
     return (size_t)num_seqs * q_len * num_q_heads * parts * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+extern "C" int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,
+                                                    int32_t dtype)
+{
+    if (num_seqs < 0 || num_kv_heads < 1 || max_context_len < 1) return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    int part_tokens = kPartTokens;
+    const int rc = part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, &part_tokens);
+    return rc != PKV_OK ? rc : part_tokens;
 }
 
 extern "C" size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,

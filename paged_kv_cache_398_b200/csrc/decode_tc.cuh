@@ -183,7 +183,9 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 // k_new / v_new non-null: the new tokens' K/V rows [S][q_len][Hkv][D] are
 // written to their slots (through the block table) by the CTA whose
 // partition holds them, and patched into the staged tiles before use.
-template <typename T, int D, int G, bool kMQ, int B>
+// PT: partition size in tokens (kPartTokens, or kLongPartTokens for large
+// batches of long contexts).
+template <typename T, int D, int G, bool kMQ, int B, int PT>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
@@ -195,6 +197,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                                int32_t max_parts, int* status)
 {
     using C = TcCfg<D>;
+    constexpr int part_tokens = PT;
+    static_assert(PT == kPartTokens || PT == kLongPartTokens, "partition sizes");
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
     constexpr int kRows = kMQ ? 16 : G;  // operand rows that can hold queries
     constexpr int kChunks = D / 8;       // 16-byte chunks per K or V row
@@ -210,13 +214,13 @@ __global__ void __launch_bounds__(kWarps * 32)
     // slice does not wait for the length (one memory round trip before the
     // first tile copies instead of two).  Entries past the sequence's own
     // blocks are loaded but never used.
-    constexpr int kPartBlocks = kPartTokens / B;
-    static_assert(kPartBlocks <= kWarps * 32, "one table entry per thread");
-    const int blk0 = p * kPartBlocks;
+    constexpr int part_blocks = part_tokens / B;
+    static_assert(part_blocks <= kWarps * 32 && part_blocks <= kMaxPartBlocks, "one table entry per thread");
+    const int blk0 = p * part_blocks;
     int32_t blk_raw = -1;
-    if ((int)threadIdx.x < kPartBlocks && blk0 + (int)threadIdx.x < mb)
+    if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
         blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
-    SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx,
+    SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens,
                                p == 0 && h == 0 && threadIdx.x == 0, status);
     if (!sr.bad && sr.ctx < q_len) {
         if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
@@ -236,15 +240,16 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int ctx = sr.ctx;
     const int nblk_seq = (ctx + B - 1) / B;
-    const int nbp = min(kPartBlocks, nblk_seq - blk0);                          // blocks of this partition
-    const int nb = min(kPartTiles, (ctx - p * kPartTokens + kTile - 1) / kTile);  // its 16-token tiles
+    const int part0 = p * part_tokens;                                         // its first position
+    const int nbp = min(part_blocks, nblk_seq - blk0);                          // blocks of this partition
+    const int nb = min(part_tokens / kTile, (ctx - part0 + kTile - 1) / kTile);  // its 16-token tiles
     const int first_new = ctx - q_len;   // position of the first new token
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
     const uint32_t tiles = pkv::smem_addr(smem + warp * (kStages * C::kStageBytes));
 
-    if ((int)threadIdx.x < nbp) {  // nbp <= kPartBlocks, and blk0 + nbp <= mb
+    if ((int)threadIdx.x < nbp) {  // nbp <= part_blocks, and blk0 + nbp <= mb
         int b = blk_raw;
         if (b < 0 || b >= num_blocks) {
             pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         const uint32_t kbase = tiles + st * C::kStageBytes;
         const uint32_t vbase = kbase + C::kTileBytes;
         const int tile = warp + k * kWarps;
-        const int pos0 = p * kPartTokens + tile * kTile;
+        const int pos0 = part0 + tile * kTile;
 
         // ---- fused slot write: this tile holds new tokens -> store and patch
         if (k_new != nullptr && pos0 + kTile > first_new) {
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                 const int jj = jlo + it / (2 * kChunks);
                 const int t = first_new + jj - pos0;                  // row in the tile
                 const int pos = first_new + jj;                          // position in the sequence
-                const int phys = s_blk[(pos - p * kPartTokens) / B];
+                const int phys = s_blk[(pos - part0) / B];
                 const T* src = (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8;
                 const uint4 val = *reinterpret_cast<const uint4*>(src);
                 st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 + (((c % 8) ^ (t & 7)) << 4),

@@ -75,6 +75,12 @@ def test_host_side_rejections(L):
     assert L.paged_attention_decode(p, p, p, p, p, 4, p, 2, 1000, 32, 8, 128, 16, 10,
                                     ctypes.c_float(0.1), 2, p, 100, None) == INV
     assert L.paged_attention_workspace_bytes(2, 32, 128, 512) == 0
+    # the partition-size query: answers that need no device, and rejections
+    assert L.paged_attention_partition_tokens(256, 8, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS"]
+    assert L.paged_attention_partition_tokens(4096, 8, 8192, C["PKV_F32"]) == C["PKV_PARTITION_TOKENS"]
+    assert L.paged_attention_partition_tokens(-1, 8, 100, C["PKV_BF16"]) == INV
+    assert L.paged_attention_partition_tokens(4, 0, 100, C["PKV_BF16"]) == INV
+    assert L.paged_attention_partition_tokens(4, 8, 100, 7) == UNS
     # order-dependent copy lists are rejected on the host
     dummy = ctypes.c_void_p(p)
     for pairs in ([[1, 1]], [[1, 2], [3, 2]], [[1, 2], [2, 3]], [[0, 8]], [[-1, 2]]):

@@ -383,6 +383,68 @@ def test_longest_contexts(dtype, lens, G, D):
     _run_full_parity(w)
 
 
+# ---------------------------------------------------------------------------
+# long partitions: a batch with enough (sequence, kv head) pairs and a long
+# maximum context splits into partitions of PARTITION_TOKENS_LONG tokens
+# ---------------------------------------------------------------------------
+def _long_mode_lens(seed, n_short):
+    g = torch.Generator().manual_seed(seed)
+    short = torch.randint(1, 200, (n_short,), generator=g).tolist()
+    return short[:n_short // 2] + [4096, 9000, 1025, 5000, 2048] + short[n_short // 2:]
+
+
+def test_partition_rule_on_this_device():
+    C = pkv._lib.C
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms
+    bf16, f32 = torch.bfloat16, torch.float32
+    assert pkv.paged_attention_partition_tokens(pairs, 1, 4096, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert pkv.paged_attention_partition_tokens(pairs - 1, 1, 4096, bf16) == pkv.PARTITION_TOKENS
+    assert pkv.paged_attention_partition_tokens(pairs, 1, 4095, bf16) == pkv.PARTITION_TOKENS
+    assert pkv.paged_attention_partition_tokens(pairs, 1, 9000, f32) == pkv.PARTITION_TOKENS
+    # the bench's 8B-GQA batch takes the long partitions, the 7B and 13B batches do not
+    assert pkv.paged_attention_partition_tokens(256, 8, 8130, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert pkv.paged_attention_partition_tokens(64, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS
+    assert pkv.paged_attention_partition_tokens(24, 32, 1986, torch.float16) == pkv.PARTITION_TOKENS
+
+
+@pytest.mark.parametrize("block_size,dtype,D,G", [
+    (16, torch.bfloat16, 128, 4),
+    (8, torch.float16, 64, 8),      # 128 blocks per partition: one table entry per thread
+    (32, torch.bfloat16, 128, 1),
+])
+def test_long_partitions_match_oracle(block_size, dtype, D, G):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    Hkv = 8
+    S = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // Hkv)
+    w = make_custom(_long_mode_lens(40 + block_size, S - 5), Hkv * G, Hkv, D, dtype, seed=41 + block_size,
+                    block_size=block_size, pad_random=True)
+    assert pkv.paged_attention_partition_tokens(S, Hkv, w.max_context_len, dtype) == pkv.PARTITION_TOKENS_LONG
+    _run_full_parity(w)
+
+
+def test_long_partitions_multi_query_fused():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    Hkv, G, D, QL, dtype = 8, 4, 128, 3, torch.bfloat16
+    S = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // Hkv)
+    lens = [max(QL, n) for n in _long_mode_lens(44, S - 5)]
+    w = make_custom(lens, Hkv * G, Hkv, D, dtype, seed=45, q_len=QL)
+    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), lens[s] - QL + j, w.block_size)
+                          for s in range(S) for j in range(QL)], dtype=torch.int64)
+    k_ref, v_ref = w.k_cache.clone(), w.v_cache.clone()
+    oracle.kv_write(k_ref, v_ref, w.k_new.reshape(S * QL, Hkv, D).contiguous(),
+                    w.v_new.reshape(S * QL, Hkv, D).contiguous(), slots)
+    ref = oracle.paged_decode_mq(w.q, k_ref, v_ref, w.block_tables, w.context_lens, w.scale)
+    g = w.to("cuda")
+    out = torch.empty_like(g.q)
+    pkv.paged_attention_decode_mq(out, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale,
+                                  max(lens), k_new=g.k_new, v_new=g.v_new)
+    torch.cuda.synchronize()
+    assert torch.equal(g.k_cache.cpu(), k_ref) and torch.equal(g.v_cache.cpu(), v_ref)
+    assert_close(out, ref)
+    assert pkv.pkv_device_status(0) == 0
+
+
 def test_bounded_wait_times_out_and_context_survives():
     """A wait on a barrier nothing arrives on gives up after its limit and
     reports PKV_DEV_WAIT_TIMEOUT; the GPU keeps working afterwards."""

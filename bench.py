@@ -90,7 +90,7 @@ class Step:
     """Everything one decode step needs, resident on the GPU."""
 
 
-def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16):
+def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16, max_ctx=None):
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 
@@ -98,6 +98,8 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     kw = {}
     if num_seqs:
         kw = {"num_prompts": max(1, num_seqs // 4)} if number == 5 else {"num_seqs": num_seqs}
+    if max_ctx and number in (2, 3, 4):
+        kw["max_ctx"] = max_ctx
     w = make_workload(number, device=device, seed=seed, block_size=block_size, **kw)   # lengths on host, values on the GPU
     S = w.num_seqs
     st = Step()
@@ -511,7 +513,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size)
+    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size, args.max_ctx)
     st.path = args.path
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
@@ -654,6 +656,8 @@ def main():
     ap.add_argument("--reference-seqs", type=int, default=16)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same recipe (profiling); the default is the full workload")
+    ap.add_argument("--max-ctx", type=int, default=None,
+                    help="shorter contexts of the same recipe (profiling; workloads 2-4)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

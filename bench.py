@@ -90,7 +90,12 @@ class Step:
     """Everything one decode step needs, resident on the GPU."""
 
 
-def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16, max_ctx=None):
+def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16, max_ctx=None,
+               q_len: int = 1):
+    """The decode step of workload `number`.  q_len > 1: every sequence
+    brings q_len new tokens (draft tokens to verify, causal among them); its
+    prompt is then ctx - q_len tokens, so the context lengths, and the K/V
+    bytes a step reads, are those of the one-token step."""
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 
@@ -100,6 +105,10 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         kw = {"num_prompts": max(1, num_seqs // 4)} if number == 5 else {"num_seqs": num_seqs}
     if max_ctx and number in (2, 3, 4):
         kw["max_ctx"] = max_ctx
+    if q_len > 1:
+        if number not in (2, 3, 4):
+            raise SystemExit("--q-len > 1 is measured on workloads 2-4")
+        kw["min_ctx"] = q_len + (64 if number == 4 else 0)   # room for the prompt and the new tokens
     w = make_workload(number, device=device, seed=seed, block_size=block_size, **kw)   # lengths on host, values on the GPU
     S = w.num_seqs
     st = Step()
@@ -122,7 +131,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
             system = torch.randint(0, 128000, (64,), generator=gen)
             t0 = time.perf_counter()
             for s in range(S):
-                own = torch.randint(0, 128000, (int(w.context_lens[s]) - 1 - 64,), generator=gen)
+                own = torch.randint(0, 128000, (int(w.context_lens[s]) - q_len - 64,), generator=gen)
                 alloc.add(s)
                 alloc.append_prompt(s, torch.cat([system, own]))
             st.admit_us_per_request = (time.perf_counter() - t0) * 1e6 / S
@@ -131,10 +140,15 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         else:
             for s in range(S):
                 alloc.add(s)
-                alloc.append_tokens(s, int(w.context_lens[s]) - 1)
+                alloc.append_tokens(s, int(w.context_lens[s]) - q_len)
         seqs = list(range(S))
         t0 = time.perf_counter()
-        slots, pairs = alloc.append_one_batch(seqs)          # this step's slots (+ CoW pairs)
+        if q_len == 1:
+            slots, pairs = alloc.append_one_batch(seqs)      # this step's slots (+ CoW pairs)
+        else:
+            per_seq = [alloc.append_tokens(s, q_len) for s in seqs]
+            slots = torch.cat([torch.as_tensor(sl, dtype=torch.int64) for sl, _ in per_seq])
+            pairs = torch.tensor([c for _, c in per_seq if c is not None], dtype=torch.int64).reshape(-1, 2)
         tables, lens = alloc.batch_tables(seqs, w.max_blocks_per_seq)
         st.host_alloc_us = (time.perf_counter() - t0) * 1e6
         assert torch.equal(lens, w.context_lens)
@@ -143,15 +157,25 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.block_tables = tables.to(device)
     st.context_lens = lens.to(device)
     st.slots = slots.to(device)
-    st.q, st.k_cache, st.v_cache = w.q, w.k_cache, w.v_cache
-    st.k_new, st.v_new = w.k_new, w.v_new
-    st.out = torch.empty_like(w.q)
-    # views with one new token per sequence, for the fused path
-    st.q4, st.out4 = st.q.unsqueeze(1), st.out.unsqueeze(1)
-    st.k_new4, st.v_new4 = st.k_new.unsqueeze(1), st.v_new.unsqueeze(1)
+    st.q_len = q_len
+    st.k_cache, st.v_cache = w.k_cache, w.v_cache
+    if q_len == 1:
+        st.q, st.k_new, st.v_new = w.q, w.k_new, w.v_new
+    else:
+        from paged_kv_cache_398_b200.workloads import _randn
+        gd = torch.Generator(device=device).manual_seed(seed + 11)
+        st.q = _randn((S, q_len, w.num_q_heads, w.head_dim), w.dtype, gd, device)
+        st.k_new = _randn((S, q_len, w.num_kv_heads, w.head_dim), w.dtype, gd, device)
+        st.v_new = _randn((S, q_len, w.num_kv_heads, w.head_dim), w.dtype, gd, device)
+    st.out = torch.empty_like(st.q)
+    # [S, q_len, ...] views for paged_attention_decode_mq; flat [S * q_len, ...] rows for paged_kv_write
+    lead = (S, q_len)
+    st.q4, st.out4 = st.q.reshape(lead + st.q.shape[-2:]), st.out.reshape(lead + st.out.shape[-2:])
+    st.k_new4, st.v_new4 = (t.reshape(lead + t.shape[-2:]) for t in (st.k_new, st.v_new))
+    st.k_rows, st.v_rows = (t.reshape(S * q_len, *t.shape[-2:]) for t in (st.k_new, st.v_new))
     st.path = "separate"
     st.max_ctx = int(lens.max())
-    ws_bytes = pkv.paged_attention_workspace_bytes(S, w.num_q_heads, w.head_dim, st.max_ctx)
+    ws_bytes = pkv.paged_attention_mq_workspace_bytes(S, q_len, w.num_q_heads, w.head_dim, st.max_ctx)
     st.workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
     e = w.q.element_size()
     ctx = lens.to(torch.int64)
@@ -159,8 +183,8 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.kv_bytes = int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * e
     uniq_blocks = len(set(tables[tables >= 0].tolist())) if number in (4, 5) else int(nblk.sum())
     st.kv_unique_bytes = uniq_blocks * w.num_kv_heads * w.block_size * w.head_dim * 2 * e  # upper bound
-    st.decode_bytes = (st.kv_bytes + 2 * S * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S)
-    st.write_bytes = 2 * 2 * S * w.num_kv_heads * w.head_dim * e + 8 * S
+    st.decode_bytes = (st.kv_bytes + 2 * S * q_len * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S)
+    st.write_bytes = 2 * 2 * S * q_len * w.num_kv_heads * w.head_dim * e + 8 * S * q_len
     st.copy_bytes = 2 * 2 * pairs.shape[0] * w.num_kv_heads * w.block_size * w.head_dim * e
     st.part_tokens = pkv.paged_attention_partition_tokens(S, w.num_kv_heads, st.max_ctx, w.dtype)
     st.max_parts = (st.max_ctx + st.part_tokens - 1) // st.part_tokens
@@ -183,12 +207,15 @@ def run_step(st, ev=None):
     if ev is not None:
         ev[1].record()
     if st.path == "separate":
-        pkv.paged_kv_write(st.k_new, st.v_new, st.k_cache, st.v_cache, st.slots)
+        pkv.paged_kv_write(st.k_rows, st.v_rows, st.k_cache, st.v_cache, st.slots)
     if ev is not None:
         ev[2].record()
-    if st.path == "separate":
+    if st.path == "separate" and st.q_len == 1:
         pkv.paged_attention_decode(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                    st.w.scale, st.max_ctx, workspace=st.workspace)
+    elif st.path == "separate":
+        pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                                      st.w.scale, st.max_ctx, workspace=st.workspace)
     else:
         pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                       st.w.scale, st.max_ctx, k_new=st.k_new4, v_new=st.v_new4,
@@ -513,14 +540,14 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size, args.max_ctx)
+    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size, args.max_ctx, args.q_len)
     st.path = args.path
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
     # the oracle sample is copied off the device before the first product step
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        base = cpu_baseline(st, threads)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and st.q_len == 1:
+        base = cpu_baseline(st, threads)   # (multi-query parity is covered by the GPU tests)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -601,11 +628,12 @@ def run_ours(args):
                    "num_q_heads": st.w.num_q_heads, "num_kv_heads": st.w.num_kv_heads,
                    "head_dim": st.w.head_dim, "block_size": st.w.block_size,
                    "context_tokens": int(st.lens_host.sum()), "max_context_len": st.max_ctx,
-                   "partition_tokens": st.part_tokens,
+                   "partition_tokens": st.part_tokens, "q_len": st.q_len,
                    "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB of K/V per step), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": 100.0 * value / peak,
         "seq_steps_per_s": S * world * args.steps / (ms_max / 1e3),
+        "new_tokens_per_s": S * st.q_len * world * args.steps / (ms_max / 1e3),
         "unique_kv_gbps": uniq_total * args.steps / (ms_max / 1e3) / 1e9,
         "kernel_ms": {"decode_mean": dec_mean, "decode_min": min(dec_ms),
                       "kv_write_mean": statistics.mean(write_ms) if write_ms else None,
@@ -656,6 +684,8 @@ def main():
     ap.add_argument("--reference-seqs", type=int, default=16)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same recipe (profiling); the default is the full workload")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="new tokens per sequence (multi-query decode, e.g. draft tokens to verify; workloads 2-4)")
     ap.add_argument("--max-ctx", type=int, default=None,
                     help="shorter contexts of the same recipe (profiling; workloads 2-4)")
     args = ap.parse_args()

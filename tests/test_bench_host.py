@@ -62,3 +62,21 @@ def test_event_brackets_are_few_and_spread():
     idx = bench.sampled_steps(1500)
     gaps = {b - a for a, b in zip(idx, idx[1:])}
     assert gaps == {25} and len(idx) == 60
+
+
+def test_multi_query_step_layout():
+    """--q-len: every sequence gets q_len new tokens at its last q_len
+    positions; the lengths (and K/V bytes) are those of the one-token step."""
+    from oracle.allocator_model import slot_for_position
+    QL = 4
+    st = bench.build_step(2, torch.device("cpu"), 0, 6, 16, None, QL)
+    one = bench.build_step(2, torch.device("cpu"), 0, 6, 16, None, 1)
+    S = st.w.num_seqs
+    assert torch.equal(st.lens_host, one.lens_host) and st.kv_bytes == one.kv_bytes
+    assert tuple(st.q4.shape) == (S, QL, st.w.num_q_heads, st.w.head_dim)
+    assert tuple(st.k_rows.shape) == (S * QL, st.w.num_kv_heads, st.w.head_dim)
+    for s in range(S):
+        for j in range(QL):
+            pos = int(st.lens_host[s]) - QL + j
+            assert int(st.slots[s * QL + j]) == slot_for_position(st.tables_host[s].tolist(), pos, 16)
+    assert st.pairs.shape == (0, 2)

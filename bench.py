@@ -93,9 +93,9 @@ class Step:
 def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16, max_ctx=None,
                q_len: int = 1):
     """The decode step of workload `number`.  q_len > 1: every sequence
-    brings q_len new tokens (draft tokens to verify, causal among them); its
-    prompt is then ctx - q_len tokens, so the context lengths, and the K/V
-    bytes a step reads, are those of the one-token step."""
+    brings q_len new tokens (draft tokens to verify, causal among them) after
+    a prompt of ctx - q_len tokens; the recipe's shortest context is raised
+    to leave room for them."""
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 

@@ -154,23 +154,34 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v)
                  : "memory");
 }
 
+// The reference max of a score row moves only when a block's max passes it
+// by more than kLazyLog2 (log2 units).  Probabilities then stay below
+// 2^kLazyLog2, so neither the fp32 sums nor the 16-bit P operand can
+// overflow, and the running sums are rescaled on few blocks instead of on
+// every block that raises the max.  The result is the same softmax: the
+// reference cancels in out = acc / l.
+constexpr float kLazyLog2 = 8.0f;
+
 // Online-softmax update of one score row held by a lane quad.  x: this
 // lane's 4 scores (log2 domain, -inf where masked); m / l: the row's
-// running max and this lane's share of the running sum.  Returns the
+// reference max and this lane's share of the running sum.  Returns the
 // factor by which earlier partial outputs must be scaled.  A row that has
 // seen no visible token yet keeps m = -inf, and every factor stays finite.
+
 __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 {
     float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float mn = fmaxf(m, mx);
-    const float mu = mn == -INFINITY ? 0.0f : mn;
-    const float alpha = pkv::fast_exp2(m - mu);
+    float alpha = 1.0f;
+    if (mx > m + kLazyLog2) {  // never while the row has seen nothing (mx = m = -inf)
+        alpha = pkv::fast_exp2(m - mx);
+        m = mx;
+    }
+    const float mu = m == -INFINITY ? 0.0f : m;
 #pragma unroll
     for (int i = 0; i < 4; ++i) x[i] = pkv::fast_exp2(x[i] - mu);
     l = l * alpha + ((x[0] + x[1]) + (x[2] + x[3]));
-    m = mn;
     return alpha;
 }
 
@@ -335,22 +346,36 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (k_new != nullptr && pos0 + kTile > first_new) {
             const int jlo = max(0, pos0 - first_new);
             const int jhi = min(q_len, pos0 + kTile - first_new);
-            const int items = (jhi - jlo) * 2 * kChunks;
-            for (int it = lane; it < items; it += 32) {
-                const int c = it % kChunks;
-                const int kv = (it / kChunks) & 1;
-                const int jj = jlo + it / (2 * kChunks);
-                const int t = first_new + jj - pos0;                  // row in the tile
-                const int pos = first_new + jj;                          // position in the sequence
-                const int phys = s_blk[(pos - part0) / B];
-                const T* src = (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8;
-                const uint4 val = *reinterpret_cast<const uint4*>(src);
-                st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 + (((c % 8) ^ (t & 7)) << 4),
-                             val);
-                if (phys >= 0) {
-                    T* dst = (kv ? v_cache_w : k_cache_w) +
-                             (((int64_t)phys * num_kv_heads + h) * B + pos % B) * D + c * 8;
-                    *reinterpret_cast<uint4*>(dst) = val;
+            const int items = (jhi - jlo) * 2 * kChunks;  // 16-byte chunks: (token, K or V, chunk)
+            constexpr int kBatch = 4;                       // loads a lane has in flight at once
+            for (int it0 = lane; it0 < items; it0 += 32 * kBatch) {
+                uint4 val[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int it = it0 + 32 * u;
+                    if (it < items) {
+                        const int c = it % kChunks, kv = (it / kChunks) & 1, jj = jlo + it / (2 * kChunks);
+                        const T* src = (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8;
+                        val[u] = __ldg(reinterpret_cast<const uint4*>(src));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int it = it0 + 32 * u;
+                    if (it < items) {
+                        const int c = it % kChunks, kv = (it / kChunks) & 1, jj = jlo + it / (2 * kChunks);
+                        const int t = first_new + jj - pos0;  // row in the tile
+                        const int pos = first_new + jj;       // position in the sequence
+                        const int phys = s_blk[(pos - part0) / B];
+                        st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 +
+                                         (((c % 8) ^ (t & 7)) << 4),
+                                     val[u]);
+                        if (phys >= 0) {
+                            T* dst = (kv ? v_cache_w : k_cache_w) +
+                                     (((int64_t)phys * num_kv_heads + h) * B + pos % B) * D + c * 8;
+                            *reinterpret_cast<uint4*>(dst) = val[u];
+                        }
+                    }
                 }
             }
             __syncwarp();
@@ -382,12 +407,15 @@ __global__ void __launch_bounds__(kWarps * 32)
             float mx = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mn = fmaxf(m_a, mx);  // every block has a visible token: finite
-            alpha_a = pkv::fast_exp2(m_a - mn);
+            // every block has a visible token, so mx is finite
+            alpha_a = 1.0f;
+            if (mx > m_a + kLazyLog2) {  // always on the first block (m_a = -inf)
+                alpha_a = pkv::fast_exp2(m_a - mx);
+                m_a = mx;
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xa[i] = pkv::fast_exp2(xa[i] - mn);
+            for (int i = 0; i < 4; ++i) xa[i] = pkv::fast_exp2(xa[i] - m_a);
             l_a = l_a * alpha_a + ((xa[0] + xa[1]) + (xa[2] + xa[3]));
-            m_a = mn;
             pa[0] = Mma<T>::pack(xa[0], xa[1]);
             pa[1] = 0u;
             pa[2] = Mma<T>::pack(xa[2], xa[3]);
@@ -480,58 +508,73 @@ __global__ void __launch_bounds__(kWarps * 32)
         l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
     }
     __syncthreads();
-    float* mg = reinterpret_cast<float*>(smem);  // [kWarps][kRows][D + 2]: m, l, acc[D]
-    static_assert(kWarps * kRows * (D + 2) * 4 <= C::kTilesBytes, "merge area must fit in the tile area");
+    // records [kWarps][kRows][kRec]: m, l, two unused words (acc starts 16-byte aligned), acc[D]
+    constexpr int kRec = D + 4;
+    float* mg = reinterpret_cast<float*>(smem);
+    static_assert(kWarps * kRows * kRec * 4 <= C::kTilesBytes, "merge area must fit in the tile area");
     if (live_a) {
-        float* rec = mg + (warp * kRows + ra) * (D + 2);
+        float* rec = mg + (warp * kRows + ra) * kRec;
         if ((lane & 3) == 0) {
             rec[0] = m_a;
             rec[1] = l_a;
         }
 #pragma unroll
-        for (int n = 0; n < C::kNTiles; ++n) {
-            rec[2 + 8 * n + qd] = o[n][0];
-            rec[2 + 8 * n + qd + 1] = o[n][1];
-        }
+        for (int n = 0; n < C::kNTiles; ++n)
+            *reinterpret_cast<float2*>(rec + 4 + 8 * n + qd) = make_float2(o[n][0], o[n][1]);
     }
     if constexpr (kMQ) {
         if (live_b) {
-            float* rec = mg + (warp * kRows + rb) * (D + 2);
+            float* rec = mg + (warp * kRows + rb) * kRec;
             if ((lane & 3) == 0) {
                 rec[0] = m_b;
                 rec[1] = l_b;
             }
 #pragma unroll
-            for (int n = 0; n < C::kNTiles; ++n) {
-                rec[2 + 8 * n + qd] = o[n][2];
-                rec[2 + 8 * n + qd + 1] = o[n][3];
-            }
+            for (int n = 0; n < C::kNTiles; ++n)
+                *reinterpret_cast<float2*>(rec + 4 + 8 * n + qd) = make_float2(o[n][2], o[n][3]);
         }
     }
     __syncthreads();
 
-    for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
-        const int r = i / D, d = i % D;
+    // One warp per query row, each lane owning head_dim / 32 consecutive
+    // outputs; the weights of the warps' records are computed once per row.
+    constexpr int kPer = D / 32;
+    using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
+    for (int r = warp; r < rows; r += kWarps) {
+        float mw[kWarps];
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[(w * kRows + r) * (D + 2)]);
+        for (int w = 0; w < kWarps; ++w) {
+            mw[w] = mg[(w * kRows + r) * kRec];
+            M = fmaxf(M, mw[w]);
+        }
         const float Mu = M == -INFINITY ? 0.0f : M;  // a row that saw no token here: all weights 0
-        float L = 0.0f, O = 0.0f;
+        float L = 0.0f, O[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) O[e] = 0.0f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float* rec = mg + (w * kRows + r) * (D + 2);
-            const float wgt = pkv::fast_exp2(rec[0] - Mu);
+            const float* rec = mg + (w * kRows + r) * kRec;
+            const float wgt = pkv::fast_exp2(mw[w] - Mu);
             L = fmaf(rec[1], wgt, L);
-            O = fmaf(rec[2 + d], wgt, O);
+            const Vec v = *reinterpret_cast<const Vec*>(rec + 4 + lane * kPer);
+            const float* vf = reinterpret_cast<const float*>(&v);
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) O[e] = fmaf(vf[e], wgt, O[e]);
         }
         const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
         if (sr.nparts == 1) {
-            pkv::store_out(out + orow * D + d, O / L);
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) pkv::store_out(out + orow * D + lane * kPer + e, O[e] / L);
         } else {
             // the reduce reads these right after this kernel: keep them in L2
             const uint64_t keep = pkv::policy_evict_last();
-            pkv::st_global_hint(ws_acc + (orow * max_parts + p) * D + d, O, keep);
-            if (d == 0) {
+            Vec ov;
+            float* of = reinterpret_cast<float*>(&ov);
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) of[e] = O[e];
+            pkv::st_global_hint(reinterpret_cast<Vec*>(ws_acc + (orow * max_parts + p) * D) + lane, ov, keep);
+            if (lane == 0) {
                 pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2, M, keep);
                 pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2 + 1, L, keep);
             }

@@ -710,7 +710,9 @@ int launch(const DecodeArgs& a)
         CUtensorMap tm_k, tm_v;
         if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
         if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
-        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
+        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
+        const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
+        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), smem, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
         auto args = [&](auto kernel) {
@@ -723,11 +725,10 @@ int launch(const DecodeArgs& a)
         // one instantiation per (multi-query, partition size); each sets its
         // shared-memory limit once per device
         auto run = [&](auto kernel, bool* configured) {
-            const int r = allow_smem(kernel, C::kSmemBytes, configured);
+            const int r = allow_smem(kernel, smem, configured);
             if (r == PKV_OK) launch_err = args(kernel);
             return r;
         };
-        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
         static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
         if (!mq && !wide) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
         else if (!mq) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);

@@ -116,8 +116,12 @@ struct TcCfg {
     static constexpr int kNTiles = D / 8;                     // P.V n-tiles
     static constexpr int kTilesBytes = kWarps * kStages * kStageBytes;
     static constexpr int kBarOff = kTilesBytes;
-    static constexpr int kBlkOff = kBarOff + kWarps * kStages * 8;
-    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBlkOff + kMaxPartBlocks * 4;
+    static constexpr int kNewBarOff = kBarOff + kWarps * kStages * 8;  // staged new-token rows have landed
+    static constexpr int kBlkOff = kNewBarOff + 8;
+    static constexpr int kNewOff = (kBlkOff + kMaxPartBlocks * 4 + 15) & ~15;  // staged new-token rows
+    static constexpr int kNewRowBytes = 2 * D * 2;                        // one token's K and V rows
+    // dynamic shared memory of a launch whose CTAs stage up to new_rows new tokens
+    static constexpr int smem_bytes(int new_rows) { return 1024 /* alignment slack */ + kNewOff + new_rows * kNewRowBytes; }
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
 };
 
@@ -147,6 +151,30 @@ __device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUte
         }
     }
 }
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// 16 bytes global -> shared (cp.async, cached in L2 only), completing on the
+// issuing thread's cp.async tracking.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued before has landed
+// (the barrier's count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(pkv::smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v)
 {
@@ -255,6 +283,18 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int nbp = min(part_blocks, nblk_seq - blk0);                          // blocks of this partition
     const int nb = min(part_tokens / kTile, (ctx - part0 + kTile - 1) / kTile);  // its 16-token tiles
     const int first_new = ctx - q_len;   // position of the first new token
+    // Fused write: the new tokens that fall in this partition, as token
+    // indices [jlo_p, jhi_p).  With several new tokens, right after the
+    // prologue every thread stages some of their K / V rows in shared memory
+    // by cp.async, so the warp that writes and patches them later never waits
+    // on global memory.  A single new token (kMQ false) is one 16-byte load
+    // per lane, done where it is patched.
+    constexpr int kNewRows = kMQ ? 16 : 0;  // capacity of the staging area, in tokens
+    const int jlo_p = max(0, part0 - first_new);
+    const int jhi_p = min(q_len, part0 + part_tokens - first_new);
+    const bool stage_new = kMQ && k_new != nullptr && jhi_p > jlo_p;  // the same for the whole CTA
+    uint64_t* new_bar = reinterpret_cast<uint64_t*>(smem + C::kNewBarOff);
+    const uint32_t new_rows = pkv::smem_addr(smem + C::kNewOff);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff) + warp * kStages;
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
@@ -271,6 +311,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (lane == 0) {
 #pragma unroll
         for (int st = 0; st < kStages; ++st) pkv::mbar_init(&bars[st], 1);
+        if (warp == 0 && stage_new) pkv::mbar_init(new_bar, kWarps * 32);  // one arrival per thread
         pkv::fence_mbar_init();
     }
     __syncthreads();
@@ -288,6 +329,17 @@ __global__ void __launch_bounds__(kWarps * 32)
                         policy);
         }
     }
+    if (stage_new) {
+        // staging layout [token - jlo_p][K or V][16-byte chunk], chunk index = it
+        const int chunks = (jhi_p - jlo_p) * 2 * kChunks;  // <= kNewRows * 2 * kChunks
+        for (int it = threadIdx.x; it < chunks; it += kWarps * 32) {
+            const int c = it % kChunks, kv = (it / kChunks) & 1, jj = jlo_p + it / (2 * kChunks);
+            cp_async_16(new_rows + it * 16,
+                        (kv ? v_new : k_new) + (((int64_t)s * q_len + jj) * num_kv_heads + h) * D + c * 8);
+        }
+        cp_async_arrive(new_bar);
+    }
+    static_assert(kNewRows * C::kNewRowBytes == kNewRows * 2 * kChunks * 16, "staging row size");
 
     // ---- Q as A fragments: rows ra = lane / 4 (a0, a2) and rb = ra + 8 (a1, a3)
     const int ra = lane >> 2, rb = ra + 8;
@@ -343,11 +395,35 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int pos0 = part0 + tile * kTile;
 
         // ---- fused slot write: this tile holds new tokens -> store and patch
-        if (k_new != nullptr && pos0 + kTile > first_new) {
+        if (stage_new && pos0 + kTile > first_new) {
+            if (!pkv::mbar_wait(new_bar, 0, kWaitLimitNs)) {
+                timed_out = true;
+                break;
+            }
             const int jlo = max(0, pos0 - first_new);
             const int jhi = min(q_len, pos0 + kTile - first_new);
             const int items = (jhi - jlo) * 2 * kChunks;  // 16-byte chunks: (token, K or V, chunk)
-            constexpr int kBatch = 4;                       // loads a lane has in flight at once
+            for (int it = lane; it < items; it += 32) {
+                const int c = it % kChunks, kv = (it / kChunks) & 1, jj = jlo + it / (2 * kChunks);
+                const int t = first_new + jj - pos0;  // row in the tile
+                const int pos = first_new + jj;       // position in the sequence
+                const int phys = s_blk[(pos - part0) / B];
+                const uint4 val = ld_shared_v4(new_rows + (((jj - jlo_p) * 2 + kv) * kChunks + c) * 16);
+                st_shared_v4(kbase + kv * C::kTileBytes + (c / 8) * kTcBoxBytes + t * 128 + (((c % 8) ^ (t & 7)) << 4),
+                             val);
+                if (phys >= 0) {
+                    T* dst = (kv ? v_cache_w : k_cache_w) +
+                             (((int64_t)phys * num_kv_heads + h) * B + pos % B) * D + c * 8;
+                    *reinterpret_cast<uint4*>(dst) = val;
+                }
+            }
+            __syncwarp();
+        } else if (!kMQ && k_new != nullptr && pos0 + kTile > first_new) {
+            // the one new token: loaded here, four 16-byte chunks in flight per lane at most
+            const int jlo = max(0, pos0 - first_new);
+            const int jhi = min(q_len, pos0 + kTile - first_new);
+            const int items = (jhi - jlo) * 2 * kChunks;  // 16-byte chunks: (token, K or V, chunk)
+            constexpr int kBatch = 4;
             for (int it0 = lane; it0 < items; it0 += 32 * kBatch) {
                 uint4 val[kBatch];
 #pragma unroll
@@ -493,6 +569,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
     }
 
+    if (stage_new) cp_async_wait_all();  // no staging copy of this thread is still in flight
     if (timed_out) {
         if (lane == 0) pkv::raise_flag(status, PKV_DEV_WAIT_TIMEOUT);
         for (int k = consumed; k < nw && k < consumed + kStages; ++k) {

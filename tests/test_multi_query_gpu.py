@@ -150,7 +150,7 @@ def test_unsupported_combinations_are_rejected():
 
 @pytest.mark.parametrize("block_size", [8, 32])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("G,q_len", [(1, 1), (4, 3), (2, 8)])
+@pytest.mark.parametrize("G,q_len", [(1, 1), (4, 3), (2, 8), (1, 16)])
 def test_multi_query_fused_block_sizes_8_and_32(block_size, dtype, G, q_len):
     lens = [max(n, q_len) for n in (5, 8, 9, 17, 33, 510, 514, 1031)]
     w = make_custom(lens, 2 * G, 2, 128, dtype, seed=7 * block_size + G + q_len, q_len=q_len,

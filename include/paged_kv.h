@@ -341,6 +341,19 @@ int pkv_debug_wait_timeout(int64_t limit_ns, void* stream);
 /* The last cudaError_t seen by any call in this thread, as an int. */
 int pkv_last_cuda_error(void);
 
+/*
+ * pkv_debug_decode_occupancy -- test hook: thread blocks per SM that the
+ * decode partition kernel of this configuration keeps resident on the
+ * current device (cudaOccupancyMaxActiveBlocksPerMultiprocessor, with the
+ * kernel's own shared memory).  group = num_q_heads / num_kv_heads; q_len > 1
+ * selects the multi-query kernel; long_partitions != 0 the
+ * PKV_PARTITION_TOKENS_LONG variant (fp16 / bf16).  Enqueues nothing.  A
+ * tensor-core kernel is built for 3 per SM (its shared memory and 168
+ * registers); fewer means a build lost a third of the bytes in flight.
+ */
+int pkv_debug_decode_occupancy(int32_t dtype, int32_t head_dim, int32_t group, int32_t q_len,
+                               int32_t block_size, int32_t long_partitions, int32_t* ctas_per_sm);
+
 /* A static, human-readable name for a PKV_* status code. */
 const char* pkv_status_string(int status);
 

@@ -645,7 +645,22 @@ struct DecodeArgs {
     void* ws;
     cudaStream_t stream;
     int* status;
+    int* occupancy_out = nullptr;  // set: report the partition kernel's CTAs per SM, launch nothing
 };
+
+// Resident CTAs per SM of `kernel` with `smem` bytes of dynamic shared memory.
+template <typename K>
+int occupancy_of(K kernel, int smem, bool* configured, int* out)
+{
+    int rc = allow_smem(kernel, smem, configured);
+    if (rc != PKV_OK) return rc;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kernel, kWarps * 32, smem);
+    if (e != cudaSuccess) {
+        pkv::record_cuda_error(e);
+        return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
 
 // Multiprocessor count of the current device, read once per device.
 int sm_count(int* out)
@@ -703,15 +718,28 @@ int launch(const DecodeArgs& a)
     int rc;
     cudaError_t launch_err = cudaSuccess;
     if constexpr (sizeof(T) == 2) {
-        // fp16 / bf16: tensor-core kernel fed by tiled TMA
+        // fp16 / bf16: tensor-core kernel fed by tiled TMA; one instantiation
+        // per (multi-query, partition size), each setting its shared-memory
+        // limit once per device
         using C = TcCfg<D>;
+        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
+        const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
+        static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
+        auto with_kernel = [&](auto&& f) {
+            if (!mq && !wide) return f(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
+            if (!mq) return f(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);
+            if (!wide) return f(decode_partition_tc_kernel<T, D, G, true, B, kPartTokens>, cfg_m);
+            return f(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens>, cfg_mw);
+        };
+        if (a.occupancy_out) {
+            return with_kernel(
+                [&](auto kernel, bool* configured) { return occupancy_of(kernel, smem, configured, a.occupancy_out); });
+        }
         const int64_t rows = (int64_t)a.NB * a.Hkv * B;
         if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
         CUtensorMap tm_k, tm_v;
         if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
         if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
-        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
-        const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
         cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), smem, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
@@ -722,24 +750,19 @@ int launch(const DecodeArgs& a)
                                       static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.q_len, a.Hq, a.Hkv,
                                       a.NB, scale_log2, max_parts, a.status);
         };
-        // one instantiation per (multi-query, partition size); each sets its
-        // shared-memory limit once per device
-        auto run = [&](auto kernel, bool* configured) {
+        rc = with_kernel([&](auto kernel, bool* configured) {
             const int r = allow_smem(kernel, smem, configured);
             if (r == PKV_OK) launch_err = args(kernel);
             return r;
-        };
-        static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
-        if (!mq && !wide) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
-        else if (!mq) rc = run(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);
-        else if (!wide) rc = run(decode_partition_tc_kernel<T, D, G, true, B, kPartTokens>, cfg_m);
-        else rc = run(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens>, cfg_mw);
+        });
         if (rc != PKV_OK) return rc;
     } else {
         // fp32: CUDA-core kernel fed by 1-D bulk copies (one query, no fused write)
         if (a.q_len != 1 || a.k_new || a.part_tokens != kPartTokens) return PKV_ERR_UNSUPPORTED;
         using C = Cfg<T, D, G>;
         static bool configured[64] = {};
+        if (a.occupancy_out)
+            return occupancy_of(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured, a.occupancy_out);
         rc = allow_smem(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured);
         if (rc != PKV_OK) return rc;
         cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), C::kSmemBytes, a.stream);
@@ -864,6 +887,34 @@ extern "C" int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t nu
     int part_tokens = kPartTokens;
     const int rc = part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, &part_tokens);
     return rc != PKV_OK ? rc : part_tokens;
+}
+
+extern "C" int pkv_debug_decode_occupancy(int32_t dtype, int32_t head_dim, int32_t group, int32_t q_len,
+                                          int32_t block_size, int32_t long_partitions, int32_t* ctas_per_sm)
+{
+    if (!ctas_per_sm || q_len < 1) return PKV_ERR_INVALID_ARG;
+    if ((block_size != 8 && block_size != 16 && block_size != 32) || (head_dim != 64 && head_dim != 128) ||
+        (group != 1 && group != 2 && group != 4 && group != 8) || q_len * group > 16 ||
+        (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) ||
+        (dtype == PKV_F32 && (q_len != 1 || long_partitions)))
+        return PKV_ERR_UNSUPPORTED;
+    *ctas_per_sm = 0;
+    DecodeArgs a{};
+    a.S = 1;
+    a.q_len = q_len;
+    a.max_ctx = long_partitions ? kLongPartTokens : kPartTokens;
+    a.Hq = group;
+    a.Hkv = 1;
+    a.NB = 1;
+    a.block_size = block_size;
+    a.part_tokens = long_partitions ? kLongPartTokens : kPartTokens;
+    a.scale = 1.0f;
+    a.occupancy_out = ctas_per_sm;
+    switch (dtype) {
+        case PKV_F32: return dispatch_d<float>(head_dim, group, a);
+        case PKV_F16: return dispatch_d<__half>(head_dim, group, a);
+        default: return dispatch_d<__nv_bfloat16>(head_dim, group, a);
+    }
 }
 
 extern "C" size_t paged_attention_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,

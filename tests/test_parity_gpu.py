@@ -469,3 +469,33 @@ def test_block_sizes_8_and_32(block_size, dtype, D, G):
     lens = [1, 7, 8, 9, 15, 16, 17, 31, 33, 511, 512, 513, 520, 1000, 4100]
     w = make_custom(lens, 2 * G, 2, D, dtype, seed=block_size * 100 + G + D, block_size=block_size)
     _run_full_parity(w)
+
+
+# ---------------------------------------------------------------------------
+# occupancy guard: every tensor-core decode kernel keeps 3 CTAs per SM
+# resident (its shared memory allows 3, and 168 registers per thread fit 3);
+# a build whose register count crept up would silently lose a third of the
+# bytes in flight
+# ---------------------------------------------------------------------------
+def test_every_decode_kernel_keeps_its_occupancy():
+    import ctypes
+    L = pkv._lib.lib()
+    C = pkv._lib.C
+    low = []
+    for dtype in (C["PKV_F16"], C["PKV_BF16"]):
+        for D in (64, 128):
+            for G in (1, 2, 4, 8):
+                for q_len in sorted({1, 16 // G} | ({2} if G <= 8 else set())):
+                    for B in (8, 16, 32):
+                        for long_p in (0, 1):
+                            n = ctypes.c_int32(0)
+                            rc = L.pkv_debug_decode_occupancy(dtype, D, G, q_len, B, long_p, ctypes.byref(n))
+                            assert rc == 0, (dtype, D, G, q_len, B, long_p, rc)
+                            if n.value < 3:
+                                low.append((dtype, D, G, q_len, B, long_p, n.value))
+    assert not low, f"below 3 CTAs per SM: {low}"
+    for D in (64, 128):   # the fp32 kernel (fp32 tiles are twice the bytes: 1 CTA per SM at head_dim 128)
+        n = ctypes.c_int32(0)
+        assert L.pkv_debug_decode_occupancy(C["PKV_F32"], D, 4, 1, 16, 0, ctypes.byref(n)) == 0 and n.value >= 1
+    n = ctypes.c_int32(0)
+    assert L.pkv_debug_decode_occupancy(C["PKV_F32"], 128, 4, 2, 16, 0, ctypes.byref(n)) == C["PKV_ERR_UNSUPPORTED"]

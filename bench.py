@@ -47,6 +47,7 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("paged_kv_cache_398_b200/csrc/decode.cu", "paged_kv_cache_398_b200/csrc/decode_tc.cuh",
                   "paged_kv_cache_398_b200/csrc/common.cuh")
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_traffic.json")
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (the measured copy peak is the roofline denominator)
 
 
 def decode_source_hash() -> str:
@@ -632,6 +633,7 @@ def run_ours(args):
                    "l2": f"inputs larger than L2 ({st.kv_bytes / 1e9:.2f} GB of K/V per step), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": 100.0 * value / peak,
+        "pct_of_nominal_hbm": 100.0 * value / NOMINAL_HBM_GBS,
         "seq_steps_per_s": S * world * args.steps / (ms_max / 1e3),
         "new_tokens_per_s": S * st.q_len * world * args.steps / (ms_max / 1e3),
         "unique_kv_gbps": uniq_total * args.steps / (ms_max / 1e3) / 1e9,

@@ -152,6 +152,15 @@ __device__ __forceinline__ void tc_issue(uint32_t dst, uint64_t* bar, const CUte
     }
 }
 
+// Transpose an 8x8 matrix of 16-bit values held as MMA fragments (lane l
+// holds row l / 4, columns 2 (l % 4) and 2 (l % 4) + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 {
     uint4 v;
@@ -376,9 +385,17 @@ __global__ void __launch_bounds__(kWarps * 32)
     const uint32_t v_row_off = (uint32_t)(((mi & 1) * 8 + r8) * 128);
     const uint32_t v_x = (uint32_t)(((mi >> 1) ^ r8) << 4);
 
-    float o[C::kNTiles][4];
+    // Multi-query: O [16 rows][D] as n-tiles, rows ra (o[.][0..1]) and rb
+    // (o[.][2..3]).  One query: O^T [D][8 rows] as m-tiles (ot), rows qd
+    // (ot[.][0], ot[.][2]) and qd + 1 (ot[.][1], ot[.][3]), head-dim entries
+    // 16 j + ra and 16 j + ra + 8; (m_a, l_a) belong to row qd and (m_b, l_b)
+    // to row qd + 1.
+    float o[kMQ ? C::kNTiles : 1][4];
+    float ot[kMQ ? 1 : C::kNTiles / 2][4];
 #pragma unroll
-    for (int n = 0; n < C::kNTiles; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
+    for (int n = 0; n < (kMQ ? C::kNTiles : 1); ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
+#pragma unroll
+    for (int n = 0; n < (kMQ ? 1 : C::kNTiles / 2); ++n) ot[n][0] = ot[n][1] = ot[n][2] = ot[n][3] = 0.0f;
     float m_a = -INFINITY, l_a = 0.0f, m_b = -INFINITY, l_b = 0.0f;
     bool timed_out = false;
     int consumed = 0;
@@ -457,53 +474,107 @@ __global__ void __launch_bounds__(kWarps * 32)
             __syncwarp();
         }
 
-        // ---- S = Q K^T for the block's 16 tokens (two 8-token tiles)
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < C::kKSteps; ++ks) {
-            uint32_t b[4];
-            const uint32_t addr = kbase + (ks / 4) * kTcBoxBytes + k_row_off + (((uint32_t)(2 * (ks % 4)) << 4) ^ k_x);
-            ldsm_x4(b, addr);
-            Mma<T>::run(s0, qa[ks], b[0], b[1]);
-            Mma<T>::run(s1, qa[ks], b[2], b[3]);
-        }
-
-        // ---- online softmax; this lane holds tokens qd, qd+1, qd+8, qd+9 of rows ra (and rb)
-        const bool mask = pos0 + kTile > first_new + 1;   // some token of this tile is not visible to all rows
-        float xa[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
-        const int tp[4] = {pos0 + qd, pos0 + qd + 1, pos0 + qd + 8, pos0 + qd + 9};
-        float alpha_a, alpha_b = 1.0f;
-        uint32_t pa[4], pl[4];  // P (hi) and, for bf16, its residual (lo)
         if constexpr (!kMQ) {
-            if (mask) {
+            // ---- one query: S^T = K Q^T, the block's 16 tokens as MMA rows and
+            // the (at most 8) query heads as its columns, so the MMA carries no
+            // padding rows.  The K fragments are the same ldmatrix tiles in A
+            // order; Q's fragments serve as the B operand.
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-steps
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (tp[i] >= lim_a) xa[i] = -INFINITY;
+            for (int ks = 0; ks < C::kKSteps; ++ks) {
+                uint32_t b[4];
+                const uint32_t addr =
+                    kbase + (ks / 4) * kTcBoxBytes + k_row_off + (((uint32_t)(2 * (ks % 4)) << 4) ^ k_x);
+                ldsm_x4(b, addr);
+                const uint32_t a[4] = {b[0], b[2], b[1], b[3]};
+                Mma<T>::run(ks % 2 ? sb : sa, a, qa[ks][0], qa[ks][2]);
             }
-            float mx = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            // every block has a visible token, so mx is finite
-            alpha_a = 1.0f;
-            if (mx > m_a + kLazyLog2) {  // always on the first block (m_a = -inf)
-                alpha_a = pkv::fast_exp2(m_a - mx);
-                m_a = mx;
-            }
+            // this lane: tokens ra (x[0], x[1]) and ra + 8 (x[2], x[3]) of rows qd, qd + 1
+            float x[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xa[i] = pkv::fast_exp2(xa[i] - m_a);
-            l_a = l_a * alpha_a + ((xa[0] + xa[1]) + (xa[2] + xa[3]));
-            pa[0] = Mma<T>::pack(xa[0], xa[1]);
-            pa[1] = 0u;
-            pa[2] = Mma<T>::pack(xa[2], xa[3]);
-            pa[3] = 0u;
+            for (int i = 0; i < 4; ++i) x[i] = (sa[i] + sb[i]) * scale_log2;
+            if (pos0 + kTile > ctx) {  // the sequence's last, partial block
+                if (pos0 + ra >= ctx) x[0] = x[1] = -INFINITY;
+                if (pos0 + ra + 8 >= ctx) x[2] = x[3] = -INFINITY;
+            }
+            float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+            for (int sh = 4; sh < 32; sh <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
+            }
+            // every block has a visible token, so both maxima are finite
+            float alpha_a = 1.0f, alpha_b = 1.0f;
+            if (mx0 > m_a + kLazyLog2) {  // always on the first block (m = -inf)
+                alpha_a = pkv::fast_exp2(m_a - mx0);
+                m_a = mx0;
+            }
+            if (mx1 > m_b + kLazyLog2) {
+                alpha_b = pkv::fast_exp2(m_b - mx1);
+                m_b = mx1;
+            }
+            x[0] = pkv::fast_exp2(x[0] - m_a);
+            x[2] = pkv::fast_exp2(x[2] - m_a);
+            x[1] = pkv::fast_exp2(x[1] - m_b);
+            x[3] = pkv::fast_exp2(x[3] - m_b);
+            l_a = l_a * alpha_a + (x[0] + x[2]);
+            l_b = l_b * alpha_b + (x[1] + x[3]);
+            // P^T as the B operand of O^T += V^T P^T: transpose each 8-token half
+            const uint32_t h0 = Mma<T>::pack(x[0], x[1]), h1 = Mma<T>::pack(x[2], x[3]);
+            const uint32_t pb0 = movmatrix_trans(h0), pb1 = movmatrix_trans(h1);
+            uint32_t lb0 = 0u, lb1 = 0u;  // bf16: the residual (lo) of P
             if constexpr (Mma<T>::kSplitP) {
-                pl[0] = Mma<T>::residual(xa[0], xa[1], pa[0]);
-                pl[1] = 0u;
-                pl[2] = Mma<T>::residual(xa[2], xa[3], pa[2]);
-                pl[3] = 0u;
+                lb0 = movmatrix_trans(Mma<T>::residual(x[0], x[1], h0));
+                lb1 = movmatrix_trans(Mma<T>::residual(x[2], x[3], h1));
+            }
+            if (__any_sync(0xffffffffu, alpha_a != 1.0f || alpha_b != 1.0f)) {
+#pragma unroll
+                for (int j = 0; j < C::kNTiles / 2; ++j) {
+                    ot[j][0] *= alpha_a;
+                    ot[j][1] *= alpha_b;
+                    ot[j][2] *= alpha_a;
+                    ot[j][3] *= alpha_b;
+                }
+            }
+            // ---- O^T += V^T P^T: 16 head-dim entries per MMA, the block's
+            // tokens as k.  V rows of tokens at or past the sequence length are
+            // zeroed: whatever the unused slots hold (even NaN) must not reach
+            // the result.  This lane's V^T fragments hold tokens qd, qd + 1
+            // (a0, a1) and qd + 8, qd + 9 (a2, a3).
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+            if (pos0 + kTile > ctx) {
+                const int t = pos0 + qd;
+                keep_lo = (t < ctx ? 0x0000ffffu : 0u) | (t + 1 < ctx ? 0xffff0000u : 0u);
+                keep_hi = (t + 8 < ctx ? 0x0000ffffu : 0u) | (t + 9 < ctx ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < C::kNTiles / 2; ++j) {
+                uint32_t v[4];
+                const uint32_t addr =
+                    vbase + (j / 4) * kTcBoxBytes + v_row_off + (((uint32_t)(2 * (j % 4)) << 4) ^ v_x);
+                ldsm_x4_trans(v, addr);
+                const uint32_t a[4] = {v[0] & keep_lo, v[2] & keep_lo, v[1] & keep_hi, v[3] & keep_hi};
+                Mma<T>::run(ot[j], a, pb0, pb1);
+                if constexpr (Mma<T>::kSplitP) Mma<T>::run(ot[j], a, lb0, lb1);
             }
         } else {
+            // ---- multi-query: S = Q K^T, 16 query rows x the block's 16 tokens (two 8-token tiles)
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < C::kKSteps; ++ks) {
+                uint32_t b[4];
+                const uint32_t addr =
+                    kbase + (ks / 4) * kTcBoxBytes + k_row_off + (((uint32_t)(2 * (ks % 4)) << 4) ^ k_x);
+                ldsm_x4(b, addr);
+                Mma<T>::run(s0, qa[ks], b[0], b[1]);
+                Mma<T>::run(s1, qa[ks], b[2], b[3]);
+            }
+
+            // ---- online softmax; this lane holds tokens qd, qd+1, qd+8, qd+9 of rows ra and rb
+            const bool mask = pos0 + kTile > first_new + 1;  // some token of this tile is not visible to all rows
+            float xa[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2, s1[1] * scale_log2};
             float xb[4] = {s0[2] * scale_log2, s0[3] * scale_log2, s1[2] * scale_log2, s1[3] * scale_log2};
+            const int tp[4] = {pos0 + qd, pos0 + qd + 1, pos0 + qd + 8, pos0 + qd + 9};
             if (mask) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -511,8 +582,9 @@ __global__ void __launch_bounds__(kWarps * 32)
                     if (tp[i] >= lim_b) xb[i] = -INFINITY;
                 }
             }
-            alpha_a = softmax_row(xa, m_a, l_a);
-            alpha_b = softmax_row(xb, m_b, l_b);
+            const float alpha_a = softmax_row(xa, m_a, l_a);
+            const float alpha_b = softmax_row(xb, m_b, l_b);
+            uint32_t pa[4], pl[4];  // P (hi) and, for bf16, its residual (lo)
             pa[0] = Mma<T>::pack(xa[0], xa[1]);
             pa[1] = Mma<T>::pack(xb[0], xb[1]);
             pa[2] = Mma<T>::pack(xa[2], xa[3]);
@@ -523,41 +595,40 @@ __global__ void __launch_bounds__(kWarps * 32)
                 pl[2] = Mma<T>::residual(xa[2], xa[3], pa[2]);
                 pl[3] = Mma<T>::residual(xb[2], xb[3], pa[3]);
             }
-        }
-        if (__any_sync(0xffffffffu, alpha_a != 1.0f || alpha_b != 1.0f)) {
+            if (__any_sync(0xffffffffu, alpha_a != 1.0f || alpha_b != 1.0f)) {
 #pragma unroll
-            for (int n = 0; n < C::kNTiles; ++n) {
-                o[n][0] *= alpha_a;
-                o[n][1] *= alpha_a;
-                if constexpr (kMQ) {
+                for (int n = 0; n < C::kNTiles; ++n) {
+                    o[n][0] *= alpha_a;
+                    o[n][1] *= alpha_a;
                     o[n][2] *= alpha_b;
                     o[n][3] *= alpha_b;
                 }
             }
-        }
 
-        // ---- O += P V over the head dimension (pairs of 8-wide tiles)
-        // V rows of tokens at or past the sequence length are zeroed: whatever
-        // the unused slots hold (even NaN) must not reach the result.
-        uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // V rows qd, qd+1 / qd+8, qd+9
-        if (pos0 + kTile > ctx) {
-            keep_lo = (tp[0] < ctx ? 0x0000ffffu : 0u) | (tp[1] < ctx ? 0xffff0000u : 0u);
-            keep_hi = (tp[2] < ctx ? 0x0000ffffu : 0u) | (tp[3] < ctx ? 0xffff0000u : 0u);
-        }
+            // ---- O += P V over the head dimension (pairs of 8-wide tiles)
+            // V rows of tokens at or past the sequence length are zeroed: whatever
+            // the unused slots hold (even NaN) must not reach the result.
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // V rows qd, qd+1 / qd+8, qd+9
+            if (pos0 + kTile > ctx) {
+                keep_lo = (tp[0] < ctx ? 0x0000ffffu : 0u) | (tp[1] < ctx ? 0xffff0000u : 0u);
+                keep_hi = (tp[2] < ctx ? 0x0000ffffu : 0u) | (tp[3] < ctx ? 0xffff0000u : 0u);
+            }
 #pragma unroll
-        for (int j = 0; j < C::kNTiles / 2; ++j) {
-            uint32_t b[4];
-            const uint32_t addr = vbase + (j / 4) * kTcBoxBytes + v_row_off + (((uint32_t)(2 * (j % 4)) << 4) ^ v_x);
-            ldsm_x4_trans(b, addr);
-            b[0] &= keep_lo;
-            b[1] &= keep_hi;
-            b[2] &= keep_lo;
-            b[3] &= keep_hi;
-            Mma<T>::run(o[2 * j], pa, b[0], b[1]);
-            Mma<T>::run(o[2 * j + 1], pa, b[2], b[3]);
-            if constexpr (Mma<T>::kSplitP) {
-                Mma<T>::run(o[2 * j], pl, b[0], b[1]);
-                Mma<T>::run(o[2 * j + 1], pl, b[2], b[3]);
+            for (int j = 0; j < C::kNTiles / 2; ++j) {
+                uint32_t b[4];
+                const uint32_t addr =
+                    vbase + (j / 4) * kTcBoxBytes + v_row_off + (((uint32_t)(2 * (j % 4)) << 4) ^ v_x);
+                ldsm_x4_trans(b, addr);
+                b[0] &= keep_lo;
+                b[1] &= keep_hi;
+                b[2] &= keep_lo;
+                b[3] &= keep_hi;
+                Mma<T>::run(o[2 * j], pa, b[0], b[1]);
+                Mma<T>::run(o[2 * j + 1], pa, b[2], b[3]);
+                if constexpr (Mma<T>::kSplitP) {
+                    Mma<T>::run(o[2 * j], pl, b[0], b[1]);
+                    Mma<T>::run(o[2 * j + 1], pl, b[2], b[3]);
+                }
             }
         }
         __syncwarp();
@@ -577,29 +648,54 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
     }
 
-    // ---- merge the warps: lane (ra, qd) holds O[ra][8n + qd .. +1] (and row rb)
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-    if constexpr (kMQ) {
-        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    }
-    __syncthreads();
+    // ---- merge the warps through shared-memory records
     // records [kWarps][kRows][kRec]: m, l, two unused words (acc starts 16-byte aligned), acc[D]
     constexpr int kRec = D + 4;
     float* mg = reinterpret_cast<float*>(smem);
     static_assert(kWarps * kRows * kRec * 4 <= C::kTilesBytes, "merge area must fit in the tile area");
-    if (live_a) {
-        float* rec = mg + (warp * kRows + ra) * kRec;
-        if ((lane & 3) == 0) {
-            rec[0] = m_a;
-            rec[1] = l_a;
-        }
+    if constexpr (!kMQ) {
+        // lane (ra, qd) holds O^T[16 j + ra (+ 8)][qd, qd + 1]; its sums cover
+        // tokens ra and ra + 8 of every block, so they add up over the 8 lanes
+        // that share qd
 #pragma unroll
-        for (int n = 0; n < C::kNTiles; ++n)
-            *reinterpret_cast<float2*>(rec + 4 + 8 * n + qd) = make_float2(o[n][0], o[n][1]);
-    }
-    if constexpr (kMQ) {
+        for (int sh = 4; sh < 32; sh <<= 1) {
+            l_a += __shfl_xor_sync(0xffffffffu, l_a, sh);
+            l_b += __shfl_xor_sync(0xffffffffu, l_b, sh);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int row = qd + e;
+            if (row < rows) {
+                float* rec = mg + (warp * kRows + row) * kRec;
+                if (ra == 0) {
+                    rec[0] = e ? m_b : m_a;
+                    rec[1] = e ? l_b : l_a;
+                }
+#pragma unroll
+                for (int j = 0; j < C::kNTiles / 2; ++j) {
+                    rec[4 + 16 * j + ra] = ot[j][e];
+                    rec[4 + 16 * j + ra + 8] = ot[j][2 + e];
+                }
+            }
+        }
+    } else {
+        // lane (ra, qd) holds O[ra][8 n + qd .. +1] and O[rb][...]
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+        __syncthreads();
+        if (live_a) {
+            float* rec = mg + (warp * kRows + ra) * kRec;
+            if ((lane & 3) == 0) {
+                rec[0] = m_a;
+                rec[1] = l_a;
+            }
+#pragma unroll
+            for (int n = 0; n < C::kNTiles; ++n)
+                *reinterpret_cast<float2*>(rec + 4 + 8 * n + qd) = make_float2(o[n][0], o[n][1]);
+        }
         if (live_b) {
             float* rec = mg + (warp * kRows + rb) * kRec;
             if ((lane & 3) == 0) {

@@ -115,6 +115,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st = Step()
     st.w = w
     st.host_alloc_us = None
+    st.host_step_us = None
     st.prefix = None
     st.admit_us_per_request = None
     if number == 5:
@@ -154,6 +155,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         st.host_alloc_us = (time.perf_counter() - t0) * 1e6
         assert torch.equal(lens, w.context_lens)
         st.alloc = alloc
+        st.host_step_us = host_step_cost(alloc, S, w.max_blocks_per_seq + 2)
     st.tables_host, st.lens_host, st.slots_host, st.pairs = tables, lens, slots, pairs
     st.block_tables = tables.to(device)
     st.context_lens = lens.to(device)
@@ -192,6 +194,26 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.launches_separate = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
     st.launches_fused = st.launches_separate - 1
     return st
+
+
+def host_step_cost(alloc, S: int, mb: int, steps: int = 20) -> float:
+    """Median host time of one more decode step's allocation, as a serving
+    loop pays it: slots (and copy-on-write pairs) for one token per sequence,
+    then the block tables refilled in place (live entries only) into reused
+    buffers.  Runs after the timed step's inputs were taken, so it changes
+    nothing the GPU sees."""
+    import paged_kv_cache_398_b200 as pkv
+    ids = torch.arange(S, dtype=torch.int64)
+    slots, pairs = torch.empty(S, dtype=torch.int64), torch.empty(S, 2, dtype=torch.int64)
+    tables, lens = torch.full((S, mb), -1, dtype=torch.int32), torch.empty(S, dtype=torch.int32)
+    alloc.batch_tables(ids, mb, tables_out=tables, lens_out=lens)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        alloc.append_one_batch(ids, slots_out=slots, pairs_out=pairs)
+        alloc.batch_tables(ids, mb, pad=pkv.TABLE_KEEP_TAIL, tables_out=tables, lens_out=lens)
+        times.append(time.perf_counter() - t0)
+    return statistics.median(times) * 1e6
 
 
 def run_step(st, ev=None):
@@ -657,6 +679,7 @@ def run_ours(args):
         "gpu_launches": (st.launches_fused if st.path == "fused" else st.launches_separate) * args.steps,
         "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
+        "host_alloc_us_per_step_steady": st.host_step_us,
         "prefix_cache": (None if st.prefix is None else
                          {"admit_us_per_request": st.admit_us_per_request, "hit_tokens": st.prefix["hit_tokens"],
                           "blocks_shared": st.prefix["hit_tokens"] // st.w.block_size,

@@ -438,8 +438,12 @@ int pkv_seq_num_tokens(const pkv_allocator* a, int64_t seq, int32_t* out);
 
 /* Block tables and context lengths of n_seqs sequences, ready for
  * paged_attention_decode.  tables_out: HOST int32
- * [n_seqs][max_blocks_per_seq]; entries past a table's end are set to pad.
+ * [n_seqs][max_blocks_per_seq]; entries past a table's end are set to pad,
+ * or left as they are when pad is PKV_TABLE_KEEP_TAIL (decode never reads
+ * them).  A serving loop that refills the same buffer every step passes
+ * PKV_TABLE_KEEP_TAIL and writes only the live entries.
  * context_lens_out: HOST int32 [n_seqs], may be NULL. */
+#define PKV_TABLE_KEEP_TAIL (-2147483647 - 1)
 int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
                      int32_t* tables_out, int32_t max_blocks_per_seq, int32_t pad,
                      int32_t* context_lens_out);

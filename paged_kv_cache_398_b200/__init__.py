@@ -16,7 +16,7 @@ The native library ``libpaged_kv.so`` is built in-tree by
 """
 
 from ._lib import LibraryMissing, PagedKVError
-from .allocator import BlockAllocator, OutOfBlocks
+from .allocator import TABLE_KEEP_TAIL, BlockAllocator, OutOfBlocks
 from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, block_copy, paged_attention_decode,
                       paged_attention_decode_mq, paged_attention_decode_noalloc,
                       paged_attention_mq_workspace_bytes, paged_attention_partition_tokens,
@@ -24,7 +24,8 @@ from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, block
                       swap_blocks_in, swap_blocks_out)
 
 __all__ = [
-    "BLOCK_SIZE", "PARTITION_TOKENS", "PARTITION_TOKENS_LONG", "BlockAllocator", "LibraryMissing", "OutOfBlocks",
+    "BLOCK_SIZE", "PARTITION_TOKENS", "PARTITION_TOKENS_LONG", "TABLE_KEEP_TAIL", "BlockAllocator",
+    "LibraryMissing", "OutOfBlocks",
     "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_decode_mq",
     "paged_attention_decode_noalloc", "paged_attention_mq_workspace_bytes", "paged_attention_partition_tokens",
     "paged_attention_workspace_bytes",

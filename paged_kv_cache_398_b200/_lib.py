@@ -29,9 +29,10 @@ def _constants() -> dict:
     out = {}
     with open(HEADER) as f:
         for line in f:
-            m = re.match(r"#define\s+(PKV_\w+)\s+\(?(-?\d+)\)?", line)
+            # an integer, or (a - b) as in the INT32_MIN spelling (-2147483647 - 1)
+            m = re.match(r"#define\s+(PKV_\w+)\s+\(?(-?\d+)(?:\s*-\s*(\d+))?\)?", line)
             if m:
-                out[m.group(1)] = int(m.group(2))
+                out[m.group(1)] = int(m.group(2)) - int(m.group(3) or 0)
     return out
 
 

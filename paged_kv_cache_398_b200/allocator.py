@@ -13,6 +13,9 @@ import torch
 from ._lib import C, PagedKVError, check, lib
 
 
+TABLE_KEEP_TAIL = C["PKV_TABLE_KEEP_TAIL"]  # batch_tables pad: leave entries past each table's end alone
+
+
 class AllocStats(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("free_blocks", ctypes.c_int32),
                 ("used_blocks", ctypes.c_int32), ("shared_blocks", ctypes.c_int32),
@@ -81,12 +84,23 @@ class BlockAllocator:
             self._h, seq, n, slots.data_ptr(), pair.data_ptr(), ctypes.byref(cow)))
         return slots[:n].tolist(), (tuple(pair.tolist()) if cow.value else None)
 
-    def append_one_batch(self, seqs):
-        """One token for each sequence: (slots int64 tensor, copy pairs int64 [N, 2])."""
-        ids = torch.as_tensor(list(seqs), dtype=torch.int64).contiguous()
+    @staticmethod
+    def _ids(seqs) -> torch.Tensor:
+        if isinstance(seqs, torch.Tensor) and seqs.dtype == torch.int64 and seqs.device.type == "cpu":
+            return seqs.contiguous()
+        return torch.as_tensor(list(seqs), dtype=torch.int64).contiguous()
+
+    def append_one_batch(self, seqs, slots_out=None, pairs_out=None):
+        """One token for each sequence: (slots int64 tensor, copy pairs int64 [N, 2]).
+        seqs: ids (a CPU int64 tensor avoids a conversion); slots_out /
+        pairs_out: optional CPU int64 buffers of at least [n] / [n, 2], reused
+        by a serving loop."""
+        ids = self._ids(seqs)
         n = ids.numel()
-        slots = torch.empty(max(n, 1), dtype=torch.int64)
-        pairs = torch.empty(max(n, 1), 2, dtype=torch.int64)
+        slots = slots_out if slots_out is not None else torch.empty(max(n, 1), dtype=torch.int64)
+        pairs = pairs_out if pairs_out is not None else torch.empty(max(n, 1), 2, dtype=torch.int64)
+        if slots.dtype != torch.int64 or slots.numel() < n or pairs.dtype != torch.int64 or pairs.numel() < 2 * n:
+            raise ValueError("slots_out / pairs_out: CPU int64 buffers of at least [n] and [n, 2]")
         ncow = ctypes.c_int32(0)
         _check("pkv_batch_append_one", self._L.pkv_batch_append_one(
             self._h, ids.data_ptr(), n, slots.data_ptr(), pairs.data_ptr(), ctypes.byref(ncow)))
@@ -116,12 +130,19 @@ class BlockAllocator:
         _check("pkv_seq_num_tokens", self._L.pkv_seq_num_tokens(self._h, seq, ctypes.byref(v)))
         return int(v.value)
 
-    def batch_tables(self, seqs, max_blocks_per_seq: int, pad: int = -1):
-        """(block_tables int32 [S, MB], context_lens int32 [S]) as host tensors."""
-        ids = torch.as_tensor(list(seqs), dtype=torch.int64).contiguous()
+    def batch_tables(self, seqs, max_blocks_per_seq: int, pad: int = -1, tables_out=None, lens_out=None):
+        """(block_tables int32 [S, MB], context_lens int32 [S]) as host tensors.
+        pad=TABLE_KEEP_TAIL leaves entries past each table's end as they are;
+        with tables_out / lens_out (CPU int32, [S, MB] / [S]) a serving loop
+        refills the same buffers every step."""
+        ids = self._ids(seqs)
         S = ids.numel()
-        tables = torch.empty(max(S, 1), max_blocks_per_seq, dtype=torch.int32)
-        lens = torch.empty(max(S, 1), dtype=torch.int32)
+        tables = tables_out if tables_out is not None else torch.empty(max(S, 1), max_blocks_per_seq, dtype=torch.int32)
+        lens = lens_out if lens_out is not None else torch.empty(max(S, 1), dtype=torch.int32)
+        if (tables.dtype != torch.int32 or not tables.is_contiguous() or tables.dim() != 2
+                or tables.shape[0] < S or tables.shape[1] != max_blocks_per_seq
+                or lens.dtype != torch.int32 or lens.numel() < S):
+            raise ValueError("tables_out / lens_out: CPU int32 buffers [>= S, max_blocks_per_seq] and [>= S]")
         _check("pkv_batch_tables", self._L.pkv_batch_tables(
             self._h, ids.data_ptr(), S, tables.data_ptr(), max_blocks_per_seq, pad, lens.data_ptr()))
         return tables[:S], lens[:S]

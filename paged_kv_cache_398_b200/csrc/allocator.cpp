@@ -323,7 +323,8 @@ int pkv_batch_tables(const pkv_allocator* a, const int64_t* seqs, int32_t n_seqs
         int32_t* row = tables_out + (int64_t)i * max_blocks_per_seq;
         int32_t n = (int32_t)s->blocks.size();
         if (n > 0) std::memcpy(row, s->blocks.data(), sizeof(int32_t) * n);
-        for (int32_t j = n; j < max_blocks_per_seq; ++j) row[j] = pad;
+        if (pad != PKV_TABLE_KEEP_TAIL)
+            for (int32_t j = n; j < max_blocks_per_seq; ++j) row[j] = pad;
         if (context_lens_out) context_lens_out[i] = (int32_t)s->ntok;
     }
     return PKV_OK;

@@ -216,6 +216,39 @@ def test_batch_tables_pad():
     assert lens.tolist() == [33, 5]
 
 
+def test_serving_loop_buffers_and_keep_tail():
+    """A serving loop refills the same host buffers every step: with
+    TABLE_KEEP_TAIL only each table's live entries are written, and reused
+    output buffers give the same slots and copy pairs as fresh ones."""
+    a = pkv.BlockAllocator(64, 16, initial_order=list(reversed(range(64))))
+    b = pkv.BlockAllocator(64, 16, initial_order=list(reversed(range(64))))
+    for x in (a, b):
+        for s, n in enumerate((40, 17, 3)):
+            x.add(s)
+            x.append_tokens(s, n)
+        x.fork(0, 3)
+    ids = torch.arange(4, dtype=torch.int64)
+    slots_buf = torch.full((8,), -7, dtype=torch.int64)
+    pairs_buf = torch.full((8, 2), -7, dtype=torch.int64)
+    tables = torch.full((4, 6), 777, dtype=torch.int32)
+    lens = torch.zeros(4, dtype=torch.int32)
+    for step in range(20):
+        s1, p1 = a.append_one_batch(ids, slots_out=slots_buf, pairs_out=pairs_buf)
+        s2, p2 = b.append_one_batch(list(range(4)))
+        assert torch.equal(s1, s2) and torch.equal(p1, p2)
+        t, n = a.batch_tables(ids, 6, pad=pkv.TABLE_KEEP_TAIL, tables_out=tables, lens_out=lens)
+        for s in range(4):
+            bt = a.block_table(s)
+            assert t[s, :len(bt)].tolist() == bt
+            assert n[s] == a.num_tokens(s)
+    # entries past the longest table each row ever had were never written
+    assert tables[2, 4:].tolist() == [777, 777]
+    full, _ = a.batch_tables(ids, 6)
+    assert (full[2, len(a.block_table(2)):] == -1).all()
+    with pytest.raises(ValueError):
+        a.batch_tables(ids, 5, tables_out=tables, lens_out=lens)
+
+
 def test_swap_out_and_in_native():
     """Preemption: a swapped-out sequence gives its blocks back, keeps its
     token count, and resumes in fresh blocks; shared blocks stay with the

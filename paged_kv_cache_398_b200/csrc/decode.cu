@@ -6,19 +6,23 @@
 // no approximations.)
 //
 // Design (B200, sm_100a):
-//  * Work unit = (partition p of PKV_PARTITION_TOKENS tokens, kv head h,
-//    sequence s): one CTA.  The G = Hq / Hkv query heads that share kv head h
-//    are computed together, so each K/V block is read from HBM once per kv
-//    head, not once per query head.
-//  * Each (block, kv head) tile is one contiguous 16 x head_dim run in the
-//    cache layout, so it is fetched with two 1-D bulk copies (K and V; TMA
-//    engine, no tensor map, no multicast) into shared memory, completing on
-//    an mbarrier.  Every warp owns a ring of kStages tile pairs and walks
-//    its share of the partition's blocks (round-robin) with its own
-//    pipeline.  All waits are bounded (about 1 s) and report a timeout
-//    through the status word instead of hanging.
-//  * Q.K: each lane holds 16 bytes of the head dimension of one token for
-//    all G query heads (fp32, pre-scaled by scale * log2 e).  The partial
+//  * Work unit = (partition p, kv head h, sequence s): one CTA.  A partition
+//    is PKV_PARTITION_TOKENS tokens, or PKV_PARTITION_TOKENS_LONG on large
+//    batches of long contexts (part_tokens_for).  The G = Hq / Hkv query
+//    heads that share kv head h are computed together, so each K/V block is
+//    read from HBM once per kv head, not once per query head.
+//  * fp16 / bf16 run the tensor-core kernel of decode_tc.cuh (tiled TMA,
+//    mma.sync).  This file holds the fp32 kernel, the split-K reduce and the
+//    launcher.
+//  * fp32: each (block, kv head) tile is one contiguous block_size x
+//    head_dim run in the cache layout, so it is fetched with 1-D bulk copies
+//    (K and V; TMA engine, no tensor map, no multicast) into shared memory,
+//    completing on an mbarrier.  Every warp owns a ring of kStages tile
+//    pairs and walks its share of the partition's blocks (round-robin) with
+//    its own pipeline.  All waits are bounded (about 1 s) and report a
+//    timeout through the status word instead of hanging.
+//  * fp32 Q.K: each lane holds 16 bytes of the head dimension of one token
+//    for all G query heads (fp32, pre-scaled by scale * log2 e).  The partial
 //    dot products of a whole block are summed across the lanes of a token
 //    by a transposed shuffle reduction: each level halves the values a
 //    lane keeps.
@@ -27,8 +31,9 @@
 //    sequence longer than one partition writes (max, sum, partial output)
 //    to the workspace, and a second kernel merges its partitions in a fixed
 //    order.
-//  * Partitioning depends only on the context length, so the result is
-//    bit-identical under any permutation of the physical placement.
+//  * Partitioning depends only on the context length and the launch shape,
+//    so the result is bit-identical under any permutation of the physical
+//    placement.
 #include <math.h>
 
 #include <cudaTypedefs.h>

@@ -7,20 +7,24 @@
 // its own 2-stage pipeline of (K tile, V tile) pairs.  The differences:
 //
 //  * Tiles arrive by 2-D tiled TMA (cp.async.bulk.tensor, no multicast) from
-//    a tensor map over the cache viewed as [num_blocks * Hkv * 16][head_dim],
-//    in boxes of 16 rows x 64 elements with the 128-byte swizzle.  The swizzle
-//    makes the ldmatrix reads below free of shared-memory bank conflicts.
-//  * Q.K^T and P.V run on the tensor cores as mma.sync m16n8k16 with fp32
-//    accumulation.  The G query heads of the kv head fill rows 0..G-1 of the
-//    16-row operand; the other rows are zero.  Per 16-token block and
-//    head_dim 128: 16 MMAs for the scores (2 token tiles x 8 k-steps) and 16
-//    for P.V (16 head-dim tiles, k = the block's 16 tokens).
+//    a tensor map over the cache viewed as [num_blocks * Hkv * B][head_dim],
+//    in boxes of 16 (or, at block size 8, two of 8) rows x 64 elements with
+//    the 128-byte swizzle.  The swizzle makes the ldmatrix reads below free
+//    of shared-memory bank conflicts.
+//  * The products run on the tensor cores as mma.sync m16n8k16 with fp32
+//    accumulation.  One query per sequence (G <= 8 query heads): S^T = K Q^T
+//    and O^T += V^T P^T, the block's 16 tokens or 16 head-dim entries as the
+//    MMA rows and the query heads as its 8 columns, so no row is padding: per
+//    block at head_dim 128, 8 MMAs for the scores and 8 for the output.
+//    Multi-query (up to 16 query rows): S = Q K^T and O += P V with the rows
+//    as the 16-row A operand, 16 + 16 MMAs per block.
 //  * Q stays in registers as MMA fragments (exact 16-bit inputs, scaled
 //    after the product in fp32).  The probabilities go from the score
-//    accumulators straight into the P.V operand.  For fp16 they are rounded
-//    to fp16 (11 significant bits).  For bf16 they are split into a bf16
-//    pair hi + lo (about 16 bits) and multiplied by two MMAs, because one
-//    bf16 rounding (8 bits) can cost 5e-3 on a short, cancelling sum.
+//    accumulators into the output MMA's operand (for P^T, transposed in
+//    registers by movmatrix).  For fp16 they are rounded to fp16 (11
+//    significant bits).  For bf16 they are split into a bf16 pair hi + lo
+//    (about 16 bits) and multiplied by two MMAs, because one bf16 rounding
+//    (8 bits) can cost 5e-3 on a short, cancelling sum.
 //  * In the sequence's last, partial block, the V operand rows of tokens past
 //    the length are zeroed, and their scores are set to -inf, so whatever
 //    the unused slots hold cannot reach the result.
@@ -370,10 +374,10 @@ __global__ void __launch_bounds__(kWarps * 32)
             qa[ks][3] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
     }
-    // positions a row may see: < lim.  Single query: every row (padding rows
-    // included, whose Q is zero) sees the whole context, so each row keeps a
-    // finite maximum.  Multi-query: a row holding no query sees nothing.
-    const int lim_a = kMQ ? (live_a ? first_new + ra / G + 1 : 0) : ctx;
+    // Multi-query: positions row ra (rb) may see are < lim_a (lim_b); a row
+    // holding no query sees nothing.  (A single query sees the whole context,
+    // so that path masks against ctx alone.)
+    const int lim_a = live_a ? first_new + ra / G + 1 : 0;
     const int lim_b = live_b ? first_new + rb / G + 1 : 0;
 
     // ---- per-lane ldmatrix addressing (128-byte swizzle: chunk c of row r is at c ^ (r % 8))

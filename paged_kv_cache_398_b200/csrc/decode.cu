@@ -727,7 +727,7 @@ int launch(const DecodeArgs& a)
         // per (multi-query, partition size), each setting its shared-memory
         // limit once per device
         using C = TcCfg<D>;
-        const bool mq = a.q_len > 1, wide = a.part_tokens == kLongPartTokens;
+        const bool mq = a.q_len * G > 8, wide = a.part_tokens == kLongPartTokens;  // 16-row form past 8 rows
         const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
         static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
         auto with_kernel = [&](auto&& f) {

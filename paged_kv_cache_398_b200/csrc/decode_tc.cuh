@@ -226,12 +226,14 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
     return alpha;
 }
 
-// One CTA = (partition p, kv head h, sequence s).
-//  kMQ = false: one query per sequence; rows 0..G-1 of the MMA operand are
-//               the G query heads of kv head h (q_len must be 1).
-//  kMQ = true : q_len new tokens per sequence; row r = j * G + g is query
-//               head h*G + g of new token j (q_len * G <= 16).  Token j sits
-//               at position ctx - q_len + j and sees positions up to its own.
+// One CTA = (partition p, kv head h, sequence s).  q_len new tokens per
+// sequence: query row r = j * G + g is query head h*G + g of new token j,
+// which sits at position ctx - q_len + j and sees positions up to its own
+// (q_len = 1: the whole context).
+//  kMQ = false: q_len * G <= 8 rows, the transposed products S^T = K Q^T and
+//               O^T += V^T P^T with the rows as the MMA's 8 columns.
+//  kMQ = true : 9..16 rows, S = Q K^T and O += P V with the rows as the
+//               16-row A operand.
 // k_new / v_new non-null: the new tokens' K/V rows [S][q_len][Hkv][D] are
 // written to their slots (through the block table) by the CTA whose
 // partition holds them, and patched into the staged tiles before use.
@@ -252,14 +254,14 @@ __global__ void __launch_bounds__(kWarps * 32)
     constexpr int part_tokens = PT;
     static_assert(PT == kPartTokens || PT == kLongPartTokens, "partition sizes");
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
-    constexpr int kRows = kMQ ? 16 : G;  // operand rows that can hold queries
+    constexpr int kRows = kMQ ? 16 : 8;  // operand rows that can hold queries
     constexpr int kChunks = D / 8;       // 16-byte chunks per K or V row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
     const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rows = kMQ ? q_len * G : G;  // live query rows
+    const int rows = q_len * G;  // live query rows
 
     // The context length and this thread's entry of the partition's table
     // slice are loaded together: the entry depends only on (s, p), so the
@@ -297,11 +299,11 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int nb = min(part_tokens / kTile, (ctx - part0 + kTile - 1) / kTile);  // its 16-token tiles
     const int first_new = ctx - q_len;   // position of the first new token
     // Fused write: the new tokens that fall in this partition, as token
-    // indices [jlo_p, jhi_p).  With several new tokens, right after the
-    // prologue every thread stages some of their K / V rows in shared memory
-    // by cp.async, so the warp that writes and patches them later never waits
-    // on global memory.  A single new token (kMQ false) is one 16-byte load
-    // per lane, done where it is patched.
+    // indices [jlo_p, jhi_p).  With up to 16 new tokens (kMQ), right after
+    // the prologue every thread stages some of their K / V rows in shared
+    // memory by cp.async, so the warp that writes and patches them later
+    // never waits on global memory.  With at most 8 (kMQ false) the warp
+    // loads them where it patches them, four 16-byte chunks in flight per lane.
     constexpr int kNewRows = kMQ ? 16 : 0;  // capacity of the staging area, in tokens
     const int jlo_p = max(0, part0 - first_new);
     const int jhi_p = min(q_len, part0 + part_tokens - first_new);
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(kWarps * 32)
             }
             __syncwarp();
         } else if (!kMQ && k_new != nullptr && pos0 + kTile > first_new) {
-            // the one new token: loaded here, four 16-byte chunks in flight per lane at most
+            // the new tokens of this block: loaded here, four 16-byte chunks in flight per lane
             const int jlo = max(0, pos0 - first_new);
             const int jhi = min(q_len, pos0 + kTile - first_new);
             const int items = (jhi - jlo) * 2 * kChunks;  // 16-byte chunks: (token, K or V, chunk)
@@ -497,9 +499,16 @@ __global__ void __launch_bounds__(kWarps * 32)
             float x[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) x[i] = (sa[i] + sb[i]) * scale_log2;
-            if (pos0 + kTile > ctx) {  // the sequence's last, partial block
-                if (pos0 + ra >= ctx) x[0] = x[1] = -INFINITY;
-                if (pos0 + ra + 8 >= ctx) x[2] = x[3] = -INFINITY;
+            if (pos0 + kTile > first_new + 1) {
+                // some token of this block lies past a row's last visible
+                // position: ctx - 1 for one query, the row's own token's
+                // position for several; padding rows keep ctx (finite scores)
+                const int lim0 = qd < rows ? first_new + qd / G + 1 : ctx;
+                const int lim1 = qd + 1 < rows ? first_new + (qd + 1) / G + 1 : ctx;
+                if (pos0 + ra >= lim0) x[0] = -INFINITY;
+                if (pos0 + ra >= lim1) x[1] = -INFINITY;
+                if (pos0 + ra + 8 >= lim0) x[2] = -INFINITY;
+                if (pos0 + ra + 8 >= lim1) x[3] = -INFINITY;
             }
             float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
@@ -507,9 +516,11 @@ __global__ void __launch_bounds__(kWarps * 32)
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, sh));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, sh));
             }
-            // every block has a visible token, so both maxima are finite
+            // A row moves its reference on its first visible token.  With
+            // several new tokens a row can see nothing in this partition yet
+            // (m = -inf): its scores are then all -inf and its weights 0.
             float alpha_a = 1.0f, alpha_b = 1.0f;
-            if (mx0 > m_a + kLazyLog2) {  // always on the first block (m = -inf)
+            if (mx0 > m_a + kLazyLog2) {
                 alpha_a = pkv::fast_exp2(m_a - mx0);
                 m_a = mx0;
             }
@@ -517,10 +528,11 @@ __global__ void __launch_bounds__(kWarps * 32)
                 alpha_b = pkv::fast_exp2(m_b - mx1);
                 m_b = mx1;
             }
-            x[0] = pkv::fast_exp2(x[0] - m_a);
-            x[2] = pkv::fast_exp2(x[2] - m_a);
-            x[1] = pkv::fast_exp2(x[1] - m_b);
-            x[3] = pkv::fast_exp2(x[3] - m_b);
+            const float mu_a = m_a == -INFINITY ? 0.0f : m_a, mu_b = m_b == -INFINITY ? 0.0f : m_b;
+            x[0] = pkv::fast_exp2(x[0] - mu_a);
+            x[2] = pkv::fast_exp2(x[2] - mu_a);
+            x[1] = pkv::fast_exp2(x[1] - mu_b);
+            x[3] = pkv::fast_exp2(x[3] - mu_b);
             l_a = l_a * alpha_a + (x[0] + x[2]);
             l_b = l_b * alpha_b + (x[1] + x[3]);
             // P^T as the B operand of O^T += V^T P^T: transpose each 8-token half

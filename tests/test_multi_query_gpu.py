@@ -82,8 +82,10 @@ MQ_LENS = [4, 15, 16, 17, 18, 33, 511, 512, 513, 514, 1024, 1026, 4099]
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("G,q_len", [(1, 1), (1, 3), (1, 16), (2, 2), (4, 1), (4, 4), (8, 2)])
+@pytest.mark.parametrize("G,q_len", [(1, 1), (1, 3), (1, 8), (1, 16), (2, 2), (2, 4), (4, 1), (4, 2), (4, 4),
+                                     (8, 2)])
 def test_multi_query_and_fused_write_match_oracle(dtype, D, G, q_len):
+    # up to 8 rows (q_len * G): the transposed kernel; 9..16 rows: the 16-row kernel
     Hkv = 2
     lens = [max(n, q_len) for n in MQ_LENS]      # every sequence holds its new tokens
     w = make_custom(lens, Hkv * G, Hkv, D, dtype, seed=31 * G + q_len + D, q_len=q_len)
@@ -150,7 +152,7 @@ def test_unsupported_combinations_are_rejected():
 
 @pytest.mark.parametrize("block_size", [8, 32])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("G,q_len", [(1, 1), (4, 3), (2, 8), (1, 16)])
+@pytest.mark.parametrize("G,q_len", [(1, 1), (4, 2), (4, 3), (2, 8), (1, 16)])
 def test_multi_query_fused_block_sizes_8_and_32(block_size, dtype, G, q_len):
     lens = [max(n, q_len) for n in (5, 8, 9, 17, 33, 510, 514, 1031)]
     w = make_custom(lens, 2 * G, 2, 128, dtype, seed=7 * block_size + G + q_len, q_len=q_len,

@@ -51,6 +51,7 @@ extern "C" int block_copy(void* k_cache, void* v_cache, const int64_t* pairs, in
                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                           int32_t num_blocks, int32_t dtype, void* stream)
 {
+    const pkv::NvtxRange nvtx("block_copy");
     const size_t eb = pkv::dtype_bytes(dtype);
     if (eb == 0) return PKV_ERR_UNSUPPORTED;
     if (num_pairs < 0 || num_kv_heads < 1 || head_dim < 1 || block_size < 1 || num_blocks < 0)

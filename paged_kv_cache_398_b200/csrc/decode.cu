@@ -935,6 +935,7 @@ extern "C" int paged_attention_decode(void* out, const void* q, const void* k_ca
                                       int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
                                       int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
+    const pkv::NvtxRange nvtx("paged_attention_decode");
     // read-only caches: the const is cast away only for the shared launcher
     return decode_entry(out, q, nullptr, nullptr, const_cast<void*>(k_cache), const_cast<void*>(v_cache),
                         block_tables, max_blocks_per_seq, context_lens, num_seqs, 1, max_context_len,
@@ -950,6 +951,7 @@ extern "C" int paged_attention_decode_mq(void* out, const void* q, const void* k
                                          int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
                                          void* workspace, size_t workspace_bytes, void* stream)
 {
+    const pkv::NvtxRange nvtx("paged_attention_decode_mq");
     return decode_entry(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                         num_seqs, q_len, max_context_len, num_q_heads, num_kv_heads, head_dim, block_size,
                         num_blocks, scale, dtype, workspace, workspace_bytes, stream);
@@ -1002,6 +1004,7 @@ extern "C" int paged_attention_decode_noalloc(void* out, const void* q, const vo
                                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                               int32_t num_blocks, float scale, int32_t dtype, void* stream)
 {
+    const pkv::NvtxRange nvtx("paged_attention_decode_noalloc");
     const size_t need = paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len);
     if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;

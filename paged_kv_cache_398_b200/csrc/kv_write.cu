@@ -49,6 +49,7 @@ extern "C" int paged_kv_write(const void* k_new, const void* v_new, void* k_cach
                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
                               int32_t dtype, void* stream)
 {
+    const pkv::NvtxRange nvtx("paged_kv_write");
     const size_t eb = pkv::dtype_bytes(dtype);
     if (eb == 0) return PKV_ERR_UNSUPPORTED;
     if (num_tokens < 0 || num_kv_heads < 1 || head_dim < 1 || block_size < 1 || num_blocks < 0)

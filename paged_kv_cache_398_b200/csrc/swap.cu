@@ -109,6 +109,7 @@ extern "C" int swap_blocks_out(const void* k_cache, const void* v_cache, const i
                                void* host_k, void* host_v, int32_t num_kv_heads, int32_t head_dim,
                                int32_t block_size, int32_t num_blocks, int32_t dtype, void* stream)
 {
+    const pkv::NvtxRange nvtx("swap_blocks_out");
     return swap_blocks(const_cast<void*>(k_cache), const_cast<void*>(v_cache), block_ids, n, host_k, host_v,
                        num_kv_heads, head_dim, block_size, num_blocks, dtype, stream, true);
 }
@@ -117,6 +118,7 @@ extern "C" int swap_blocks_in(void* k_cache, void* v_cache, const int64_t* block
                               const void* host_v, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                               int32_t num_blocks, int32_t dtype, void* stream)
 {
+    const pkv::NvtxRange nvtx("swap_blocks_in");
     return swap_blocks(k_cache, v_cache, block_ids, n, const_cast<void*>(host_k), const_cast<void*>(host_v),
                        num_kv_heads, head_dim, block_size, num_blocks, dtype, stream, false);
 }

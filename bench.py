@@ -171,11 +171,7 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         st.k_new = _randn((S, q_len, w.num_kv_heads, w.head_dim), w.dtype, gd, device)
         st.v_new = _randn((S, q_len, w.num_kv_heads, w.head_dim), w.dtype, gd, device)
     st.out = torch.empty_like(st.q)
-    # [S, q_len, ...] views for paged_attention_decode_mq; flat [S * q_len, ...] rows for paged_kv_write
-    lead = (S, q_len)
-    st.q4, st.out4 = st.q.reshape(lead + st.q.shape[-2:]), st.out.reshape(lead + st.out.shape[-2:])
-    st.k_new4, st.v_new4 = (t.reshape(lead + t.shape[-2:]) for t in (st.k_new, st.v_new))
-    st.k_rows, st.v_rows = (t.reshape(S * q_len, *t.shape[-2:]) for t in (st.k_new, st.v_new))
+    pack_step_inputs(st, device)
     st.path = "separate"
     st.max_ctx = int(lens.max())
     ws_bytes = pkv.paged_attention_mq_workspace_bytes(S, q_len, w.num_q_heads, w.head_dim, st.max_ctx)
@@ -194,6 +190,34 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.launches_separate = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
     st.launches_fused = st.launches_separate - 1
     return st
+
+
+STEP_INPUTS = ("q", "k_new", "v_new", "slots", "block_tables", "context_lens")
+
+
+def pack_step_inputs(st, device):
+    """Place a step's inputs (q, new K/V, slots, tables, lengths) in one
+    device buffer, each at a 256-byte aligned offset, with a pinned host
+    mirror, so the end-to-end loop moves them with one host-to-device copy
+    instead of six.  The tensors are rebound to views of the buffer."""
+    offs, total = [], 0
+    for name in STEP_INPUTS:
+        t = getattr(st, name)
+        offs.append(total)
+        total += -(-t.numel() * t.element_size() // 256) * 256
+    st.in_dev = torch.empty(max(total, 256), dtype=torch.uint8, device=device)
+    for name, off in zip(STEP_INPUTS, offs):
+        t = getattr(st, name).contiguous()
+        view = st.in_dev[off:off + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        view.copy_(t)
+        setattr(st, name, view)
+    st.in_host = st.in_dev.cpu().pin_memory() if st.in_dev.is_cuda else st.in_dev.clone()
+    S, q_len = st.q.shape[0], st.q_len
+    # [S, q_len, ...] views for paged_attention_decode_mq; flat [S * q_len, ...] rows for paged_kv_write
+    lead = (S, q_len)
+    st.q4, st.out4 = st.q.reshape(lead + st.q.shape[-2:]), st.out.reshape(lead + st.out.shape[-2:])
+    st.k_new4, st.v_new4 = (t.reshape(lead + t.shape[-2:]) for t in (st.k_new, st.v_new))
+    st.k_rows, st.v_rows = (t.reshape(S * q_len, *t.shape[-2:]) for t in (st.k_new, st.v_new))
 
 
 def host_step_cost(alloc, S: int, mb: int, steps: int = 20) -> float:
@@ -596,18 +620,14 @@ def run_ours(args):
     write_ms = [ev[1].elapsed_time(ev[2]) for ev in evs.values()] if st.path == "separate" else None
 
     # ---- end to end: host inputs in, host output out, every step ------------
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    h_in = {"q": pin(st.q), "k_new": pin(st.k_new), "v_new": pin(st.v_new), "slots": pin(st.slots),
-            "tables": pin(st.block_tables), "lens": pin(st.context_lens)}
-    d_in = {"q": st.q, "k_new": st.k_new, "v_new": st.v_new, "slots": st.slots, "tables": st.block_tables,
-            "lens": st.context_lens}
+    # the step's inputs (q, new K/V, slots, tables, lengths) sit packed in one
+    # pinned host buffer and go over in one copy; the output comes back in one
     h_out = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    h2d = st.in_host.numel()
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        for k2, t in h_in.items():
-            d_in[k2].copy_(t, non_blocking=True)
+        st.in_dev.copy_(st.in_host, non_blocking=True)
         run_step(st)
         h_out.copy_(st.out, non_blocking=True)
 

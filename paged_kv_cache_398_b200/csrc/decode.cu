@@ -38,6 +38,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 
@@ -609,7 +610,7 @@ int encode_cache_map(CUtensorMap* map, const void* cache, int64_t rows, int D, i
 // Once per device and kernel instantiation: allow more than 48 KiB of
 // dynamic shared memory.
 template <typename K>
-int allow_smem(K kernel, int bytes, bool* configured)
+int allow_smem(K kernel, int bytes, std::atomic<bool>* configured)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -617,13 +618,13 @@ int allow_smem(K kernel, int bytes, bool* configured)
         pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
         return PKV_ERR_CUDA;
     }
-    if (!configured[dev]) {
+    if (!configured[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess) {
             pkv::record_cuda_error(e);
             return PKV_ERR_CUDA;
         }
-        configured[dev] = true;
+        configured[dev].store(true, std::memory_order_release);  // setting it twice is harmless
     }
     return PKV_OK;
 }
@@ -655,7 +656,7 @@ struct DecodeArgs {
 
 // Resident CTAs per SM of `kernel` with `smem` bytes of dynamic shared memory.
 template <typename K>
-int occupancy_of(K kernel, int smem, bool* configured, int* out)
+int occupancy_of(K kernel, int smem, std::atomic<bool>* configured, int* out)
 {
     int rc = allow_smem(kernel, smem, configured);
     if (rc != PKV_OK) return rc;
@@ -670,23 +671,23 @@ int occupancy_of(K kernel, int smem, bool* configured, int* out)
 // Multiprocessor count of the current device, read once per device.
 int sm_count(int* out)
 {
-    static int cached[64] = {};
+    static std::atomic<int> cached[64] = {};  // 0: not read yet
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) {
         pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidDevice : e);
         return PKV_ERR_CUDA;
     }
-    if (cached[dev] == 0) {
+    if (cached[dev].load(std::memory_order_relaxed) == 0) {
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess || n < 1) {
             pkv::record_cuda_error(e == cudaSuccess ? cudaErrorInvalidValue : e);
             return PKV_ERR_CUDA;
         }
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    *out = cached[dev];
+    *out = cached[dev].load(std::memory_order_relaxed);
     return PKV_OK;
 }
 
@@ -729,7 +730,7 @@ int launch(const DecodeArgs& a)
         using C = TcCfg<D>;
         const bool mq = a.q_len * G > 8, wide = a.part_tokens == kLongPartTokens;  // 16-row form past 8 rows
         const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
-        static bool cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
+        static std::atomic<bool> cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
         auto with_kernel = [&](auto&& f) {
             if (!mq && !wide) return f(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
             if (!mq) return f(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);
@@ -738,7 +739,7 @@ int launch(const DecodeArgs& a)
         };
         if (a.occupancy_out) {
             return with_kernel(
-                [&](auto kernel, bool* configured) { return occupancy_of(kernel, smem, configured, a.occupancy_out); });
+                [&](auto kernel, std::atomic<bool>* configured) { return occupancy_of(kernel, smem, configured, a.occupancy_out); });
         }
         const int64_t rows = (int64_t)a.NB * a.Hkv * B;
         if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
@@ -755,7 +756,7 @@ int launch(const DecodeArgs& a)
                                       static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.q_len, a.Hq, a.Hkv,
                                       a.NB, scale_log2, max_parts, a.status);
         };
-        rc = with_kernel([&](auto kernel, bool* configured) {
+        rc = with_kernel([&](auto kernel, std::atomic<bool>* configured) {
             const int r = allow_smem(kernel, smem, configured);
             if (r == PKV_OK) launch_err = args(kernel);
             return r;
@@ -765,7 +766,7 @@ int launch(const DecodeArgs& a)
         // fp32: CUDA-core kernel fed by 1-D bulk copies (one query, no fused write)
         if (a.q_len != 1 || a.k_new || a.part_tokens != kPartTokens) return PKV_ERR_UNSUPPORTED;
         using C = Cfg<T, D, G>;
-        static bool configured[64] = {};
+        static std::atomic<bool> configured[64] = {};
         if (a.occupancy_out)
             return occupancy_of(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured, a.occupancy_out);
         rc = allow_smem(decode_partition_kernel<T, D, G, B>, C::kSmemBytes, configured);

@@ -499,3 +499,45 @@ def test_every_decode_kernel_keeps_its_occupancy():
         assert L.pkv_debug_decode_occupancy(C["PKV_F32"], D, 4, 1, 16, 0, ctypes.byref(n)) == 0 and n.value >= 1
     n = ctypes.c_int32(0)
     assert L.pkv_debug_decode_occupancy(C["PKV_F32"], 128, 4, 2, 16, 0, ctypes.byref(n)) == C["PKV_ERR_UNSUPPORTED"]
+
+
+def test_concurrent_host_threads_on_their_own_streams():
+    """Two host threads decode different batches at once, each on its own
+    stream with its own workspace (ctypes releases the GIL, so the calls
+    overlap on the host, first-call set-up included); each result equals
+    the same call made alone, bit for bit."""
+    import threading
+    batches = [make_custom([700, 33, 2100, 5], 16, 4, 128, torch.bfloat16, seed=60).to("cuda"),
+               make_custom([1500, 900, 64], 8, 8, 64, torch.float16, seed=61).to("cuda")]
+
+    def decode(w, stream):
+        out = torch.empty_like(w.q)
+        with torch.cuda.stream(stream):
+            ws = torch.zeros(max(1, pkv.paged_attention_workspace_bytes(w.num_seqs, w.num_q_heads, w.head_dim,
+                                                                         w.max_context_len)),
+                             dtype=torch.uint8, device="cuda")
+            for _ in range(5):
+                pkv.paged_attention_decode(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens,
+                                           w.scale, w.max_context_len, workspace=ws)
+        stream.synchronize()
+        return out
+
+    alone = [decode(w, torch.cuda.Stream()) for w in batches]
+    results = [None, None]
+    errors = []
+
+    def worker(i):
+        try:
+            results[i] = decode(batches[i], torch.cuda.Stream())
+        except Exception as e:  # surfaced below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    for got, ref in zip(results, alone):
+        assert torch.equal(got, ref)
+    assert pkv.pkv_device_status(0) == 0

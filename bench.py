@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 DECODE_SOURCES = ("paged_kv_cache_398_b200/csrc/decode.cu", "paged_kv_cache_398_b200/csrc/decode_tc.cuh",
-                  "paged_kv_cache_398_b200/csrc/common.cuh")
+                  "paged_kv_cache_398_b200/csrc/decode_common.cuh", "paged_kv_cache_398_b200/csrc/common.cuh")
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_traffic.json")
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (the measured copy peak is the roofline denominator)
 
@@ -92,11 +92,13 @@ class Step:
 
 
 def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: int = 16, max_ctx=None,
-               q_len: int = 1):
+               q_len: int = 1, path: str = "fused"):
     """The decode step of workload `number`.  q_len > 1: every sequence
     brings q_len new tokens (draft tokens to verify, causal among them) after
     a prompt of ctx - q_len tokens; the recipe's shortest context is raised
-    to leave room for them."""
+    to leave room for them.  path 'shared': the host also plans which
+    sequences share leading blocks (pkv_shared_prefix_plan), and the plan's
+    two arrays travel with the step's inputs."""
     import paged_kv_cache_398_b200 as pkv
     from paged_kv_cache_398_b200.workloads import make_workload
 
@@ -157,6 +159,17 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         st.alloc = alloc
         st.host_step_us = host_step_cost(alloc, S, w.max_blocks_per_seq + 2)
     st.tables_host, st.lens_host, st.slots_host, st.pairs = tables, lens, slots, pairs
+    st.inputs = STEP_INPUTS
+    st.plan, st.host_plan_us = None, None
+    if path == "shared":
+        if q_len != 1:
+            raise SystemExit("--path shared decodes one new token per sequence")
+        t0 = time.perf_counter()
+        st.plan = pkv.pkv_shared_prefix_plan(tables, lens, w.block_size,
+                                             pkv.SHARED_MAX_ROWS // (w.num_q_heads // w.num_kv_heads))
+        st.host_plan_us = (time.perf_counter() - t0) * 1e6
+        st.groups, st.shared_lens = st.plan.groups, st.plan.shared_lens
+        st.inputs = STEP_INPUTS + ("groups", "shared_lens")
     st.block_tables = tables.to(device)
     st.context_lens = lens.to(device)
     st.slots = slots.to(device)
@@ -174,7 +187,9 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     pack_step_inputs(st, device)
     st.path = "separate"
     st.max_ctx = int(lens.max())
-    ws_bytes = pkv.paged_attention_mq_workspace_bytes(S, q_len, w.num_q_heads, w.head_dim, st.max_ctx)
+    ws_bytes = (pkv.paged_attention_shared_workspace_bytes(S, w.num_q_heads, w.head_dim, st.max_ctx)
+                if path == "shared" else
+                pkv.paged_attention_mq_workspace_bytes(S, q_len, w.num_q_heads, w.head_dim, st.max_ctx))
     st.workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
     e = w.q.element_size()
     ctx = lens.to(torch.int64)
@@ -189,6 +204,17 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.max_parts = (st.max_ctx + st.part_tokens - 1) // st.part_tokens
     st.launches_separate = (1 if pairs.shape[0] else 0) + 1 + 1 + (1 if st.max_parts > 1 else 0)
     st.launches_fused = st.launches_separate - 1
+    st.shared_bytes = None
+    if st.plan is not None:
+        # block copies, group pass (if any group), own pass, reduce
+        st.launches_shared = (1 if pairs.shape[0] else 0) + (1 if st.plan.groups.shape[0] else 0) + 2
+        # K/V the two passes must read under the plan: each group's shared
+        # positions once, every sequence's own positions once
+        x = st.plan.shared_lens.to(torch.int64)
+        first = st.plan.groups[:, 0].to(torch.int64)
+        tokens = int(x[first].sum()) + int((ctx - x).sum())
+        st.shared_bytes = (tokens * w.num_kv_heads * w.head_dim * 2 * e + 2 * S * w.num_q_heads * w.head_dim * e
+                           + 4 * int(nblk.sum()) + 4 * S + 4 * S + 8 * first.numel() + st.write_bytes)
     return st
 
 
@@ -201,12 +227,12 @@ def pack_step_inputs(st, device):
     mirror, so the end-to-end loop moves them with one host-to-device copy
     instead of six.  The tensors are rebound to views of the buffer."""
     offs, total = [], 0
-    for name in STEP_INPUTS:
+    for name in st.inputs:
         t = getattr(st, name)
         offs.append(total)
         total += -(-t.numel() * t.element_size() // 256) * 256
     st.in_dev = torch.empty(max(total, 256), dtype=torch.uint8, device=device)
-    for name, off in zip(STEP_INPUTS, offs):
+    for name, off in zip(st.inputs, offs):
         t = getattr(st, name).contiguous()
         view = st.in_dev[off:off + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
         view.copy_(t)
@@ -263,6 +289,11 @@ def run_step(st, ev=None):
     elif st.path == "separate":
         pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                       st.w.scale, st.max_ctx, workspace=st.workspace)
+    elif st.path == "shared":
+        pl = st.plan
+        pkv.paged_attention_decode_shared(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                                          st.w.scale, st.max_ctx, st.groups, st.shared_lens, pl.max_shared_len,
+                                          pl.max_own_len, k_new=st.k_new, v_new=st.v_new, workspace=st.workspace)
     else:
         pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                       st.w.scale, st.max_ctx, k_new=st.k_new4, v_new=st.v_new4,
@@ -348,9 +379,18 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the oracle on the host cores
 # ----------------------------------------------------------------------------
-def sub_workload(w, tables, lens, pairs, seqs):
+def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False):
     """The listed sequences' blocks (plus copy sources) copied to the host and
-    relabelled 0..n-1, with their tables, as an oracle input."""
+    relabelled 0..n-1, with their tables, as an oracle input.
+
+    repeated: the input of the step as the timed loop runs it, after it has
+    already run once.  A step is not idempotent when a sequence's new token
+    lands in a copy-on-write source block (a sample whose own output still
+    fits in the prompt's partial block): the next repetition copies that
+    token into its siblings' blocks.  meta["pre_writes"] then holds the new
+    token of every sequence of the batch, sampled or not, whose slot lies in
+    these blocks, for oracle_step_timed to apply once (copies + those writes)
+    before the step it times."""
     from paged_kv_cache_398_b200.workloads import DecodeWorkload
     B = w.block_size
     need = []
@@ -367,13 +407,24 @@ def sub_workload(w, tables, lens, pairs, seqs):
         n = -(-int(lens[s]) // B)
         sbt[r, :n] = torch.tensor([remap[b] for b in tables[s, :n].tolist()], dtype=torch.int32)
     sel = torch.tensor(seqs, dtype=torch.int64, device=w.q.device)
+    meta = {}
+    if repeated:
+        writers, slots = [], []
+        for s in range(lens.shape[0]):
+            pos = int(lens[s]) - 1
+            b = int(tables[s, pos // B])
+            if b in remap:
+                writers.append(s)
+                slots.append(remap[b] * B + pos % B)
+        wsel = torch.tensor(writers, dtype=torch.int64, device=w.q.device)
+        meta["pre_writes"] = (torch.tensor(slots, dtype=torch.int64), w.k_new[wsel].cpu(), w.v_new[wsel].cpu())
     return DecodeWorkload(
         name=w.name + "-sample", dtype=w.dtype, num_seqs=len(seqs), num_q_heads=w.num_q_heads,
         num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=B, num_blocks=len(ids),
         context_lens=lens[seqs].contiguous(), block_tables=sbt,
         copy_pairs=torch.tensor([(remap[a], remap[b]) for a, b in sub_pairs], dtype=torch.int64).reshape(-1, 2),
         q=w.q[sel].cpu(), k_cache=w.k_cache[idx].cpu(), v_cache=w.v_cache[idx].cpu(),
-        k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(), scale=w.scale, seed=w.seed)
+        k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(), scale=w.scale, seed=w.seed, meta=meta)
 
 
 def oracle_step_timed(sub, threads: int, keep=None):
@@ -388,6 +439,11 @@ def oracle_step_timed(sub, threads: int, keep=None):
     slots = torch.tensor([slot_for_position(sub.block_tables[s].tolist(), int(sub.context_lens[s]) - 1, B)
                           for s in range(sub.num_seqs)], dtype=torch.int64)
     k, v = sub.k_cache.clone(), sub.v_cache.clone()
+    if "pre_writes" in sub.meta:                 # the step's earlier repetition (untimed)
+        pre_slots, pre_k, pre_v = sub.meta["pre_writes"]
+        if sub.copy_pairs.numel():
+            oracle.block_copy(k, v, sub.copy_pairs)
+        oracle.kv_write(k, v, pre_k, pre_v, pre_slots)
     t0 = time.perf_counter()
     if sub.copy_pairs.numel():
         oracle.block_copy(k, v, sub.copy_pairs)
@@ -429,7 +485,7 @@ def cpu_baseline(st, threads: int):
     t1 = oracle_step_timed(probe, 1)
     per_tok = t1 / max(1, int(lens[0]))
     seqs = pick_sample(lens, 30.0, per_tok)
-    sub = sub_workload(st.w, tables, lens, pairs, seqs)
+    sub = sub_workload(st.w, tables, lens, pairs, seqs, repeated=True)
     refs = []
     t = oracle_step_timed(sub, threads, keep=refs)
     return {"value": sample_kv_bytes(sub) / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -440,8 +496,9 @@ def cpu_baseline(st, threads: int):
 
 def parity_on_sample(st, base, atol: float = 2e-3, rtol: float = 1e-2):
     """The timed steps' output of the sampled sequences against the oracle's
-    fp64 output of the same step (repeating a step leaves the cache as one
-    step leaves it, so the last step's output is the one to compare)."""
+    fp64 output of the same step as the loop repeats it (from its second
+    repetition on, every repetition leaves the cache as the one before, so
+    the last step's output is the one to compare)."""
     import numpy as np
     got = st.out[torch.tensor(base["seqs"], device=st.out.device)].double().cpu().numpy()
     ref = np.stack(base["refs"])
@@ -587,7 +644,7 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size, args.max_ctx, args.q_len)
+    st = build_step(args.workload, dev, rank, args.num_seqs, args.block_size, args.max_ctx, args.q_len, args.path)
     st.path = args.path
     torch.cuda.synchronize(dev)
     threads = cpu_threads()
@@ -658,8 +715,10 @@ def run_ours(args):
     S = st.w.num_seqs
     value = kv_total * args.steps / (ms_max / 1e3) / 1e9
     dec_mean = statistics.mean(dec_ms)
-    # the fused call also moves the new tokens' K/V (read and written once)
-    call_bytes = st.decode_bytes + (st.write_bytes if st.path == "fused" else 0)
+    # the fused call also moves the new tokens' K/V (read and written once);
+    # the shared-prefix call reads each group's shared blocks once
+    call_bytes = (st.shared_bytes if st.path == "shared" else
+                  st.decode_bytes + (st.write_bytes if st.path == "fused" else 0))
     achieved = call_bytes / (dec_mean / 1e3) / 1e9
     clk = clocks.summary(t_wall0, t_wall1)
     line = {
@@ -684,9 +743,11 @@ def run_ours(args):
                       "block_copy_mean": statistics.mean(copy_ms) if copy_ms else None,
                       "sampled_steps": len(dec_ms),
                       "how": "CUDA events around each call on its stream, in evenly spread timed steps"},
-        "roofline": {"kernel": ("paged_attention_decode_mq with fused slot write (partition kernel + split-K reduce)"
-                                if st.path == "fused" else
-                                "paged_attention_decode (partition kernel + split-K reduce)"),
+        "roofline": {"kernel": {"fused": "paged_attention_decode_mq with fused slot write "
+                                         "(partition kernel + split-K reduce)",
+                                "shared": "paged_attention_decode_shared with fused slot write "
+                                          "(group pass + own pass + split-K reduce)",
+                                "separate": "paged_attention_decode (partition kernel + split-K reduce)"}[st.path],
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path, st.w.block_size),
@@ -696,10 +757,14 @@ def run_ours(args):
         "parity": parity_on_sample(st, base) if base else None,
         "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_steps},
-        "gpu_launches": (st.launches_fused if st.path == "fused" else st.launches_separate) * args.steps,
+        "gpu_launches": {"fused": st.launches_fused, "separate": st.launches_separate,
+                         "shared": getattr(st, "launches_shared", None)}[st.path] * args.steps,
         "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
         "host_alloc_us_per_step_steady": st.host_step_us,
+        "shared_prefix": (None if st.plan is None else
+                          {"groups": int(st.plan.groups.shape[0]), "max_shared_len": st.plan.max_shared_len,
+                           "max_own_len": st.plan.max_own_len, "host_plan_us": st.host_plan_us}),
         "prefix_cache": (None if st.prefix is None else
                          {"admit_us_per_request": st.admit_us_per_request, "hit_tokens": st.prefix["hit_tokens"],
                           "blocks_shared": st.prefix["hit_tokens"] // st.w.block_size,
@@ -724,8 +789,9 @@ def main():
     ap.add_argument("--no-swap", action="store_true", help="skip the swap-out / swap-in measurement")
     ap.add_argument("--block-size", type=int, default=16, choices=[8, 16, 32],
                     help="tokens per block (the pages use 16)")
-    ap.add_argument("--path", choices=["fused", "separate"], default="fused",
-                    help="fused: slot write inside the decode launch; separate: paged_kv_write then decode")
+    ap.add_argument("--path", choices=["fused", "separate", "shared"], default="fused",
+                    help="fused: slot write inside the decode launch; separate: paged_kv_write then decode; "
+                         "shared: fused, reading the blocks a group of samples shares once per step")
     ap.add_argument("--reference-seqs", type=int, default=16)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="smaller batch of the same recipe (profiling); the default is the full workload")

@@ -74,6 +74,8 @@ extern "C" {
 #define PKV_DEV_BAD_CONTEXT 4    /* context_len < 1, beyond the table row, or
                                     above the max_context_len of the launch   */
 #define PKV_DEV_WAIT_TIMEOUT 8   /* an on-chip copy wait gave up (bounded spin) */
+#define PKV_DEV_BAD_PLAN 16      /* a shared-prefix plan that does not fit the
+                                    lengths or the launch (decode_shared)     */
 
 /*
  * paged_kv_write -- store the new tokens' key and value rows in their slots.
@@ -224,6 +226,90 @@ int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const
                               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                               int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Shared-prefix decode.  Samples forked from one prompt (and requests that
+ * found the same cached prefix) hold the same physical blocks for their
+ * common positions ("Copy-on-Write: Sharing KV Cache", "Parallel Sampling"
+ * and "Prefix Caching").  The pages share those blocks to save memory;
+ * these two calls also read them once per step instead of once per sample.
+ * The result is the same attention as paged_attention_decode, within its
+ * rounding.
+ *
+ * pkv_shared_prefix_plan -- host only.  From the host copies of a batch's
+ * block tables and context lengths, find groups: runs of consecutive
+ * sequences (in batch order) whose tables start with the same physical
+ * blocks.  For each group it picks x, the shared length: a multiple of
+ * block_size, below every member's length, and covered by the blocks the
+ * members have in common.
+ *
+ *  block_tables   host, int32 [num_seqs][max_blocks_per_seq]
+ *  context_lens   host, int32 [num_seqs]; each in [1, max_blocks_per_seq *
+ *                 block_size], else PKV_ERR_INVALID_ARG
+ *  max_group      members per group, at most; for decode:
+ *                 PKV_SHARED_MAX_ROWS / (num_q_heads / num_kv_heads).  A
+ *                 longer run splits into several groups.
+ *  min_shared_tokens  a group forms only where x >= this (and x >= one block)
+ *  groups_out     host, int32 [num_seqs][2]: (first sequence, members) of each
+ *                 group, in batch order; *num_groups_out of them are set
+ *  shared_lens_out  host, int32 [num_seqs]: the group's x for each member,
+ *                 0 for a sequence in no group
+ *  max_shared_len_out  max of shared_lens_out (0 if no group)
+ *  max_own_len_out  max over sequences of context_lens[s] - shared_lens_out[s]
+ * Groups have at least 2 members and never overlap.  The result depends only
+ * on the arguments.
+ */
+#define PKV_SHARED_MAX_ROWS 16
+int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
+                           int32_t max_group, int32_t min_shared_tokens, int32_t* groups_out,
+                           int32_t* num_groups_out, int32_t* shared_lens_out, int32_t* max_shared_len_out,
+                           int32_t* max_own_len_out);
+
+/*
+ * paged_attention_decode_shared -- one decode step (one new token per
+ * sequence, optionally fused with its slot write) with a plan from
+ * pkv_shared_prefix_plan.  Computes exactly what paged_attention_decode_mq
+ * with q_len 1 computes:
+ *
+ *   out[s][i][:] = sum_{t < ctx_s} softmax_t(scale * q[s][i] . K_s[t]) * V_s[t]
+ *
+ * but in two passes.  The group pass reads the blocks of positions [0, x) of
+ * a group once, through the first member's table, and attends all members'
+ * query heads to them together (members x (num_q_heads / num_kv_heads) rows
+ * of one 16-row tensor-core operand).  Each sequence's own pass reads its
+ * positions [x, ctx), and the split-K reduce merges both.
+ *
+ *  groups         device, int32 [num_groups][2], as groups_out; may be NULL
+ *                 when num_groups is 0
+ *  shared_lens    device, int32 [num_seqs], as shared_lens_out
+ *  max_shared_len host, as max_shared_len_out (>= every group's x)
+ *  max_own_len    host, as max_own_len_out (>= every ctx_s - x_s); with
+ *                 max_shared_len it sizes the grids, so the host never
+ *                 reads device data
+ *  workspace      >= paged_attention_shared_workspace_bytes(...) bytes,
+ *                 256-byte aligned (never NULL)
+ *  All other arguments are those of paged_attention_decode_mq with q_len 1.
+ * The plan is a promise about the tables: the members of a group hold the
+ * same blocks for positions [0, x).  The call checks what it can see
+ * cheaply: a group outside the batch, with more than PKV_SHARED_MAX_ROWS
+ * rows, or whose x does not fit the launch, raises PKV_DEV_BAD_PLAN and is
+ * skipped; a member whose own x differs from its group's, or is not below
+ * its length, raises PKV_DEV_BAD_PLAN.  Outputs of sequences named in such
+ * a plan are then unspecified (never out-of-bounds accesses).  A sequence in
+ * no group with x = 0 is computed whole by its own pass.  fp32 caches return
+ * PKV_ERR_UNSUPPORTED.
+ */
+size_t paged_attention_shared_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                              int32_t max_context_len);
+int paged_attention_decode_shared(void* out, const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, const int32_t* block_tables,
+                                  int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
+                                  int32_t max_context_len, const int32_t* groups, int32_t num_groups,
+                                  const int32_t* shared_lens, int32_t max_shared_len, int32_t max_own_len,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * paged_attention_decode_noalloc -- paged_attention_decode without a

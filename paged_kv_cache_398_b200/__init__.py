@@ -7,6 +7,8 @@ C ABI of ``include/paged_kv.h``:
 
 * ``paged_kv_write``          -- slot write of the new tokens' K/V
 * ``paged_attention_decode``  -- decode attention through the block tables
+* ``paged_attention_decode_shared`` -- decode reading a group's shared blocks once
+  (plan from ``pkv_shared_prefix_plan``)
 * ``block_copy``              -- copy-on-write block copy
 * ``swap_blocks_out`` / ``swap_blocks_in`` -- preemption: blocks to / from host memory
 * ``BlockAllocator``          -- host block allocator (free list, refcounts, CoW)
@@ -17,17 +19,19 @@ The native library ``libpaged_kv.so`` is built in-tree by
 
 from ._lib import LibraryMissing, PagedKVError
 from .allocator import TABLE_KEEP_TAIL, BlockAllocator, OutOfBlocks
-from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, block_copy, paged_attention_decode,
-                      paged_attention_decode_mq, paged_attention_decode_noalloc,
-                      paged_attention_mq_workspace_bytes, paged_attention_partition_tokens,
-                      paged_attention_workspace_bytes, paged_kv_write, pkv_device_status, pkv_slot_mapping,
-                      swap_blocks_in, swap_blocks_out)
+from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, SHARED_MAX_ROWS, SharedPrefixPlan,
+                      block_copy, paged_attention_decode, paged_attention_decode_mq, paged_attention_decode_noalloc,
+                      paged_attention_decode_shared, paged_attention_mq_workspace_bytes,
+                      paged_attention_partition_tokens, paged_attention_shared_workspace_bytes,
+                      paged_attention_workspace_bytes, paged_kv_write, pkv_device_status, pkv_shared_prefix_plan,
+                      pkv_slot_mapping, swap_blocks_in, swap_blocks_out)
 
 __all__ = [
     "BLOCK_SIZE", "PARTITION_TOKENS", "PARTITION_TOKENS_LONG", "TABLE_KEEP_TAIL", "BlockAllocator",
     "LibraryMissing", "OutOfBlocks",
     "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_decode_mq",
-    "paged_attention_decode_noalloc", "paged_attention_mq_workspace_bytes", "paged_attention_partition_tokens",
-    "paged_attention_workspace_bytes",
+    "paged_attention_decode_noalloc", "paged_attention_decode_shared", "paged_attention_mq_workspace_bytes",
+    "paged_attention_partition_tokens", "paged_attention_shared_workspace_bytes", "paged_attention_workspace_bytes",
+    "SHARED_MAX_ROWS", "SharedPrefixPlan", "pkv_shared_prefix_plan",
     "paged_kv_write", "pkv_device_status", "pkv_slot_mapping", "swap_blocks_in", "swap_blocks_out",
 ]

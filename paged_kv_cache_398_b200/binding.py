@@ -10,7 +10,7 @@ raise ``PagedKVError``, carrying the library's status code.
 from __future__ import annotations
 
 import ctypes
-from typing import Optional
+from typing import NamedTuple, Optional
 
 import torch
 
@@ -169,6 +169,96 @@ def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, context_le
                                          float(scale), _dtype_code(k_cache), ws_ptr or None, ws_bytes,
                                          _stream(q.device, stream))
     check("paged_attention_decode_mq", rc)
+    return out
+
+
+SHARED_MAX_ROWS = C["PKV_SHARED_MAX_ROWS"]
+
+
+class SharedPrefixPlan(NamedTuple):
+    """pkv_shared_prefix_plan's result: groups int32 [num_groups, 2] (first
+    sequence, members), shared_lens int32 [S], and the two grid bounds."""
+    groups: torch.Tensor
+    shared_lens: torch.Tensor
+    max_shared_len: int
+    max_own_len: int
+
+    def to(self, device) -> "SharedPrefixPlan":
+        return SharedPrefixPlan(self.groups.to(device), self.shared_lens.to(device), self.max_shared_len,
+                                self.max_own_len)
+
+
+def pkv_shared_prefix_plan(block_tables, context_lens, block_size: int, max_group: int,
+                           min_shared_tokens: int = 128) -> SharedPrefixPlan:
+    """Groups of consecutive sequences whose tables start with the same
+    blocks, from HOST int32 block_tables [S, MB] and context_lens [S].
+    max_group: members per group, at most (SHARED_MAX_ROWS // (Hq // Hkv)
+    for decode)."""
+    bt = torch.as_tensor(block_tables, dtype=torch.int32).contiguous()
+    cl = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
+    if bt.device.type != "cpu" or cl.device.type != "cpu" or bt.dim() != 2 or cl.dim() != 1 or \
+            bt.shape[0] != cl.shape[0]:
+        raise ValueError("block_tables [S, MB] and context_lens [S] must be host int32 tensors")
+    S = cl.shape[0]
+    groups = torch.empty(max(S, 1), 2, dtype=torch.int32)
+    shared = torch.empty(max(S, 1), dtype=torch.int32)
+    ng, mx_shared, mx_own = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    check("pkv_shared_prefix_plan", lib().pkv_shared_prefix_plan(
+        bt.data_ptr() if S else None, max(bt.shape[1], 1), cl.data_ptr() if S else None, S, int(block_size),
+        int(max_group), int(min_shared_tokens), groups.data_ptr(), ctypes.byref(ng), shared.data_ptr(),
+        ctypes.byref(mx_shared), ctypes.byref(mx_own)))
+    return SharedPrefixPlan(groups[:ng.value].clone(), shared[:S].clone(), int(mx_shared.value), int(mx_own.value))
+
+
+def paged_attention_shared_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
+                                           max_context_len: int) -> int:
+    return int(lib().paged_attention_shared_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))
+
+
+def paged_attention_decode_shared(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                  max_context_len: int, groups, shared_lens, max_shared_len: int, max_own_len: int,
+                                  k_new=None, v_new=None, workspace: Optional[torch.Tensor] = None,
+                                  stream=None) -> torch.Tensor:
+    """Decode q [S, Hq, D] reading each group's shared blocks once; the plan
+    (groups [num_groups, 2], shared_lens [S] on the GPU, the two bounds) is
+    pkv_shared_prefix_plan's.  With k_new / v_new [S, Hkv, D] the new
+    tokens are written to their slots in the same call.  Returns out [S, Hq, D]."""
+    NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
+    _cuda("q", q, k_cache.dtype, 3)
+    _cuda("out", out, k_cache.dtype, 3)
+    _cuda("block_tables", block_tables, torch.int32, 2)
+    _cuda("context_lens", context_lens, torch.int32, 1)
+    _cuda("shared_lens", shared_lens, torch.int32, 1)
+    S, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (S, Hq, D):
+        raise ValueError("q/out must be [S, Hq, D] with the cache's head_dim")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S or shared_lens.shape[0] != S:
+        raise ValueError("block_tables/context_lens/shared_lens must have one row per sequence")
+    ng = 0 if groups is None else int(groups.shape[0])
+    if ng:
+        _cuda("groups", groups, torch.int32, 2)
+        if groups.shape[1] != 2:
+            raise ValueError("groups must be [num_groups, 2]")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    kn = vn = None
+    if k_new is not None:
+        _cuda("k_new", k_new, k_cache.dtype, 3)
+        _cuda("v_new", v_new, k_cache.dtype, 3)
+        if tuple(k_new.shape) != (S, Hkv, D) or tuple(v_new.shape) != (S, Hkv, D):
+            raise ValueError("k_new/v_new must be [S, Hkv, D]")
+        kn, vn = k_new.data_ptr(), v_new.data_ptr()
+    if workspace is None:
+        need = paged_attention_shared_workspace_bytes(S, Hq, D, max_context_len)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _cuda("workspace", workspace)
+    rc = lib().paged_attention_decode_shared(
+        out.data_ptr(), q.data_ptr(), kn, vn, k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
+        block_tables.shape[1], context_lens.data_ptr(), S, int(max_context_len),
+        groups.data_ptr() if ng else None, ng, shared_lens.data_ptr(), int(max_shared_len), int(max_own_len),
+        Hq, Hkv, D, B, NB, float(scale), _dtype_code(k_cache), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream(q.device, stream))
+    check("paged_attention_decode_shared", rc)
     return out
 
 

@@ -239,7 +239,20 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 // partition holds them, and patched into the staged tiles before use.
 // PT: partition size in tokens (kPartTokens, or kLongPartTokens for large
 // batches of long contexts).
-template <typename T, int D, int G, bool kMQ, int B, int PT>
+// kPlan (paged_attention_decode_shared; kPlanNone otherwise):
+//  kPlanGroup: blockIdx.z is group g of plan_groups = (first sequence, n).
+//              Its members' queries (one new token each, q_len = 1) are
+//              rows j * G + g of the 16-row operand, and the CTA attends
+//              partition p of the positions [0, x) that their block tables
+//              share (x = shared_lens[first]), through the first member's
+//              table, with no new tokens and no causal limit.  A member is
+//              covered when its own shared_lens entry is x and x is below its
+//              length (shared_split); rows of other members stay empty.
+//              Every covered row writes a split-K record at slot p.
+//  kPlanOwn:   partition p of sequence s covers its positions from its
+//              shared length x (shared_split) on; its records follow the
+//              group pass's ceil(x / PT).
+template <typename T, int D, int G, bool kMQ, int B, int PT, int kPlan = kPlanNone>
 __global__ void __launch_bounds__(kWarps * 32)
     decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
@@ -248,56 +261,147 @@ __global__ void __launch_bounds__(kWarps * 32)
                                const int32_t* __restrict__ block_tables, int32_t mb,
                                const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t q_len,
                                int32_t num_q_heads, int32_t num_kv_heads, int32_t num_blocks, float scale_log2,
-                               int32_t max_parts, int* status)
+                               int32_t max_parts, int* status, const int32_t* __restrict__ plan_groups,
+                               const int32_t* __restrict__ shared_lens, int32_t num_seqs)
 {
     using C = TcCfg<D>;
     constexpr int part_tokens = PT;
     static_assert(PT == kPartTokens || PT == kLongPartTokens, "partition sizes");
+    static_assert(kPlan != kPlanGroup || kMQ, "the group pass uses the 16-row form");
+    static_assert(kPlan != kPlanOwn || !kMQ, "a sequence's own pass has one query");
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
     constexpr int kRows = kMQ ? 16 : 8;  // operand rows that can hold queries
     constexpr int kChunks = D / 8;       // 16-byte chunks per K or V row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
-    const int p = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int p = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rows = q_len * G;  // live query rows
-
-    // The context length and this thread's entry of the partition's table
-    // slice are loaded together: the entry depends only on (s, p), so the
-    // slice does not wait for the length (one memory round trip before the
-    // first tile copies instead of two).  Entries past the sequence's own
-    // blocks are loaded but never used.
+    const bool report = p == 0 && h == 0 && threadIdx.x == 0;
     constexpr int part_blocks = part_tokens / B;
     static_assert(part_blocks <= kWarps * 32 && part_blocks <= kMaxPartBlocks, "one table entry per thread");
-    const int blk0 = p * part_blocks;
-    int32_t blk_raw = -1;
-    if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
-        blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
-    SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens,
-                               p == 0 && h == 0 && threadIdx.x == 0, status);
-    if (!sr.bad && sr.ctx < q_len) {
-        if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
-        sr.bad = true;
-    }
-    if (sr.bad) {
-        if (p == 0) {
-            for (int i = threadIdx.x; i < rows * D; i += blockDim.x) {
-                const int r = i / D;
-                const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
-                pkv::store_out(out + orow * D + i % D, 0.0f);
-            }
-        }
-        return;
-    }
-    if (p >= sr.nparts) return;
 
-    const int ctx = sr.ctx;
+    // s: the sequence whose block table the CTA walks; row0: the query /
+    // output row of its first query token; ctx: positions attended (the
+    // shared length x in the group pass); part0 / blk0: the partition's first
+    // position / table entry; slot: its split-K record; nparts: the
+    // sequence's partitions in all.  In the group pass, cover bit j marks
+    // member j as computed here.
+    int s, row0, nq, ctx, part0, blk0, slot, nparts, x_own = 0;
+    uint32_t cover = 0u;
+    int32_t blk_raw = -1;
+    if constexpr (kPlan == kPlanGroup) {
+        const int g = blockIdx.z;
+        const int first = pkv::ld_early(plan_groups + 2 * (int64_t)g);
+        const int n = pkv::ld_early(plan_groups + 2 * (int64_t)g + 1);
+        if (first < 0 || n < 1 || n * G > kRows || first > num_seqs - n) {
+            if (report) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+            return;
+        }
+        const int x = pkv::ld_early(shared_lens + first);
+        if (x < 1 || x % B != 0 || x > max_ctx || (int64_t)x > (int64_t)mb * B ||
+            (x + part_tokens - 1) / part_tokens > (int)gridDim.x) {
+            if (report) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+            return;
+        }
+        if (p * part_tokens >= x) return;
+        s = first;
+        row0 = first;
+        nq = n;
+        ctx = x;
+        part0 = p * part_tokens;
+        blk0 = p * part_blocks;
+        slot = p;
+        nparts = 2;  // records, never the final output
+        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
+            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+        // members: covered when their own split is x (warp 0, one lane each)
+        if (warp == 0) {
+            bool cov = false, stray = false;
+            if (lane < n) {
+                const int cj = pkv::ld_early(context_lens + first + lane);
+                const int xj = pkv::ld_early(shared_lens + first + lane);
+                cov = xj == x && cj >= 1 && cj <= max_ctx && (int64_t)cj <= (int64_t)mb * B &&
+                      shared_split(xj, cj, B) == x;
+                stray = !cov;
+            }
+            cover = __ballot_sync(0xffffffffu, cov);
+            const uint32_t strays = __ballot_sync(0xffffffffu, stray);  // the whole warp votes
+            if (report && strays != 0u) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+        }
+    } else if constexpr (kPlan == kPlanOwn) {
+        s = blockIdx.z;
+        const int x_raw = pkv::ld_early(shared_lens + s);
+        SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens, report, status);
+        if (!sr.bad && sr.ctx < q_len) {
+            if (report) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
+            sr.bad = true;
+        }
+        if (sr.bad) {
+            if (p == 0) {
+                for (int i = threadIdx.x; i < q_len * G * D; i += blockDim.x) {
+                    const int r = i / D;
+                    const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
+                    pkv::store_out(out + orow * D + i % D, 0.0f);
+                }
+            }
+            return;
+        }
+        const int x = shared_split(x_raw, sr.ctx, B);
+        const int own_parts = (sr.ctx - x + part_tokens - 1) / part_tokens;
+        if (report && ((x_raw != 0 && x == 0) || own_parts > (int)gridDim.x))
+            pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+        if (p >= own_parts) return;
+        row0 = s * q_len;
+        nq = q_len;
+        ctx = sr.ctx;
+        part0 = x + p * part_tokens;
+        blk0 = part0 / B;
+        x_own = x;  // slot and nparts follow from it after the loop
+        slot = nparts = 0;
+        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
+            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+    } else {
+        // The context length and this thread's entry of the partition's table
+        // slice are loaded together: the entry depends only on (s, p), so the
+        // slice does not wait for the length (one memory round trip before
+        // the first tile copies instead of two).  Entries past the sequence's
+        // own blocks are loaded but never used.
+        s = blockIdx.z;
+        blk0 = p * part_blocks;
+        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
+            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+        SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens,
+                                   p == 0 && h == 0 && threadIdx.x == 0, status);
+        if (!sr.bad && sr.ctx < q_len) {
+            if (p == 0 && h == 0 && threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_CONTEXT);
+            sr.bad = true;
+        }
+        if (sr.bad) {
+            if (p == 0) {
+                for (int i = threadIdx.x; i < q_len * G * D; i += blockDim.x) {
+                    const int r = i / D;
+                    const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
+                    pkv::store_out(out + orow * D + i % D, 0.0f);
+                }
+            }
+            return;
+        }
+        if (p >= sr.nparts) return;
+        row0 = s * q_len;
+        nq = q_len;
+        ctx = sr.ctx;
+        part0 = p * part_tokens;
+        slot = p;
+        nparts = sr.nparts;
+    }
+    const int rows = nq * G;  // query rows
+
     const int nblk_seq = (ctx + B - 1) / B;
-    const int part0 = p * part_tokens;                                         // its first position
     const int nbp = min(part_blocks, nblk_seq - blk0);                          // blocks of this partition
     const int nb = min(part_tokens / kTile, (ctx - part0 + kTile - 1) / kTile);  // its 16-token tiles
-    const int first_new = ctx - q_len;   // position of the first new token
+    // position of the first new token (the group pass has none: its rows see all of [0, x))
+    const int first_new = kPlan == kPlanGroup ? ctx - 1 : ctx - q_len;
     // Fused write: the new tokens that fall in this partition, as token
     // indices [jlo_p, jhi_p).  With up to 16 new tokens (kMQ), right after
     // the prologue every thread stages some of their K / V rows in shared
@@ -307,7 +411,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     constexpr int kNewRows = kMQ ? 16 : 0;  // capacity of the staging area, in tokens
     const int jlo_p = max(0, part0 - first_new);
     const int jhi_p = min(q_len, part0 + part_tokens - first_new);
-    const bool stage_new = kMQ && k_new != nullptr && jhi_p > jlo_p;  // the same for the whole CTA
+    const bool stage_new =
+        kMQ && kPlan != kPlanGroup && k_new != nullptr && jhi_p > jlo_p;  // the same for the whole CTA
     uint64_t* new_bar = reinterpret_cast<uint64_t*>(smem + C::kNewBarOff);
     const uint32_t new_rows = pkv::smem_addr(smem + C::kNewOff);
 
@@ -329,7 +434,14 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (warp == 0 && stage_new) pkv::mbar_init(new_bar, kWarps * 32);  // one arrival per thread
         pkv::fence_mbar_init();
     }
-    __syncthreads();
+    if constexpr (kPlan == kPlanGroup) {
+        // the group pass stages nothing: the staging barrier's word carries the cover bits
+        if (threadIdx.x == 0) *reinterpret_cast<volatile uint32_t*>(new_bar) = cover;
+        __syncthreads();
+        cover = *reinterpret_cast<volatile uint32_t*>(new_bar);
+    } else {
+        __syncthreads();
+    }
 
     const int nw = nb > warp ? (nb - warp + kWarps - 1) / kWarps : 0;
     uint64_t policy = 0;
@@ -359,19 +471,19 @@ __global__ void __launch_bounds__(kWarps * 32)
     // ---- Q as A fragments: rows ra = lane / 4 (a0, a2) and rb = ra + 8 (a1, a3)
     const int ra = lane >> 2, rb = ra + 8;
     const int qd = 2 * (lane & 3);
-    const bool live_a = ra < rows;
-    const bool live_b = kMQ && rb < rows;
+    const bool live_a = ra < rows && (kPlan != kPlanGroup || ((cover >> (ra / G)) & 1u));
+    const bool live_b = kMQ && rb < rows && (kPlan != kPlanGroup || ((cover >> (rb / G)) & 1u));
     uint32_t qa[C::kKSteps][4];
 #pragma unroll
     for (int ks = 0; ks < C::kKSteps; ++ks) {
         qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
         if (live_a) {
-            const T* qrow = q + (((int64_t)s * q_len + ra / G) * num_q_heads + h * G + ra % G) * D + 16 * ks + qd;
+            const T* qrow = q + (((int64_t)row0 + ra / G) * num_q_heads + h * G + ra % G) * D + 16 * ks + qd;
             qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
             qa[ks][2] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
         if (live_b) {
-            const T* qrow = q + (((int64_t)s * q_len + rb / G) * num_q_heads + h * G + rb % G) * D + 16 * ks + qd;
+            const T* qrow = q + (((int64_t)row0 + rb / G) * num_q_heads + h * G + rb % G) * D + 16 * ks + qd;
             qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow);
             qa[ks][3] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
@@ -379,8 +491,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     // Multi-query: positions row ra (rb) may see are < lim_a (lim_b); a row
     // holding no query sees nothing.  (A single query sees the whole context,
     // so that path masks against ctx alone.)
-    const int lim_a = live_a ? first_new + ra / G + 1 : 0;
-    const int lim_b = live_b ? first_new + rb / G + 1 : 0;
+    const int lim_a = live_a ? (kPlan == kPlanGroup ? ctx : first_new + ra / G + 1) : 0;
+    const int lim_b = live_b ? (kPlan == kPlanGroup ? ctx : first_new + rb / G + 1) : 0;
 
     // ---- per-lane ldmatrix addressing (128-byte swizzle: chunk c of row r is at c ^ (r % 8))
     const int mi = lane >> 3, r8 = lane & 7;
@@ -729,7 +841,12 @@ __global__ void __launch_bounds__(kWarps * 32)
     // outputs; the weights of the warps' records are computed once per row.
     constexpr int kPer = D / 32;
     using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
+    if constexpr (kPlan == kPlanOwn) {
+        slot = (x_own + part_tokens - 1) / part_tokens + p;
+        nparts = split_parts(x_own, ctx, part_tokens);
+    }
     for (int r = warp; r < rows; r += kWarps) {
+        if (kPlan == kPlanGroup && !((cover >> (r / G)) & 1u)) continue;  // a member computed elsewhere
         float mw[kWarps];
         float M = -INFINITY;
 #pragma unroll
@@ -751,8 +868,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
             for (int e = 0; e < kPer; ++e) O[e] = fmaf(vf[e], wgt, O[e]);
         }
-        const int64_t orow = ((int64_t)s * q_len + r / G) * num_q_heads + h * G + r % G;
-        if (sr.nparts == 1) {
+        const int64_t orow = ((int64_t)row0 + r / G) * num_q_heads + h * G + r % G;
+        if (nparts == 1) {
 #pragma unroll
             for (int e = 0; e < kPer; ++e) pkv::store_out(out + orow * D + lane * kPer + e, O[e] / L);
         } else {
@@ -762,10 +879,10 @@ __global__ void __launch_bounds__(kWarps * 32)
             float* of = reinterpret_cast<float*>(&ov);
 #pragma unroll
             for (int e = 0; e < kPer; ++e) of[e] = O[e];
-            pkv::st_global_hint(reinterpret_cast<Vec*>(ws_acc + (orow * max_parts + p) * D) + lane, ov, keep);
+            pkv::st_global_hint(reinterpret_cast<Vec*>(ws_acc + (orow * max_parts + slot) * D) + lane, ov, keep);
             if (lane == 0) {
-                pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2, M, keep);
-                pkv::st_global_hint(ws_ml + (orow * max_parts + p) * 2 + 1, L, keep);
+                pkv::st_global_hint(ws_ml + (orow * max_parts + slot) * 2, M, keep);
+                pkv::st_global_hint(ws_ml + (orow * max_parts + slot) * 2 + 1, L, keep);
             }
         }
     }

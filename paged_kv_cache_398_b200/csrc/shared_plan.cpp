@@ -1,0 +1,81 @@
+// Host side of shared-prefix decode: find, in a batch's block tables, the
+// runs of consecutive sequences that start with the same physical blocks
+// (samples forked from one prompt, requests that found one cached prefix:
+// "Copy-on-Write: Sharing KV Cache", "Parallel Sampling", "Prefix Caching"),
+// and the length x whose blocks each such group can read once per step.
+//
+// Greedy, in batch order: a group starts at sequence i and takes i + 1,
+// i + 2, ... while the blocks every member has in common still cover at
+// least min_shared_tokens positions and the group has room.  x is those
+// common blocks times the block size, kept below every member's length, so
+// each member still has its own last position (where the step's new token
+// lands) for its own pass.
+#include <algorithm>
+#include <cstdint>
+
+#include "paged_kv.h"
+
+namespace {
+
+// Leading entries of rows a and b that name the same valid block, up to n.
+int32_t common_blocks(const int32_t* a, const int32_t* b, int32_t n)
+{
+    int32_t k = 0;
+    while (k < n && a[k] >= 0 && a[k] == b[k]) ++k;
+    return k;
+}
+
+}  // namespace
+
+extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
+                                      int32_t max_group, int32_t min_shared_tokens, int32_t* groups_out,
+                                      int32_t* num_groups_out, int32_t* shared_lens_out,
+                                      int32_t* max_shared_len_out, int32_t* max_own_len_out)
+{
+    if (num_seqs < 0 || max_blocks_per_seq < 1 || block_size < 1 || max_group < 1 || min_shared_tokens < 0 ||
+        !num_groups_out || !max_shared_len_out || !max_own_len_out)
+        return PKV_ERR_INVALID_ARG;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !groups_out || !shared_lens_out))
+        return PKV_ERR_INVALID_ARG;
+    const int64_t cap = (int64_t)max_blocks_per_seq * block_size;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (context_lens[s] < 1 || context_lens[s] > cap) return PKV_ERR_INVALID_ARG;
+
+    auto row = [&](int32_t s) { return block_tables + (int64_t)s * max_blocks_per_seq; };
+    // blocks of sequence s that lie wholly below its last position
+    auto below_last = [&](int32_t s) { return (context_lens[s] - 1) / block_size; };
+    const int64_t min_tokens = std::max<int64_t>(min_shared_tokens, block_size);
+
+    int32_t ng = 0, max_shared = 0, max_own = 0;
+    int32_t i = 0;
+    while (i < num_seqs) {
+        int32_t common = below_last(i);  // blocks all members hold, so far
+        int32_t n = 1;
+        while (i + n < num_seqs && n < max_group) {
+            const int32_t j = i + n;
+            const int32_t c = common_blocks(row(i), row(j), std::min(common, below_last(j)));
+            if ((int64_t)c * block_size < min_tokens) break;
+            common = c;
+            ++n;
+        }
+        const int32_t x = n >= 2 ? common * block_size : 0;
+        if (n >= 2) {
+            groups_out[2 * ng] = i;
+            groups_out[2 * ng + 1] = n;
+            ++ng;
+        } else {
+            n = 1;
+        }
+        for (int32_t j = i; j < i + n; ++j) {
+            shared_lens_out[j] = x;
+            max_own = std::max(max_own, context_lens[j] - x);
+        }
+        max_shared = std::max(max_shared, x);
+        i += n;
+    }
+    *num_groups_out = ng;
+    *max_shared_len_out = max_shared;
+    *max_own_len_out = max_own;
+    return PKV_OK;
+}

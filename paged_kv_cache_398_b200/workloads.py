@@ -289,3 +289,59 @@ def make_custom(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int
                           copy_pairs=torch.empty(0, 2, dtype=torch.int64), q=q, k_cache=k_cache,
                           v_cache=v_cache, k_new=k_new, v_new=v_new, scale=1.0 / math.sqrt(D),
                           seed=seed, meta={"workload": "custom"})
+
+
+def make_sampling(num_prompts: int, samples: int, prompt_range, output_range, num_q_heads: int,
+                  num_kv_heads: int, head_dim: int, dtype, device="cpu", *, seed: int = 1234,
+                  block_size: int = BLOCK_SIZE) -> DecodeWorkload:
+    """Parallel sampling with any head shape: `samples` consecutive sequences
+    per prompt share the prompt's full blocks; the prompt's partial last
+    block stays with sample 0 and the other samples get fresh blocks filled by
+    copy-on-write copies (the step's copy pairs); each sample then has its own
+    output blocks.  Prompt and output lengths are uniform in the given
+    inclusive ranges.  The layout of workload "8b_gqa_sampling", with the
+    same draw order (lengths, pool permutation, Q, cache, new K/V)."""
+    g = torch.Generator().manual_seed(seed)
+    B = block_size
+    plen = torch.randint(prompt_range[0], prompt_range[1] + 1, (num_prompts,), generator=g).tolist()
+    olen = torch.randint(output_range[0], output_range[1] + 1, (num_prompts * samples,), generator=g).tolist()
+    ctx = [plen[i // samples] + olen[i] for i in range(num_prompts * samples)]
+    need = 0
+    for i in range(num_prompts):
+        need += plen[i] // B + (samples if plen[i] % B else 0)
+        for j in range(samples):
+            need += _nblk(ctx[i * samples + j], B) - _nblk(plen[i], B)
+    NB = need + _nblk(need, 8)
+    perm = torch.randperm(NB, generator=g).tolist()
+    k, tables, pairs = 0, [], []
+    for i in range(num_prompts):
+        full = perm[k:k + plen[i] // B]
+        k += plen[i] // B
+        part = []
+        if plen[i] % B:
+            part = perm[k:k + samples]
+            k += samples
+            pairs += [(part[0], part[j]) for j in range(1, samples)]
+        for j in range(samples):
+            nout = _nblk(ctx[i * samples + j], B) - _nblk(plen[i], B)
+            tables.append(full + ([part[j]] if part else []) + perm[k:k + nout])
+            k += nout
+    MB = max(len(t) for t in tables)
+    bt = torch.full((len(tables), MB), -1, dtype=torch.int32)
+    for s, row in enumerate(tables):
+        bt[s, :len(row)] = torch.tensor(row, dtype=torch.int32)
+    S, Hq, Hkv, D = len(ctx), num_q_heads, num_kv_heads, head_dim
+    dev = torch.device(device)
+    gd = g if dev.type == "cpu" else torch.Generator(device=dev).manual_seed(seed)
+    q = _randn((S, Hq, D), dtype, gd, dev)
+    k_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
+    v_cache = _randn((NB, Hkv, B, D), dtype, gd, dev)
+    k_new = _randn((S, Hkv, D), dtype, gd, dev)
+    v_new = _randn((S, Hkv, D), dtype, gd, dev)
+    return DecodeWorkload(name="sampling", dtype=dtype, num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv,
+                          head_dim=D, block_size=B, num_blocks=NB,
+                          context_lens=torch.tensor(ctx, dtype=torch.int32), block_tables=bt,
+                          copy_pairs=torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2), q=q,
+                          k_cache=k_cache, v_cache=v_cache, k_new=k_new, v_new=v_new,
+                          scale=1.0 / math.sqrt(D), seed=seed,
+                          meta={"workload": "sampling", "prompt_lens": plen, "samples": samples})

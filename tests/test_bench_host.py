@@ -36,6 +36,35 @@ def test_sample_gives_the_same_outputs_as_the_whole_batch():
     assert np.array_equal(np.stack(refs), whole[seqs])
 
 
+def test_repeated_step_reference_matches_the_batch_stepped_twice():
+    """A sample whose new token lands in the copy-on-write source block makes
+    a repeated step differ from the first; the sampled reference of the
+    repeated step equals the whole batch's oracle step applied twice."""
+    w = make_workload(5, device="cpu", num_prompts=40, max_prompt=300, max_output=6)
+    B = w.block_size
+    srcs = {int(a) for a, _ in w.copy_pairs.tolist()}
+    writers_into_src = [s for s in range(w.num_seqs)
+                        if int(w.block_tables[s, (int(w.context_lens[s]) - 1) // B]) in srcs]
+    assert writers_into_src                            # the case this covers occurs in this batch
+    seqs = sorted({s + 1 for s in writers_into_src if s % 4 == 0} | {2, 5})
+    sub = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs, repeated=True)
+    refs = []
+    bench.oracle_step_timed(sub, 2, keep=refs)
+    # the whole batch, stepped twice by the oracle
+    import oracle
+    from oracle.allocator_model import slot_for_position
+    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - 1, B)
+                          for s in range(w.num_seqs)], dtype=torch.int64)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    for _ in range(2):
+        oracle.block_copy(k, v, w.copy_pairs)
+        oracle.kv_write(k, v, w.k_new, w.v_new, slots)
+    twice = oracle.paged_decode(w.q, k, v, w.block_tables, w.context_lens, w.scale)
+    assert np.array_equal(np.stack(refs), twice[seqs])
+    once = _full_oracle_step(w)
+    assert not np.array_equal(once[seqs], twice[seqs])   # the repetition does change these rows
+
+
 def test_parity_summary_counts_out_of_tolerance_elements():
     w = make_workload(1, device="cpu")
     seqs = list(range(w.num_seqs))

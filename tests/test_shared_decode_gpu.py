@@ -1,0 +1,195 @@
+"""Shared-prefix decode against the oracle (needs a B200).
+
+paged_attention_decode_shared reads the blocks a group of samples shares
+once and attends all the group's query heads to them together, then each
+sample's own blocks, and merges both.  The oracle knows nothing of groups:
+it applies the step's copy-on-write copies and slot writes to a CPU copy of
+the cache and decodes every sequence alone through its own block table.
+Writes must be bit-exact; attention within |gpu - ref| <= 2e-3 + 1e-2 |ref|.
+"""
+
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_398_b200 as pkv
+from paged_kv_cache_398_b200.workloads import make_sampling, make_workload
+from test_parity_gpu import _sub_workload, assert_close, oracle_slots, oracle_step
+
+pytestmark = pytest.mark.gpu
+BAD_PLAN = pkv._lib.C["PKV_DEV_BAD_PLAN"]
+
+
+@pytest.fixture(autouse=True)
+def _clean_status(cuda_device):
+    pkv.pkv_device_status(0, clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def shared_step(g, host, min_shared_tokens=128, plan=None, out=None):
+    """Copy-on-write copies, then the fused write + shared-prefix decode (product)."""
+    G = g.num_q_heads // g.num_kv_heads
+    if plan is None:
+        plan = pkv.pkv_shared_prefix_plan(host.block_tables, host.context_lens, host.block_size,
+                                          pkv.SHARED_MAX_ROWS // G, min_shared_tokens)
+    if g.copy_pairs.numel():
+        pkv.block_copy(g.k_cache, g.v_cache, g.copy_pairs.cpu())
+    d = plan.to("cuda")
+    out = torch.empty_like(g.q) if out is None else out
+    pkv.paged_attention_decode_shared(out, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale,
+                                      g.max_context_len, d.groups, d.shared_lens, d.max_shared_len,
+                                      d.max_own_len, k_new=g.k_new, v_new=g.v_new)
+    return out, plan
+
+
+def _parity(w, min_shared_tokens=128):
+    g = w.to("cuda")
+    out, plan = shared_step(g, w, min_shared_tokens)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(0) == 0
+    ref, k_ref, v_ref = oracle_step(w, oracle_slots(w))
+    assert torch.equal(g.k_cache.cpu(), k_ref) and torch.equal(g.v_cache.cpu(), v_ref)
+    assert_close(out, ref, f"shared decode {w.dtype} B={w.block_size} G={w.num_q_heads // w.num_kv_heads}")
+    return plan
+
+
+@pytest.mark.parametrize("dtype,B,D,Hq,Hkv,samples", [
+    (torch.bfloat16, 16, 128, 32, 8, 4),   # the 8B-GQA sampling shape: 16 rows per group
+    (torch.float16, 8, 64, 4, 4, 16),      # one query head per kv head: 16 samples per group
+    (torch.bfloat16, 32, 128, 16, 2, 2),   # 8 query heads per kv head: groups of 2
+    (torch.float16, 16, 128, 8, 4, 8),     # 2 per kv head: 8 samples
+    (torch.bfloat16, 8, 128, 8, 2, 3),     # groups smaller than the operand allows
+])
+def test_shared_decode_matches_oracle(dtype, B, D, Hq, Hkv, samples):
+    w = make_sampling(5, samples, (1, 1400), (1, 300), Hq, Hkv, D, dtype, seed=70 + B + samples, block_size=B)
+    plan = _parity(w)
+    # every prompt with at least 128 shared tokens forms a group of all its samples
+    expect = sum(1 for p in w.meta["prompt_lens"] if (p // B) * B >= 128)
+    assert plan.groups.shape[0] == expect
+    assert all(n == samples for _, n in plan.groups.tolist())
+
+
+def test_shared_lengths_on_partition_edges():
+    # prompts whose shared part ends just before, on and after a partition boundary
+    dtype, B = torch.bfloat16, 16
+    for i, p in enumerate([511, 512, 513, 1023, 1024, 1040]):
+        w = make_sampling(1, 4, (p, p), (1, 40), 32, 8, 128, dtype, seed=90 + i, block_size=B)
+        plan = _parity(w, min_shared_tokens=B)
+        assert plan.shared_lens.tolist() == [(p // B) * B] * 4
+
+
+def test_without_groups_equals_multi_query_decode_bitwise():
+    # no group forms: every sequence goes through its own pass from position 0,
+    # which is the ordinary partitioning of paged_attention_decode_mq
+    w = make_sampling(4, 4, (200, 900), (1, 200), 32, 8, 128, torch.bfloat16, seed=5)
+    a, b = w.to("cuda"), w.to("cuda")
+    out_shared, plan = shared_step(a, w, min_shared_tokens=1 << 20)
+    assert plan.groups.numel() == 0
+    if b.copy_pairs.numel():
+        pkv.block_copy(b.k_cache, b.v_cache, b.copy_pairs.cpu())
+    out_mq = torch.empty(w.num_seqs, 1, w.num_q_heads, w.head_dim, dtype=w.dtype, device="cuda")
+    pkv.paged_attention_decode_mq(out_mq, b.q[:, None].contiguous(), b.k_cache, b.v_cache, b.block_tables,
+                                  b.context_lens, b.scale, b.max_context_len, k_new=b.k_new[:, None].contiguous(),
+                                  v_new=b.v_new[:, None].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(out_shared, out_mq[:, 0])
+    assert torch.equal(a.k_cache, b.k_cache) and torch.equal(a.v_cache, b.v_cache)
+
+
+def test_placement_permutation_is_bitwise_invariant():
+    w = make_sampling(4, 4, (100, 1500), (1, 300), 32, 8, 128, torch.bfloat16, seed=8)
+    perm = torch.randperm(w.num_blocks, generator=torch.Generator().manual_seed(1))
+    inv = torch.argsort(perm)
+    w2 = make_sampling(4, 4, (100, 1500), (1, 300), 32, 8, 128, torch.bfloat16, seed=8)
+    w2.k_cache, w2.v_cache = w.k_cache[inv].clone(), w.v_cache[inv].clone()   # block b moves to perm[b]
+    w2.block_tables = torch.where(w.block_tables >= 0, perm[w.block_tables.clamp(min=0).long()].int(),
+                                  w.block_tables)
+    w2.copy_pairs = perm[w.copy_pairs]
+    o1, _ = shared_step(w.to("cuda"), w)
+    o2, _ = shared_step(w2.to("cuda"), w2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_long_partitions_sampling_batch():
+    # enough (sequence, kv head) pairs and long enough prompts for 1024-token partitions
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    prompts = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // 32)   # 4 samples x 8 kv heads each
+    w = make_sampling(prompts, 4, (2000, 4096), (1, 1024), 32, 8, 128, torch.bfloat16, seed=11)
+    assert pkv.paged_attention_partition_tokens(w.num_seqs, 8, w.max_context_len, w.dtype) == \
+        pkv.PARTITION_TOKENS_LONG
+    plan = _parity(w)
+    assert plan.groups.shape[0] == prompts
+
+
+def test_full_size_sampling_workload_sampled():
+    host = make_workload(5, device="cuda")
+    w = host.to("cuda")
+    S = w.num_seqs
+    order = torch.argsort(host.context_lens, descending=True).tolist()
+    gen = torch.Generator().manual_seed(55)
+    seqs = sorted(set([order[0], order[-1]] + torch.randperm(S, generator=gen)[:6].tolist()))
+    sub = _sub_workload(w, seqs)                   # taken before the product step
+    out, plan = shared_step(w, host)
+    torch.cuda.synchronize()
+    assert plan.groups.shape[0] == sum(1 for p in host.meta["prompt_lens"] if p >= 128)
+    assert pkv.pkv_device_status(0) == 0
+    ref, _, _ = oracle_step(sub, oracle_slots(sub))
+    assert_close(out[torch.tensor(seqs, device="cuda")], ref, "8b_gqa_sampling shared")
+
+
+def test_inconsistent_plans_are_flagged_and_stay_in_bounds():
+    w = make_sampling(3, 4, (300, 600), (1, 100), 32, 8, 128, torch.bfloat16, seed=21)
+    G = 4
+    good = pkv.pkv_shared_prefix_plan(w.block_tables, w.context_lens, w.block_size, pkv.SHARED_MAX_ROWS // G)
+    assert good.groups.shape[0] == 3
+    cases = []
+    bad = good.shared_lens.clone()
+    bad[1] += w.block_size                       # a member whose x differs from its group's
+    cases.append(good._replace(shared_lens=bad))
+    g_out = good.groups.clone()
+    g_out[2, 0] = w.num_seqs - 2                 # a group that runs past the batch
+    cases.append(good._replace(groups=g_out))
+    g_big = good.groups.clone()
+    g_big[0, 1] = 5                              # 5 members x 4 query heads > 16 rows
+    cases.append(good._replace(groups=g_big))
+    for plan in cases:
+        g = w.to("cuda")
+        shared_step(g, w, plan=plan)
+        torch.cuda.synchronize()
+        assert pkv.pkv_device_status(0) & BAD_PLAN
+    # shared lengths past the group grid: x >= 528 needs two 512-token
+    # partitions, the bound given sizes the grid for one
+    w2 = make_sampling(3, 4, (530, 600), (1, 100), 32, 8, 128, torch.bfloat16, seed=22)
+    good2 = pkv.pkv_shared_prefix_plan(w2.block_tables, w2.context_lens, w2.block_size, pkv.SHARED_MAX_ROWS // G)
+    assert good2.max_shared_len > pkv.PARTITION_TOKENS
+    shared_step(w2.to("cuda"), w2, plan=good2._replace(max_shared_len=16))
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(0) & BAD_PLAN
+    # the context is intact: a consistent plan still matches the oracle
+    _parity(w)
+
+
+def test_rejected_calls():
+    w = make_sampling(2, 4, (300, 400), (1, 50), 32, 8, 128, torch.bfloat16, seed=31).to("cuda")
+    plan = pkv.pkv_shared_prefix_plan(w.block_tables.cpu(), w.context_lens.cpu(), 16, 4).to("cuda")
+    out = torch.empty_like(w.q)
+    args = (out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, w.max_context_len,
+            plan.groups, plan.shared_lens)
+    with pytest.raises(pkv.PagedKVError):       # workspace too small
+        pkv.paged_attention_decode_shared(*args, plan.max_shared_len, plan.max_own_len,
+                                          workspace=torch.empty(256, dtype=torch.uint8, device="cuda"))
+    with pytest.raises(pkv.PagedKVError):       # own-length bound of 0
+        pkv.paged_attention_decode_shared(*args, plan.max_shared_len, 0)
+    with pytest.raises(pkv.PagedKVError):       # shared bound not below the longest context
+        pkv.paged_attention_decode_shared(*args, w.max_context_len, plan.max_own_len)
+    f = make_sampling(2, 2, (40, 60), (1, 10), 4, 4, 64, torch.float32, seed=3).to("cuda")
+    fp = pkv.pkv_shared_prefix_plan(f.block_tables.cpu(), f.context_lens.cpu(), 16, 16, 16).to("cuda")
+    with pytest.raises(pkv.PagedKVError) as e:   # fp32: the tensor-core kernel takes 16-bit inputs
+        pkv.paged_attention_decode_shared(torch.empty_like(f.q), f.q, f.k_cache, f.v_cache, f.block_tables,
+                                          f.context_lens, f.scale, f.max_context_len, fp.groups, fp.shared_lens,
+                                          fp.max_shared_len, fp.max_own_len)
+    assert e.value.code == pkv._lib.C["PKV_ERR_UNSUPPORTED"]
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(0) == 0

@@ -12,16 +12,29 @@
 // lands) for its own pass.
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 
 #include "paged_kv.h"
 
 namespace {
 
-// Leading entries of rows a and b that name the same valid block, up to n.
-int32_t common_blocks(const int32_t* a, const int32_t* b, int32_t n)
+// Leading entries of rows a and b that are equal, up to n: whole chunks by
+// memcmp (sibling rows agree over a whole prompt), then the differing chunk
+// entry by entry.
+int32_t common_entries(const int32_t* a, const int32_t* b, int32_t n)
+{
+    constexpr int32_t kChunk = 16;
+    int32_t k = 0;
+    while (k + kChunk <= n && std::memcmp(a + k, b + k, kChunk * sizeof(int32_t)) == 0) k += kChunk;
+    while (k < n && a[k] == b[k]) ++k;
+    return k;
+}
+
+// Leading entries of a row that name a block (non-negative), up to n.
+int32_t valid_entries(const int32_t* a, int32_t n)
 {
     int32_t k = 0;
-    while (k < n && a[k] >= 0 && a[k] == b[k]) ++k;
+    while (k < n && a[k] >= 0) ++k;
     return k;
 }
 
@@ -50,11 +63,11 @@ extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_b
     int32_t ng = 0, max_shared = 0, max_own = 0;
     int32_t i = 0;
     while (i < num_seqs) {
-        int32_t common = below_last(i);  // blocks all members hold, so far
+        int32_t common = valid_entries(row(i), below_last(i));  // blocks all members hold, so far
         int32_t n = 1;
         while (i + n < num_seqs && n < max_group) {
             const int32_t j = i + n;
-            const int32_t c = common_blocks(row(i), row(j), std::min(common, below_last(j)));
+            const int32_t c = common_entries(row(i), row(j), std::min(common, below_last(j)));
             if ((int64_t)c * block_size < min_tokens) break;
             common = c;
             ++n;

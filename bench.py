@@ -164,12 +164,20 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     if path == "shared":
         if q_len != 1:
             raise SystemExit("--path shared decodes one new token per sequence")
+        pt = pkv.paged_attention_partition_tokens(S, w.num_kv_heads, int(lens.max()), w.dtype)
         t0 = time.perf_counter()
         st.plan = pkv.pkv_shared_prefix_plan(tables, lens, w.block_size,
-                                             pkv.SHARED_MAX_ROWS // (w.num_q_heads // w.num_kv_heads))
+                                             pkv.SHARED_MAX_ROWS // (w.num_q_heads // w.num_kv_heads), pt)
         st.host_plan_us = (time.perf_counter() - t0) * 1e6
-        st.groups, st.shared_lens = st.plan.groups, st.plan.shared_lens
-        st.inputs = STEP_INPUTS + ("groups", "shared_lens")
+        times = []                               # as a serving loop pays it, step after step
+        for _ in range(20):
+            t0 = time.perf_counter()
+            pkv.pkv_shared_prefix_plan(tables, lens, w.block_size,
+                                       pkv.SHARED_MAX_ROWS // (w.num_q_heads // w.num_kv_heads), pt)
+            times.append(time.perf_counter() - t0)
+        st.host_plan_us_steady = statistics.median(times) * 1e6
+        st.groups, st.shared_lens, st.work = st.plan.groups, st.plan.shared_lens, st.plan.work
+        st.inputs = STEP_INPUTS + ("groups", "shared_lens", "work")
     st.block_tables = tables.to(device)
     st.context_lens = lens.to(device)
     st.slots = slots.to(device)
@@ -206,15 +214,16 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     st.launches_fused = st.launches_separate - 1
     st.shared_bytes = None
     if st.plan is not None:
-        # block copies, group pass (if any group), own pass, reduce
-        st.launches_shared = (1 if pairs.shape[0] else 0) + (1 if st.plan.groups.shape[0] else 0) + 2
+        # block copies, both passes (one launch), reduce
+        st.launches_shared = (1 if pairs.shape[0] else 0) + 2
         # K/V the two passes must read under the plan: each group's shared
         # positions once, every sequence's own positions once
         x = st.plan.shared_lens.to(torch.int64)
         first = st.plan.groups[:, 0].to(torch.int64)
         tokens = int(x[first].sum()) + int((ctx - x).sum())
         st.shared_bytes = (tokens * w.num_kv_heads * w.head_dim * 2 * e + 2 * S * w.num_q_heads * w.head_dim * e
-                           + 4 * int(nblk.sum()) + 4 * S + 4 * S + 8 * first.numel() + st.write_bytes)
+                           + 4 * int(nblk.sum()) + 4 * S + 4 * S + 8 * first.numel()
+                           + 8 * st.plan.work.shape[0] + st.write_bytes)
     return st
 
 
@@ -292,8 +301,8 @@ def run_step(st, ev=None):
     elif st.path == "shared":
         pl = st.plan
         pkv.paged_attention_decode_shared(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
-                                          st.w.scale, st.max_ctx, st.groups, st.shared_lens, pl.max_shared_len,
-                                          pl.max_own_len, k_new=st.k_new, v_new=st.v_new, workspace=st.workspace)
+                                          st.w.scale, st.max_ctx, st.groups, st.shared_lens, st.work, pl.part_tokens,
+                                          k_new=st.k_new, v_new=st.v_new, workspace=st.workspace)
     else:
         pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                       st.w.scale, st.max_ctx, k_new=st.k_new4, v_new=st.v_new4,
@@ -746,7 +755,7 @@ def run_ours(args):
         "roofline": {"kernel": {"fused": "paged_attention_decode_mq with fused slot write "
                                          "(partition kernel + split-K reduce)",
                                 "shared": "paged_attention_decode_shared with fused slot write "
-                                          "(group pass + own pass + split-K reduce)",
+                                          "(group and own passes in one launch + split-K reduce)",
                                 "separate": "paged_attention_decode (partition kernel + split-K reduce)"}[st.path],
                      "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
@@ -763,8 +772,10 @@ def run_ours(args):
         "host_alloc_us_per_step": st.host_alloc_us,
         "host_alloc_us_per_step_steady": st.host_step_us,
         "shared_prefix": (None if st.plan is None else
-                          {"groups": int(st.plan.groups.shape[0]), "max_shared_len": st.plan.max_shared_len,
-                           "max_own_len": st.plan.max_own_len, "host_plan_us": st.host_plan_us}),
+                          {"groups": int(st.plan.groups.shape[0]), "work_items": int(st.plan.work.shape[0]),
+                           "max_shared_len": st.plan.max_shared_len,
+                           "max_own_len": st.plan.max_own_len, "host_plan_us": st.host_plan_us,
+                           "host_plan_us_steady": st.host_plan_us_steady}),
         "prefix_cache": (None if st.prefix is None else
                          {"admit_us_per_request": st.admit_us_per_request, "hit_tokens": st.prefix["hit_tokens"],
                           "blocks_shared": st.prefix["hit_tokens"] // st.w.block_size,

@@ -250,10 +250,20 @@ int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const
  *                 PKV_SHARED_MAX_ROWS / (num_q_heads / num_kv_heads).  A
  *                 longer run splits into several groups.
  *  min_shared_tokens  a group forms only where x >= this (and x >= one block)
+ *  part_tokens    the decode launch's partition size:
+ *                 paged_attention_partition_tokens(num_seqs, num_kv_heads,
+ *                 max_context_len, dtype)
  *  groups_out     host, int32 [num_seqs][2]: (first sequence, members) of each
  *                 group, in batch order; *num_groups_out of them are set
  *  shared_lens_out  host, int32 [num_seqs]: the group's x for each member,
  *                 0 for a sequence in no group
+ *  work_out       host, int32 [work_cap][2]: the decode launch's work items,
+ *                 *num_work_out of them.  (~g, p) is partition p (of
+ *                 part_tokens positions) of group g's shared positions
+ *                 [0, x); (s, p) is partition p of sequence s's own positions
+ *                 [x, ctx).  Longest first.  work_out NULL: only
+ *                 *num_work_out is set (a size query).  A work_cap below the
+ *                 count returns PKV_ERR_INVALID_ARG with *num_work_out set.
  *  max_shared_len_out  max of shared_lens_out (0 if no group)
  *  max_own_len_out  max over sequences of context_lens[s] - shared_lens_out[s]
  * Groups have at least 2 members and never overlap.  The result depends only
@@ -262,9 +272,10 @@ int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const
 #define PKV_SHARED_MAX_ROWS 16
 int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_seq,
                            const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
-                           int32_t max_group, int32_t min_shared_tokens, int32_t* groups_out,
-                           int32_t* num_groups_out, int32_t* shared_lens_out, int32_t* max_shared_len_out,
-                           int32_t* max_own_len_out);
+                           int32_t max_group, int32_t min_shared_tokens, int32_t part_tokens,
+                           int32_t* groups_out, int32_t* num_groups_out, int32_t* shared_lens_out,
+                           int32_t* work_out, int32_t work_cap, int32_t* num_work_out,
+                           int32_t* max_shared_len_out, int32_t* max_own_len_out);
 
 /*
  * paged_attention_decode_shared -- one decode step (one new token per
@@ -274,28 +285,32 @@ int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_s
  *
  *   out[s][i][:] = sum_{t < ctx_s} softmax_t(scale * q[s][i] . K_s[t]) * V_s[t]
  *
- * but in two passes.  The group pass reads the blocks of positions [0, x) of
- * a group once, through the first member's table, and attends all members'
- * query heads to them together (members x (num_q_heads / num_kv_heads) rows
- * of one 16-row tensor-core operand).  Each sequence's own pass reads its
- * positions [x, ctx), and the split-K reduce merges both.
+ * but in two passes, run by one launch over the plan's work list.  The group
+ * pass reads the blocks of positions [0, x) of a group once, through the
+ * first member's table, and attends all members' query heads to them
+ * together (members x (num_q_heads / num_kv_heads) rows of one 16-row
+ * tensor-core operand).  Each sequence's own pass reads its positions
+ * [x, ctx), and the split-K reduce merges both.
  *
  *  groups         device, int32 [num_groups][2], as groups_out; may be NULL
  *                 when num_groups is 0
  *  shared_lens    device, int32 [num_seqs], as shared_lens_out
- *  max_shared_len host, as max_shared_len_out (>= every group's x)
- *  max_own_len    host, as max_own_len_out (>= every ctx_s - x_s); with
- *                 max_shared_len it sizes the grids, so the host never
- *                 reads device data
+ *  work           device, int32 [num_work][2], as work_out, 8-byte aligned;
+ *                 num_work (>= 1) sizes the grid, so the host never reads
+ *                 device data
+ *  work_part_tokens  the part_tokens the list was made for; it must equal
+ *                 this launch's partition size, else PKV_ERR_INVALID_ARG
  *  workspace      >= paged_attention_shared_workspace_bytes(...) bytes,
  *                 256-byte aligned (never NULL)
  *  All other arguments are those of paged_attention_decode_mq with q_len 1.
  * The plan is a promise about the tables: the members of a group hold the
  * same blocks for positions [0, x).  The call checks what it can see
- * cheaply: a group outside the batch, with more than PKV_SHARED_MAX_ROWS
- * rows, or whose x does not fit the launch, raises PKV_DEV_BAD_PLAN and is
- * skipped; a member whose own x differs from its group's, or is not below
- * its length, raises PKV_DEV_BAD_PLAN.  Outputs of sequences named in such
+ * cheaply: a work item naming a group or sequence outside the batch or a
+ * partition past max_context_len, a group with more than
+ * PKV_SHARED_MAX_ROWS rows, or one whose x does not fit the cache or
+ * max_context_len raises PKV_DEV_BAD_PLAN and is skipped; a member whose own
+ * x differs from its group's, or is not below its length, raises
+ * PKV_DEV_BAD_PLAN.  Outputs of sequences named in such
  * a plan are then unspecified (never out-of-bounds accesses).  A sequence in
  * no group with x = 0 is computed whole by its own pass.  fp32 caches return
  * PKV_ERR_UNSUPPORTED.
@@ -306,9 +321,9 @@ int paged_attention_decode_shared(void* out, const void* q, const void* k_new, c
                                   void* k_cache, void* v_cache, const int32_t* block_tables,
                                   int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t num_seqs,
                                   int32_t max_context_len, const int32_t* groups, int32_t num_groups,
-                                  const int32_t* shared_lens, int32_t max_shared_len, int32_t max_own_len,
-                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                                  int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
+                                  const int32_t* shared_lens, const int32_t* work, int32_t num_work,
+                                  int32_t work_part_tokens, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t dtype,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*

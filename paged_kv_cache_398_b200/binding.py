@@ -177,23 +177,27 @@ SHARED_MAX_ROWS = C["PKV_SHARED_MAX_ROWS"]
 
 class SharedPrefixPlan(NamedTuple):
     """pkv_shared_prefix_plan's result: groups int32 [num_groups, 2] (first
-    sequence, members), shared_lens int32 [S], and the two grid bounds."""
+    sequence, members), shared_lens int32 [S], the decode launch's work list
+    int32 [num_work, 2] for partitions of part_tokens, and two bounds."""
     groups: torch.Tensor
     shared_lens: torch.Tensor
+    work: torch.Tensor
+    part_tokens: int
     max_shared_len: int
     max_own_len: int
 
     def to(self, device) -> "SharedPrefixPlan":
-        return SharedPrefixPlan(self.groups.to(device), self.shared_lens.to(device), self.max_shared_len,
-                                self.max_own_len)
+        return self._replace(groups=self.groups.to(device), shared_lens=self.shared_lens.to(device),
+                             work=self.work.to(device))
 
 
-def pkv_shared_prefix_plan(block_tables, context_lens, block_size: int, max_group: int,
+def pkv_shared_prefix_plan(block_tables, context_lens, block_size: int, max_group: int, part_tokens: int,
                            min_shared_tokens: int = 128) -> SharedPrefixPlan:
     """Groups of consecutive sequences whose tables start with the same
-    blocks, from HOST int32 block_tables [S, MB] and context_lens [S].
-    max_group: members per group, at most (SHARED_MAX_ROWS // (Hq // Hkv)
-    for decode)."""
+    blocks, and the decode launch's work list, from HOST int32 block_tables
+    [S, MB] and context_lens [S].  max_group: members per group, at most
+    (SHARED_MAX_ROWS // (Hq // Hkv) for decode); part_tokens: the launch's
+    partition size (paged_attention_partition_tokens)."""
     bt = torch.as_tensor(block_tables, dtype=torch.int32).contiguous()
     cl = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
     if bt.device.type != "cpu" or cl.device.type != "cpu" or bt.dim() != 2 or cl.dim() != 1 or \
@@ -202,12 +206,17 @@ def pkv_shared_prefix_plan(block_tables, context_lens, block_size: int, max_grou
     S = cl.shape[0]
     groups = torch.empty(max(S, 1), 2, dtype=torch.int32)
     shared = torch.empty(max(S, 1), dtype=torch.int32)
-    ng, mx_shared, mx_own = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    # at most one item per partition of each sequence, plus one where a split adds one
+    cap = max(1, S * (-(-max(bt.shape[1], 1) * int(block_size) // max(int(part_tokens), 1)) + 1))
+    work = torch.empty(cap, 2, dtype=torch.int32)
+    ng, nw = ctypes.c_int32(0), ctypes.c_int32(0)
+    mx_shared, mx_own = ctypes.c_int32(0), ctypes.c_int32(0)
     check("pkv_shared_prefix_plan", lib().pkv_shared_prefix_plan(
         bt.data_ptr() if S else None, max(bt.shape[1], 1), cl.data_ptr() if S else None, S, int(block_size),
-        int(max_group), int(min_shared_tokens), groups.data_ptr(), ctypes.byref(ng), shared.data_ptr(),
-        ctypes.byref(mx_shared), ctypes.byref(mx_own)))
-    return SharedPrefixPlan(groups[:ng.value].clone(), shared[:S].clone(), int(mx_shared.value), int(mx_own.value))
+        int(max_group), int(min_shared_tokens), int(part_tokens), groups.data_ptr(), ctypes.byref(ng),
+        shared.data_ptr(), work.data_ptr(), cap, ctypes.byref(nw), ctypes.byref(mx_shared), ctypes.byref(mx_own)))
+    return SharedPrefixPlan(groups[:ng.value].clone(), shared[:S].clone(), work[:nw.value].clone(),
+                            int(part_tokens), int(mx_shared.value), int(mx_own.value))
 
 
 def paged_attention_shared_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
@@ -216,24 +225,28 @@ def paged_attention_shared_workspace_bytes(num_seqs: int, num_q_heads: int, head
 
 
 def paged_attention_decode_shared(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
-                                  max_context_len: int, groups, shared_lens, max_shared_len: int, max_own_len: int,
+                                  max_context_len: int, groups, shared_lens, work, work_part_tokens: int,
                                   k_new=None, v_new=None, workspace: Optional[torch.Tensor] = None,
                                   stream=None) -> torch.Tensor:
-    """Decode q [S, Hq, D] reading each group's shared blocks once; the plan
-    (groups [num_groups, 2], shared_lens [S] on the GPU, the two bounds) is
-    pkv_shared_prefix_plan's.  With k_new / v_new [S, Hkv, D] the new
-    tokens are written to their slots in the same call.  Returns out [S, Hq, D]."""
+    """Decode q [S, Hq, D] reading each group's shared blocks once.  groups
+    [num_groups, 2], shared_lens [S] and work [num_work, 2] (int32, on the
+    GPU) and work_part_tokens come from pkv_shared_prefix_plan.  With k_new /
+    v_new [S, Hkv, D] the new tokens are written to their slots in the same
+    call.  Returns out [S, Hq, D]."""
     NB, Hkv, B, D = _cache_shape(k_cache, v_cache)
     _cuda("q", q, k_cache.dtype, 3)
     _cuda("out", out, k_cache.dtype, 3)
     _cuda("block_tables", block_tables, torch.int32, 2)
     _cuda("context_lens", context_lens, torch.int32, 1)
     _cuda("shared_lens", shared_lens, torch.int32, 1)
+    _cuda("work", work, torch.int32, 2)
     S, Hq, Dq = q.shape
     if Dq != D or tuple(out.shape) != (S, Hq, D):
         raise ValueError("q/out must be [S, Hq, D] with the cache's head_dim")
     if block_tables.shape[0] != S or context_lens.shape[0] != S or shared_lens.shape[0] != S:
         raise ValueError("block_tables/context_lens/shared_lens must have one row per sequence")
+    if work.shape[1] != 2:
+        raise ValueError("work must be [num_work, 2]")
     ng = 0 if groups is None else int(groups.shape[0])
     if ng:
         _cuda("groups", groups, torch.int32, 2)
@@ -255,9 +268,9 @@ def paged_attention_decode_shared(out, q, k_cache, v_cache, block_tables, contex
     rc = lib().paged_attention_decode_shared(
         out.data_ptr(), q.data_ptr(), kn, vn, k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(),
         block_tables.shape[1], context_lens.data_ptr(), S, int(max_context_len),
-        groups.data_ptr() if ng else None, ng, shared_lens.data_ptr(), int(max_shared_len), int(max_own_len),
-        Hq, Hkv, D, B, NB, float(scale), _dtype_code(k_cache), workspace.data_ptr(),
-        workspace.numel() * workspace.element_size(), _stream(q.device, stream))
+        groups.data_ptr() if ng else None, ng, shared_lens.data_ptr(), work.data_ptr() if work.numel() else None,
+        int(work.shape[0]), int(work_part_tokens), Hq, Hkv, D, B, NB, float(scale), _dtype_code(k_cache),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(q.device, stream))
     check("paged_attention_decode_shared", rc)
     return out
 

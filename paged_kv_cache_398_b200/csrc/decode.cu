@@ -481,7 +481,7 @@ int launch(const DecodeArgs& a)
                                       static_cast<const T*>(a.q), static_cast<const T*>(a.k_new),
                                       static_cast<const T*>(a.v_new), static_cast<T*>(a.k_cache),
                                       static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.q_len, a.Hq, a.Hkv,
-                                      a.NB, scale_log2, max_parts, a.status, nullptr, nullptr, a.S);
+                                      a.NB, scale_log2, max_parts, a.status);
         };
         rc = with_kernel([&](auto kernel, std::atomic<bool>* configured) {
             const int r = allow_smem(kernel, smem, configured);

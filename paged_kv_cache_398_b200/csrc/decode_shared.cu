@@ -4,15 +4,19 @@
 // "Parallel Sampling" and "Prefix Caching": samples of one prompt hold the
 // same physical blocks for the prompt.)
 //
-// Three launches on the caller's stream, each staged behind the previous one
-// by programmatic dependent launch:
-//  1. group pass, one CTA per (partition p of [0, x), kv head h, group g):
-//     the tensor-core kernel of decode_tc.cuh in its 16-row form, with the
-//     members' query heads as its rows (kPlanGroup).  Each K/V tile of the
-//     shared positions crosses HBM once for the whole group.
-//  2. own pass, one CTA per (partition p of [x, ctx), h, sequence s): the
-//     one-query form, fused with the new token's slot write (kPlanOwn).
-//  3. split-K reduce over the group's partitions followed by the
+// Two launches on the caller's stream, the second staged behind the first by
+// programmatic dependent launch:
+//  1. decode_shared_tc_kernel, one CTA per (work item, kv head).  The host's
+//     work list names every partition of both passes, longest first:
+//     - group pass (partition p of [0, x) of group g): the tensor-core body
+//       of decode_tc.cuh in its 16-row form, with the members' query heads
+//       as its rows (kPlanGroup).  Each K/V tile of the shared positions
+//       crosses HBM once for the whole group;
+//     - own pass (partition p of [x, ctx) of sequence s): the one-query
+//       form, fused with the new token's slot write (kPlanOwn).
+//     One launch for both keeps the SMs busy across the passes, and the list
+//     holds no partition that starts only to exit.
+//  2. split-K reduce over the group's partitions followed by the
 //     sequence's own (decode_reduce_kernel with shared_lens).
 // The workspace has one record slot per row beyond ceil(max_ctx / PT),
 // because a split at x can add one partition.
@@ -36,8 +40,8 @@ struct SharedArgs {
     const int32_t* groups;
     int32_t num_groups;
     const int32_t* shared_lens;
-    int32_t max_shared;
-    int32_t max_own;
+    const int32_t* work;
+    int32_t num_work;
     int32_t Hq;
     int32_t Hkv;
     int32_t NB;
@@ -70,47 +74,30 @@ int launch_shared(const SharedArgs& a)
     if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
     const int smem = C::smem_bytes(0);  // neither pass stages new tokens' rows
 
-    auto run = [&](auto kernel, std::atomic<bool>* configured, dim3 grid, const void* k_new, const void* v_new) {
+    // 1. both passes
+    static std::atomic<bool> cfg_n[64] = {}, cfg_w[64] = {};
+    auto run = [&](auto kernel, std::atomic<bool>* configured) {
         int r = allow_smem(kernel, smem, configured);
         if (r != PKV_OK) return r;
-        cudaLaunchConfig_t cfg = pkv::pdl_config(grid, dim3(kWarps * 32), smem, a.stream);
+        cudaLaunchConfig_t cfg =
+            pkv::pdl_config(dim3((unsigned)((int64_t)a.num_work * a.Hkv)), dim3(kWarps * 32), smem, a.stream);
         cudaLaunchAttribute attr[1];
         pkv::pdl_attribute(&cfg, attr);
         const cudaError_t e = cudaLaunchKernelEx(
             &cfg, kernel, tm_k, tm_v, static_cast<T*>(a.out), ws_acc, ws_ml, static_cast<const T*>(a.q),
-            static_cast<const T*>(k_new), static_cast<const T*>(v_new), static_cast<T*>(a.k_cache),
-            static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, 1, a.Hq, a.Hkv, a.NB, scale_log2, slots,
-            a.status, a.groups, a.shared_lens, a.S);
+            static_cast<const T*>(a.k_new), static_cast<const T*>(a.v_new), static_cast<T*>(a.k_cache),
+            static_cast<T*>(a.v_cache), a.bt, a.mb, a.cl, a.max_ctx, a.Hq, a.Hkv, a.NB, scale_log2, slots, a.status,
+            a.groups, a.num_groups, a.shared_lens, a.S, reinterpret_cast<const int2*>(a.work));
         if (e != cudaSuccess) {
             pkv::record_cuda_error(e);
             return PKV_ERR_CUDA;
         }
         return pkv::check_launch();
     };
-
-    // 1. group pass
-    if (a.num_groups > 0) {
-        static std::atomic<bool> cfg_g[64] = {}, cfg_gw[64] = {};
-        const dim3 grid((unsigned)((a.max_shared + a.part_tokens - 1) / a.part_tokens), (unsigned)a.Hkv,
-                        (unsigned)a.num_groups);
-        rc = wide ? run(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens, kPlanGroup>, cfg_gw, grid,
-                        nullptr, nullptr)
-                  : run(decode_partition_tc_kernel<T, D, G, true, B, kPartTokens, kPlanGroup>, cfg_g, grid, nullptr,
-                        nullptr);
-        if (rc != PKV_OK) return rc;
-    }
-    // 2. each sequence's own positions, with the fused slot write
-    {
-        static std::atomic<bool> cfg_o[64] = {}, cfg_ow[64] = {};
-        const dim3 grid((unsigned)((a.max_own + a.part_tokens - 1) / a.part_tokens), (unsigned)a.Hkv,
-                        (unsigned)a.S);
-        rc = wide ? run(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens, kPlanOwn>, cfg_ow, grid,
-                        a.k_new, a.v_new)
-                  : run(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens, kPlanOwn>, cfg_o, grid, a.k_new,
-                        a.v_new);
-        if (rc != PKV_OK) return rc;
-    }
-    // 3. merge (always: a sequence split at x has records only)
+    rc = wide ? run(decode_shared_tc_kernel<T, D, G, B, kLongPartTokens>, cfg_w)
+              : run(decode_shared_tc_kernel<T, D, G, B, kPartTokens>, cfg_n);
+    if (rc != PKV_OK) return rc;
+    // 2. merge (always: a sequence split at x has records only)
     cudaLaunchConfig_t cfg = pkv::pdl_config(dim3((unsigned)((qrows + 3) / 4)), dim3(128), 0, a.stream);
     cudaLaunchAttribute attr[1];
     pkv::pdl_attribute(&cfg, attr);
@@ -170,10 +157,11 @@ extern "C" int paged_attention_decode_shared(void* out, const void* q, const voi
                                              void* k_cache, void* v_cache, const int32_t* block_tables,
                                              int32_t max_blocks_per_seq, const int32_t* context_lens,
                                              int32_t num_seqs, int32_t max_context_len, const int32_t* groups,
-                                             int32_t num_groups, const int32_t* shared_lens, int32_t max_shared_len,
-                                             int32_t max_own_len, int32_t num_q_heads, int32_t num_kv_heads,
-                                             int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
-                                             int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
+                                             int32_t num_groups, const int32_t* shared_lens, const int32_t* work,
+                                             int32_t num_work, int32_t work_part_tokens, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                             int32_t num_blocks, float scale, int32_t dtype, void* workspace,
+                                             size_t workspace_bytes, void* stream)
 {
     const pkv::NvtxRange nvtx("paged_attention_decode_shared");
     if (pkv::dtype_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
@@ -188,11 +176,10 @@ extern "C" int paged_attention_decode_shared(void* out, const void* q, const voi
     if (num_seqs == 0) return PKV_OK;
     if (max_context_len < 1 || num_seqs > 65535 || num_kv_heads > 65535 || num_groups > num_seqs)
         return PKV_ERR_INVALID_ARG;
-    if (max_own_len < 1 || max_own_len > max_context_len) return PKV_ERR_INVALID_ARG;
-    if (num_groups > 0 && (!groups || ((uintptr_t)groups & 3u) || max_shared_len < 1 ||
-                           max_shared_len >= max_context_len))
-        return PKV_ERR_INVALID_ARG;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !shared_lens || !workspace)
+    if (num_work < 1 || (int64_t)num_work * num_kv_heads > INT32_MAX) return PKV_ERR_INVALID_ARG;
+    if (num_groups > 0 && (!groups || ((uintptr_t)groups & 3u))) return PKV_ERR_INVALID_ARG;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !shared_lens || !work ||
+        !workspace || ((uintptr_t)work & 7u))
         return PKV_ERR_INVALID_ARG;
     if (!pkv::aligned16(q) || !pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) ||
         ((uintptr_t)out % pkv::dtype_bytes(dtype)) || ((uintptr_t)block_tables & 3u) ||
@@ -206,10 +193,11 @@ extern "C" int paged_attention_decode_shared(void* out, const void* q, const voi
     int part_tokens = kPartTokens;
     const int rc = part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, &part_tokens);
     if (rc != PKV_OK) return rc;
+    if (work_part_tokens != part_tokens) return PKV_ERR_INVALID_ARG;  // the list was made for another split
     const SharedArgs a{out,          q,           k_new,           v_new,          k_cache,
                        v_cache,      block_tables, max_blocks_per_seq, context_lens, num_seqs,
                        max_context_len, num_groups > 0 ? groups : nullptr, num_groups, shared_lens,
-                       num_groups > 0 ? max_shared_len : 0, max_own_len, num_q_heads, num_kv_heads, num_blocks,
+                       work,         num_work,    num_q_heads,     num_kv_heads,   num_blocks,
                        block_size,   part_tokens, scale,           workspace,      (cudaStream_t)stream,
                        status};
     if (dtype == PKV_F16) return shared_d<__half>(head_dim, G, a);

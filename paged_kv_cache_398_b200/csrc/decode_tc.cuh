@@ -226,8 +226,8 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
     return alpha;
 }
 
-// One CTA = (partition p, kv head h, sequence s).  q_len new tokens per
-// sequence: query row r = j * G + g is query head h*G + g of new token j,
+// The work of one CTA: partition p, kv head h, and z = sequence s (or, in
+// the group pass, group g).  q_len new tokens per sequence: query row r = j * G + g is query head h*G + g of new token j,
 // which sits at position ctx - q_len + j and sees positions up to its own
 // (q_len = 1: the whole context).
 //  kMQ = false: q_len * G <= 8 rows, the transposed products S^T = K Q^T and
@@ -240,7 +240,7 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 // PT: partition size in tokens (kPartTokens, or kLongPartTokens for large
 // batches of long contexts).
 // kPlan (paged_attention_decode_shared; kPlanNone otherwise):
-//  kPlanGroup: blockIdx.z is group g of plan_groups = (first sequence, n).
+//  kPlanGroup: z is group g of plan_groups = (first sequence, n).
 //              Its members' queries (one new token each, q_len = 1) are
 //              rows j * G + g of the 16-row operand, and the CTA attends
 //              partition p of the positions [0, x) that their block tables
@@ -252,17 +252,19 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 //  kPlanOwn:   partition p of sequence s covers its positions from its
 //              shared length x (shared_split) on; its records follow the
 //              group pass's ceil(x / PT).
-template <typename T, int D, int G, bool kMQ, int B, int PT, int kPlan = kPlanNone>
-__global__ void __launch_bounds__(kWarps * 32)
-    decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                               T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
-                               const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
-                               T* __restrict__ k_cache_w, T* __restrict__ v_cache_w,
-                               const int32_t* __restrict__ block_tables, int32_t mb,
-                               const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t q_len,
-                               int32_t num_q_heads, int32_t num_kv_heads, int32_t num_blocks, float scale_log2,
-                               int32_t max_parts, int* status, const int32_t* __restrict__ plan_groups,
-                               const int32_t* __restrict__ shared_lens, int32_t num_seqs)
+// The kernels below run it for one work item each.
+template <typename T, int D, int G, bool kMQ, int B, int PT, int kPlan>
+__device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUtensorMap* tm_v, T* __restrict__ out,
+                                             float* __restrict__ ws_acc, float* __restrict__ ws_ml,
+                                             const T* __restrict__ q, const T* __restrict__ k_new,
+                                             const T* __restrict__ v_new, T* __restrict__ k_cache_w,
+                                             T* __restrict__ v_cache_w, const int32_t* __restrict__ block_tables,
+                                             int32_t mb, const int32_t* __restrict__ context_lens, int32_t max_ctx,
+                                             int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads,
+                                             int32_t num_blocks, float scale_log2, int32_t max_parts, int* status,
+                                             const int32_t* __restrict__ plan_groups,
+                                             const int32_t* __restrict__ shared_lens, int32_t num_seqs, const int p,
+                                             const int h, const int z)
 {
     using C = TcCfg<D>;
     constexpr int part_tokens = PT;
@@ -275,7 +277,6 @@ __global__ void __launch_bounds__(kWarps * 32)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
-    const int p = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool report = p == 0 && h == 0 && threadIdx.x == 0;
     constexpr int part_blocks = part_tokens / B;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     uint32_t cover = 0u;
     int32_t blk_raw = -1;
     if constexpr (kPlan == kPlanGroup) {
-        const int g = blockIdx.z;
+        const int g = z;
         const int first = pkv::ld_early(plan_groups + 2 * (int64_t)g);
         const int n = pkv::ld_early(plan_groups + 2 * (int64_t)g + 1);
         if (first < 0 || n < 1 || n * G > kRows || first > num_seqs - n) {
@@ -299,8 +300,7 @@ __global__ void __launch_bounds__(kWarps * 32)
             return;
         }
         const int x = pkv::ld_early(shared_lens + first);
-        if (x < 1 || x % B != 0 || x > max_ctx || (int64_t)x > (int64_t)mb * B ||
-            (x + part_tokens - 1) / part_tokens > (int)gridDim.x) {
+        if (x < 1 || x % B != 0 || x > max_ctx || (int64_t)x > (int64_t)mb * B) {
             if (report) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
             return;
         }
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kWarps * 32)
             if (report && strays != 0u) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
         }
     } else if constexpr (kPlan == kPlanOwn) {
-        s = blockIdx.z;
+        s = z;
         const int x_raw = pkv::ld_early(shared_lens + s);
         SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens, report, status);
         if (!sr.bad && sr.ctx < q_len) {
@@ -349,8 +349,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         const int x = shared_split(x_raw, sr.ctx, B);
         const int own_parts = (sr.ctx - x + part_tokens - 1) / part_tokens;
-        if (report && ((x_raw != 0 && x == 0) || own_parts > (int)gridDim.x))
-            pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+        if (report && x_raw != 0 && x == 0) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
         if (p >= own_parts) return;
         row0 = s * q_len;
         nq = q_len;
@@ -367,7 +366,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         // slice does not wait for the length (one memory round trip before
         // the first tile copies instead of two).  Entries past the sequence's
         // own blocks are loaded but never used.
-        s = blockIdx.z;
+        s = z;
         blk0 = p * part_blocks;
         if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
             blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
@@ -447,12 +446,12 @@ __global__ void __launch_bounds__(kWarps * 32)
     uint64_t policy = 0;
     if (lane == 0) {
         policy = pkv::policy_evict_first();
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm_v)) : "memory");
         for (int k = 0; k < nw && k < kStages; ++k) {
             int r0, r1;
             tile_rows<B>(s_blk, nbp, warp + k * kWarps, num_kv_heads, h, r0, r1);
-            tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], &tm_k, &tm_v, r0, r1, B == 8,
+            tc_issue<D>(tiles + (k % kStages) * C::kStageBytes, &bars[k % kStages], tm_k, tm_v, r0, r1, B == 8,
                         policy);
         }
     }
@@ -764,7 +763,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (lane == 0 && k + kStages < nw) {
             int r0, r1;
             tile_rows<B>(s_blk, nbp, warp + (k + kStages) * kWarps, num_kv_heads, h, r0, r1);
-            tc_issue<D>(kbase, &bars[st], &tm_k, &tm_v, r0, r1, B == 8, policy);
+            tc_issue<D>(kbase, &bars[st], tm_k, tm_v, r0, r1, B == 8, policy);
         }
     }
 
@@ -885,6 +884,67 @@ __global__ void __launch_bounds__(kWarps * 32)
                 pkv::st_global_hint(ws_ml + (orow * max_parts + slot) * 2 + 1, L, keep);
             }
         }
+    }
+}
+
+// An ordinary launch: one CTA per (partition, kv head, sequence) of the grid.
+template <typename T, int D, int G, bool kMQ, int B, int PT>
+__global__ void __launch_bounds__(kWarps * 32)
+    decode_partition_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                               T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
+                               const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
+                               T* __restrict__ k_cache_w, T* __restrict__ v_cache_w,
+                               const int32_t* __restrict__ block_tables, int32_t mb,
+                               const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t q_len,
+                               int32_t num_q_heads, int32_t num_kv_heads, int32_t num_blocks, float scale_log2,
+                               int32_t max_parts, int* status)
+{
+    partition_tc<T, D, G, kMQ, B, PT, kPlanNone>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, k_new, v_new, k_cache_w,
+                                                  v_cache_w, block_tables, mb, context_lens, max_ctx, q_len,
+                                                  num_q_heads, num_kv_heads, num_blocks, scale_log2, max_parts,
+                                                  status, nullptr, nullptr, 0, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+// paged_attention_decode_shared: both passes in one launch, one CTA per (work
+// item, kv head), kv head fastest.  A work item (int32 pair) is (~g, p): the
+// group pass over partition p of group g's shared positions, or (s, p):
+// partition p of sequence s's own positions (with its new token's slot
+// write).  The host lists the items longest first, so the long group
+// partitions start early and the short ones fill the tail.  3 CTAs per SM
+// for both forms: the register budget is capped at 168.
+template <typename T, int D, int G, int B, int PT>
+__global__ void __launch_bounds__(kWarps * 32, 3)
+    decode_shared_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            T* __restrict__ out, float* __restrict__ ws_acc, float* __restrict__ ws_ml,
+                            const T* __restrict__ q, const T* __restrict__ k_new, const T* __restrict__ v_new,
+                            T* __restrict__ k_cache_w, T* __restrict__ v_cache_w,
+                            const int32_t* __restrict__ block_tables, int32_t mb,
+                            const int32_t* __restrict__ context_lens, int32_t max_ctx, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t num_blocks, float scale_log2, int32_t max_parts,
+                            int* status, const int32_t* __restrict__ plan_groups, int32_t num_groups,
+                            const int32_t* __restrict__ shared_lens, int32_t num_seqs,
+                            const int2* __restrict__ work)
+{
+    pkv::grid_dependency_wait();  // the work list may come from the previous kernel
+    const int item = (int)(blockIdx.x / (unsigned)num_kv_heads), h = (int)(blockIdx.x % (unsigned)num_kv_heads);
+    int2 w;
+    asm volatile("ld.global.nc.v2.s32 {%0, %1}, [%2];" : "=r"(w.x), "=r"(w.y) : "l"(work + item));
+    // a partition index past ceil(max_ctx / PT) fits no sequence (and keeps p * PT in range)
+    if (w.y < 0 || w.y >= (max_ctx + PT - 1) / PT || (w.x < 0 ? ~w.x >= num_groups : w.x >= num_seqs)) {
+        if (threadIdx.x == 0) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+        return;
+    }
+    if (w.x < 0) {
+        partition_tc<T, D, G, true, B, PT, kPlanGroup>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, nullptr, nullptr,
+                                                        k_cache_w, v_cache_w, block_tables, mb, context_lens, max_ctx,
+                                                        1, num_q_heads, num_kv_heads, num_blocks, scale_log2,
+                                                        max_parts, status, plan_groups, shared_lens, num_seqs, w.y, h,
+                                                        ~w.x);
+    } else {
+        partition_tc<T, D, G, false, B, PT, kPlanOwn>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, k_new, v_new, k_cache_w,
+                                                       v_cache_w, block_tables, mb, context_lens, max_ctx, 1,
+                                                       num_q_heads, num_kv_heads, num_blocks, scale_log2, max_parts,
+                                                       status, plan_groups, shared_lens, num_seqs, w.y, h, w.x);
     }
 }
 

@@ -10,9 +10,16 @@
 // common blocks times the block size, kept below every member's length, so
 // each member still has its own last position (where the step's new token
 // lands) for its own pass.
+//
+// The work list names every partition of both passes for the decode launch
+// (one thread block per item and kv head): (~g, p) for partition p of group
+// g's shared positions, (s, p) for partition p of sequence s's own.  Items go
+// longest first (ties: group items, then batch order), so the long ones
+// start early and the short ones fill the end of the launch.
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "paged_kv.h"
 
@@ -42,12 +49,14 @@ int32_t valid_entries(const int32_t* a, int32_t n)
 
 extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_seq,
                                       const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
-                                      int32_t max_group, int32_t min_shared_tokens, int32_t* groups_out,
-                                      int32_t* num_groups_out, int32_t* shared_lens_out,
+                                      int32_t max_group, int32_t min_shared_tokens, int32_t part_tokens,
+                                      int32_t* groups_out, int32_t* num_groups_out, int32_t* shared_lens_out,
+                                      int32_t* work_out, int32_t work_cap, int32_t* num_work_out,
                                       int32_t* max_shared_len_out, int32_t* max_own_len_out)
 {
     if (num_seqs < 0 || max_blocks_per_seq < 1 || block_size < 1 || max_group < 1 || min_shared_tokens < 0 ||
-        !num_groups_out || !max_shared_len_out || !max_own_len_out)
+        part_tokens < 1 || work_cap < 0 || !num_groups_out || !num_work_out || !max_shared_len_out ||
+        !max_own_len_out)
         return PKV_ERR_INVALID_ARG;
     if (num_seqs > 0 && (!block_tables || !context_lens || !groups_out || !shared_lens_out))
         return PKV_ERR_INVALID_ARG;
@@ -90,5 +99,38 @@ extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_b
     *num_groups_out = ng;
     *max_shared_len_out = max_shared;
     *max_own_len_out = max_own;
+
+    // the work list: (tokens, first, second) per item, longest first
+    struct Item {
+        int32_t tokens, a, p;
+    };
+    std::vector<Item> items;
+    try {
+        items.reserve((size_t)num_seqs + (size_t)ng * 4);
+    } catch (...) {
+        return PKV_ERR_INVALID_ARG;  // no memory for the list: nothing is written
+    }
+    try {
+        for (int32_t g = 0; g < ng; ++g) {
+            const int32_t x = shared_lens_out[groups_out[2 * g]];
+            for (int32_t p = 0; (int64_t)p * part_tokens < x; ++p)
+                items.push_back({std::min(part_tokens, x - p * part_tokens), ~g, p});
+        }
+        for (int32_t s = 0; s < num_seqs; ++s) {
+            const int32_t own = context_lens[s] - shared_lens_out[s];
+            for (int32_t p = 0; (int64_t)p * part_tokens < own; ++p)
+                items.push_back({std::min(part_tokens, own - p * part_tokens), s, p});
+        }
+    } catch (...) {
+        return PKV_ERR_INVALID_ARG;
+    }
+    std::stable_sort(items.begin(), items.end(), [](const Item& l, const Item& r) { return l.tokens > r.tokens; });
+    *num_work_out = (int32_t)items.size();
+    if (!work_out) return PKV_OK;  // a query of the size
+    if ((int64_t)items.size() > work_cap) return PKV_ERR_INVALID_ARG;
+    for (size_t k = 0; k < items.size(); ++k) {
+        work_out[2 * k] = items[k].a;
+        work_out[2 * k + 1] = items[k].p;
+    }
     return PKV_OK;
 }

@@ -27,19 +27,24 @@ def _clean_status(cuda_device):
     torch.cuda.synchronize()
 
 
+def make_plan(host, min_shared_tokens=128):
+    G = host.num_q_heads // host.num_kv_heads
+    pt = pkv.paged_attention_partition_tokens(host.num_seqs, host.num_kv_heads, host.max_context_len, host.dtype)
+    return pkv.pkv_shared_prefix_plan(host.block_tables, host.context_lens, host.block_size,
+                                      pkv.SHARED_MAX_ROWS // G, pt, min_shared_tokens)
+
+
 def shared_step(g, host, min_shared_tokens=128, plan=None, out=None):
     """Copy-on-write copies, then the fused write + shared-prefix decode (product)."""
-    G = g.num_q_heads // g.num_kv_heads
     if plan is None:
-        plan = pkv.pkv_shared_prefix_plan(host.block_tables, host.context_lens, host.block_size,
-                                          pkv.SHARED_MAX_ROWS // G, min_shared_tokens)
+        plan = make_plan(host, min_shared_tokens)
     if g.copy_pairs.numel():
         pkv.block_copy(g.k_cache, g.v_cache, g.copy_pairs.cpu())
     d = plan.to("cuda")
     out = torch.empty_like(g.q) if out is None else out
     pkv.paged_attention_decode_shared(out, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale,
-                                      g.max_context_len, d.groups, d.shared_lens, d.max_shared_len,
-                                      d.max_own_len, k_new=g.k_new, v_new=g.v_new)
+                                      g.max_context_len, d.groups, d.shared_lens, d.work, d.part_tokens,
+                                      k_new=g.k_new, v_new=g.v_new)
     return out, plan
 
 
@@ -141,8 +146,7 @@ def test_full_size_sampling_workload_sampled():
 
 def test_inconsistent_plans_are_flagged_and_stay_in_bounds():
     w = make_sampling(3, 4, (300, 600), (1, 100), 32, 8, 128, torch.bfloat16, seed=21)
-    G = 4
-    good = pkv.pkv_shared_prefix_plan(w.block_tables, w.context_lens, w.block_size, pkv.SHARED_MAX_ROWS // G)
+    good = make_plan(w)
     assert good.groups.shape[0] == 3
     cases = []
     bad = good.shared_lens.clone()
@@ -154,42 +158,40 @@ def test_inconsistent_plans_are_flagged_and_stay_in_bounds():
     g_big = good.groups.clone()
     g_big[0, 1] = 5                              # 5 members x 4 query heads > 16 rows
     cases.append(good._replace(groups=g_big))
+    for item in ([~7, 0], [w.num_seqs, 0], [0, -1], [0, 1 << 20]):
+        work = good.work.clone()                 # a group or sequence outside the batch, a bad partition
+        work[-1] = torch.tensor(item, dtype=torch.int32)
+        cases.append(good._replace(work=work))
     for plan in cases:
         g = w.to("cuda")
         shared_step(g, w, plan=plan)
         torch.cuda.synchronize()
         assert pkv.pkv_device_status(0) & BAD_PLAN
-    # shared lengths past the group grid: x >= 528 needs two 512-token
-    # partitions, the bound given sizes the grid for one
-    w2 = make_sampling(3, 4, (530, 600), (1, 100), 32, 8, 128, torch.bfloat16, seed=22)
-    good2 = pkv.pkv_shared_prefix_plan(w2.block_tables, w2.context_lens, w2.block_size, pkv.SHARED_MAX_ROWS // G)
-    assert good2.max_shared_len > pkv.PARTITION_TOKENS
-    shared_step(w2.to("cuda"), w2, plan=good2._replace(max_shared_len=16))
-    torch.cuda.synchronize()
-    assert pkv.pkv_device_status(0) & BAD_PLAN
     # the context is intact: a consistent plan still matches the oracle
     _parity(w)
 
 
 def test_rejected_calls():
     w = make_sampling(2, 4, (300, 400), (1, 50), 32, 8, 128, torch.bfloat16, seed=31).to("cuda")
-    plan = pkv.pkv_shared_prefix_plan(w.block_tables.cpu(), w.context_lens.cpu(), 16, 4).to("cuda")
+    host = make_sampling(2, 4, (300, 400), (1, 50), 32, 8, 128, torch.bfloat16, seed=31)
+    plan = make_plan(host).to("cuda")
     out = torch.empty_like(w.q)
     args = (out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, w.max_context_len,
             plan.groups, plan.shared_lens)
     with pytest.raises(pkv.PagedKVError):       # workspace too small
-        pkv.paged_attention_decode_shared(*args, plan.max_shared_len, plan.max_own_len,
+        pkv.paged_attention_decode_shared(*args, plan.work, plan.part_tokens,
                                           workspace=torch.empty(256, dtype=torch.uint8, device="cuda"))
-    with pytest.raises(pkv.PagedKVError):       # own-length bound of 0
-        pkv.paged_attention_decode_shared(*args, plan.max_shared_len, 0)
-    with pytest.raises(pkv.PagedKVError):       # shared bound not below the longest context
-        pkv.paged_attention_decode_shared(*args, w.max_context_len, plan.max_own_len)
-    f = make_sampling(2, 2, (40, 60), (1, 10), 4, 4, 64, torch.float32, seed=3).to("cuda")
-    fp = pkv.pkv_shared_prefix_plan(f.block_tables.cpu(), f.context_lens.cpu(), 16, 16, 16).to("cuda")
+    with pytest.raises(pkv.PagedKVError):       # an empty work list
+        pkv.paged_attention_decode_shared(*args, plan.work[:0], plan.part_tokens)
+    with pytest.raises(pkv.PagedKVError):       # a list made for another partition size
+        pkv.paged_attention_decode_shared(*args, plan.work, plan.part_tokens * 2)
+    f = make_sampling(2, 2, (40, 60), (1, 10), 4, 4, 64, torch.float32, seed=3)
+    fp = pkv.pkv_shared_prefix_plan(f.block_tables, f.context_lens, 16, 16, pkv.PARTITION_TOKENS, 16).to("cuda")
+    f = f.to("cuda")
     with pytest.raises(pkv.PagedKVError) as e:   # fp32: the tensor-core kernel takes 16-bit inputs
         pkv.paged_attention_decode_shared(torch.empty_like(f.q), f.q, f.k_cache, f.v_cache, f.block_tables,
                                           f.context_lens, f.scale, f.max_context_len, fp.groups, fp.shared_lens,
-                                          fp.max_shared_len, fp.max_own_len)
+                                          fp.work, fp.part_tokens)
     assert e.value.code == pkv._lib.C["PKV_ERR_UNSUPPORTED"]
     torch.cuda.synchronize()
     assert pkv.pkv_device_status(0) == 0

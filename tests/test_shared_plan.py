@@ -19,6 +19,7 @@ import torch
 import paged_kv_cache_398_b200 as pkv
 
 B = 16
+PT = 512   # partition size of the work lists
 
 
 def _tables(rows):
@@ -53,18 +54,33 @@ def _check_valid(tables, lens, plan, max_group, min_tokens, block_size=B):
             assert shared[j] == 0
     assert plan.max_shared_len == max(shared + [0])
     assert plan.max_own_len == max(int(lens[j]) - shared[j] for j in range(S))
+    # the work list: every partition of both passes exactly once, longest first
+    pt = plan.part_tokens
+    expect = {}
+    for g, (first, n) in enumerate(plan.groups.tolist()):
+        x = shared[first]
+        for p in range(-(-x // pt)):
+            expect[(~g, p)] = min(pt, x - p * pt)
+    for j in range(S):
+        own = int(lens[j]) - shared[j]
+        for p in range(-(-own // pt)):
+            expect[(j, p)] = min(pt, own - p * pt)
+    items = [tuple(it) for it in plan.work.tolist()]
+    assert len(items) == len(set(items)) and set(items) == set(expect)
+    sizes = [expect[it] for it in items]
+    assert sizes == sorted(sizes, reverse=True)
 
 
 def test_parallel_sampling_example():
     # four outputs of one prompt: blocks 0-5 shared, unique blocks [6,7], [8,9], [10,11], [12,13]
     rows = [[0, 1, 2, 3, 4, 5, 6 + 2 * j, 7 + 2 * j] for j in range(4)]
     lens = torch.tensor([6 * B + 20] * 4, dtype=torch.int32)
-    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=4, min_shared_tokens=B)
+    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=4, part_tokens=PT, min_shared_tokens=B)
     assert plan.groups.tolist() == [[0, 4]]
     assert plan.shared_lens.tolist() == [6 * B] * 4          # the 6 prompt blocks, read once
     assert plan.max_own_len == 20
     # two query rows per sample (G = 8): groups of at most 2
-    plan2 = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=2, min_shared_tokens=B)
+    plan2 = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=2, part_tokens=PT, min_shared_tokens=B)
     assert plan2.groups.tolist() == [[0, 2], [2, 2]]
 
 
@@ -72,11 +88,11 @@ def test_prefix_caching_example():
     # system prompt in blocks 0-3; requests with unique [4,5,6], [7,8,9], [10,11]
     rows = [[0, 1, 2, 3, 4, 5, 6], [0, 1, 2, 3, 7, 8, 9], [0, 1, 2, 3, 10, 11]]
     lens = torch.tensor([7 * B, 7 * B - 3, 6 * B - 1], dtype=torch.int32)
-    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=16, min_shared_tokens=64)
+    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=16, part_tokens=PT, min_shared_tokens=64)
     assert plan.groups.tolist() == [[0, 3]]
     assert plan.shared_lens.tolist() == [64, 64, 64]
     # a threshold above the system prompt: no group
-    none = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=16, min_shared_tokens=65)
+    none = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=16, part_tokens=PT, min_shared_tokens=65)
     assert none.groups.numel() == 0 and none.shared_lens.tolist() == [0, 0, 0]
     assert none.max_own_len == 7 * B
 
@@ -86,7 +102,7 @@ def test_shared_length_stays_below_every_member_length():
     # its last position must stay with its own pass, so x is 2 blocks
     rows = [[5, 6, 7], [5, 6, 7, 8]]
     lens = torch.tensor([3 * B, 3 * B + 4], dtype=torch.int32)
-    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=4, min_shared_tokens=1)
+    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=4, part_tokens=PT, min_shared_tokens=1)
     assert plan.groups.tolist() == [[0, 2]] and plan.shared_lens.tolist() == [2 * B, 2 * B]
     assert plan.max_own_len == B + 4
 
@@ -94,7 +110,7 @@ def test_shared_length_stays_below_every_member_length():
 def test_a_different_first_block_ends_a_run():
     rows = [[1, 2, 3], [1, 2, 9], [4, 2, 3], [4, 2, 3]]
     lens = torch.tensor([3 * B] * 4, dtype=torch.int32)
-    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=8, min_shared_tokens=1)
+    plan = pkv.pkv_shared_prefix_plan(_tables(rows), lens, B, max_group=8, part_tokens=PT, min_shared_tokens=1)
     assert plan.groups.tolist() == [[0, 2], [2, 2]]
     assert plan.shared_lens.tolist() == [2 * B, 2 * B, 2 * B, 2 * B]
 
@@ -128,8 +144,9 @@ def _forked_batch(seed, block_size, n_prompts=6, samples=4):
 def test_plans_of_forked_batches_are_valid(block_size, max_group, min_tokens):
     for seed in range(5):
         tables, lens = _forked_batch(seed * 7 + block_size, block_size)
-        plan = pkv.pkv_shared_prefix_plan(tables, lens, block_size, max_group, min_tokens)
-        _check_valid(tables, lens, plan, max_group, min_tokens, block_size)
+        for pt in (64, 512):
+            plan = pkv.pkv_shared_prefix_plan(tables, lens, block_size, max_group, pt, min_tokens)
+            _check_valid(tables, lens, plan, max_group, min_tokens, block_size)
 
 
 def _best_by_search(tables, lens, max_group, min_tokens):
@@ -183,7 +200,7 @@ def test_greedy_matches_search_on_sampling_batches():
                 lens.append((len(prompt) + len(own) - 1) * B + rng.randint(1, B))
         rows, lens = rows[:9], lens[:9]
         t, cl = _tables(rows), torch.tensor(lens, dtype=torch.int32)
-        plan = pkv.pkv_shared_prefix_plan(t, cl, B, max_group=4, min_shared_tokens=1)
+        plan = pkv.pkv_shared_prefix_plan(t, cl, B, max_group=4, part_tokens=PT, min_shared_tokens=1)
         _check_valid(t, cl, plan, 4, 1)
         saved = sum((n - 1) * plan.shared_lens[f].item() // B for f, n in plan.groups.tolist())
         assert saved == _best_by_search(t, cl, 4, 1), trial
@@ -192,11 +209,29 @@ def test_greedy_matches_search_on_sampling_batches():
 def test_invalid_arguments():
     t = _tables([[0, 1], [0, 1]])
     with pytest.raises(pkv.PagedKVError):
-        pkv.pkv_shared_prefix_plan(t, torch.tensor([0, 5], dtype=torch.int32), B, 4)        # length 0
+        pkv.pkv_shared_prefix_plan(t, torch.tensor([0, 5], dtype=torch.int32), B, 4, PT)        # length 0
     with pytest.raises(pkv.PagedKVError):
-        pkv.pkv_shared_prefix_plan(t, torch.tensor([2 * B + 1, 5], dtype=torch.int32), B, 4)  # past the row
+        pkv.pkv_shared_prefix_plan(t, torch.tensor([2 * B + 1, 5], dtype=torch.int32), B, 4, PT)  # past the row
     with pytest.raises(pkv.PagedKVError):
-        pkv.pkv_shared_prefix_plan(t, torch.tensor([5, 5], dtype=torch.int32), B, 0)        # no room
+        pkv.pkv_shared_prefix_plan(t, torch.tensor([5, 5], dtype=torch.int32), B, 0, PT)        # no room
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pkv_shared_prefix_plan(t, torch.tensor([5, 5], dtype=torch.int32), B, 4, 0)         # no partition size
     empty = pkv.pkv_shared_prefix_plan(torch.empty(0, 4, dtype=torch.int32), torch.empty(0, dtype=torch.int32),
-                                       B, 4)
+                                       B, 4, PT)
     assert empty.groups.numel() == 0 and empty.max_shared_len == 0 and empty.max_own_len == 0
+    assert empty.work.numel() == 0
+
+
+def test_work_list_size_query_and_short_buffer():
+    import ctypes
+    rows = [[0, 1, 2, 3, 4, 5, 6 + 2 * j, 7 + 2 * j] for j in range(4)]
+    t, lens = _tables(rows), torch.tensor([6 * B + 20] * 4, dtype=torch.int32)
+    L = pkv._lib.lib()
+    g, sh = torch.empty(4, 2, dtype=torch.int32), torch.empty(4, dtype=torch.int32)
+    ng, nw, a, b = (ctypes.c_int32(0) for _ in range(4))
+    args = (t.data_ptr(), t.shape[1], lens.data_ptr(), 4, B, 4, B, 32, g.data_ptr(), ctypes.byref(ng), sh.data_ptr())
+    assert L.pkv_shared_prefix_plan(*args, None, 0, ctypes.byref(nw), ctypes.byref(a), ctypes.byref(b)) == 0
+    assert nw.value == 3 + 4                  # 96 shared tokens in 32-token partitions, one own item each
+    w = torch.empty(6, 2, dtype=torch.int32)
+    rc = L.pkv_shared_prefix_plan(*args, w.data_ptr(), 6, ctypes.byref(nw), ctypes.byref(a), ctypes.byref(b))
+    assert rc == pkv._lib.C["PKV_ERR_INVALID_ARG"] and nw.value == 7

@@ -327,6 +327,16 @@ int paged_attention_decode_shared(void* out, const void* q, const void* k_new, c
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pkv_debug_shared_occupancy -- test hook: resident thread blocks per SM of
+ * paged_attention_decode_shared's kernel for this instantiation (fp16 /
+ * bf16), as the CUDA occupancy calculator reports it with the kernel's
+ * shared memory.  Launches nothing.  Returns PKV_ERR_UNSUPPORTED for shapes
+ * the call does not build.
+ */
+int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32_t group, int32_t block_size,
+                               int32_t long_partitions, int32_t* ctas_per_sm);
+
+/*
  * paged_attention_decode_noalloc -- paged_attention_decode without a
  * caller-supplied workspace, for callers that cannot allocate device memory
  * when they decode.  Examples: code that runs while a stream is being

@@ -51,6 +51,7 @@ struct SharedArgs {
     void* ws;
     cudaStream_t stream;
     int* status;
+    int* occupancy_out = nullptr;  // set: report the shared kernel's CTAs per SM, launch nothing
 };
 
 // Record slots per (sequence, query head) row.
@@ -60,22 +61,26 @@ template <typename T, int D, int G, int B>
 int launch_shared(const SharedArgs& a)
 {
     using C = TcCfg<D>;
+    const bool wide = a.part_tokens == kLongPartTokens;
+    const int smem = C::smem_bytes(0);  // neither pass stages new tokens' rows
+    static std::atomic<bool> cfg_n[64] = {}, cfg_w[64] = {};
+    if (a.occupancy_out) {
+        return wide ? occupancy_of(decode_shared_tc_kernel<T, D, G, B, kLongPartTokens>, smem, cfg_w, a.occupancy_out)
+                    : occupancy_of(decode_shared_tc_kernel<T, D, G, B, kPartTokens>, smem, cfg_n, a.occupancy_out);
+    }
     const int slots = shared_record_slots(a.max_ctx, a.part_tokens);
     const int64_t qrows = (int64_t)a.S * a.Hq;
     float* ws_acc = static_cast<float*>(a.ws);
     float* ws_ml = ws_acc + (size_t)qrows * slots * D;
     const float scale_log2 = (float)((double)a.scale * 1.4426950408889634);
-    const bool wide = a.part_tokens == kLongPartTokens;
     const int64_t rows = (int64_t)a.NB * a.Hkv * B;
     if (rows > INT32_MAX) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
     CUtensorMap tm_k, tm_v;
     int rc;
     if ((rc = encode_cache_map<T>(&tm_k, a.k_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
     if ((rc = encode_cache_map<T>(&tm_v, a.v_cache, rows, D, B == 8 ? 8 : 16)) != PKV_OK) return rc;
-    const int smem = C::smem_bytes(0);  // neither pass stages new tokens' rows
 
     // 1. both passes
-    static std::atomic<bool> cfg_n[64] = {}, cfg_w[64] = {};
     auto run = [&](auto kernel, std::atomic<bool>* configured) {
         int r = allow_smem(kernel, smem, configured);
         if (r != PKV_OK) return r;
@@ -202,4 +207,26 @@ extern "C" int paged_attention_decode_shared(void* out, const void* q, const voi
                        status};
     if (dtype == PKV_F16) return shared_d<__half>(head_dim, G, a);
     return shared_d<__nv_bfloat16>(head_dim, G, a);
+}
+
+extern "C" int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32_t group, int32_t block_size,
+                                          int32_t long_partitions, int32_t* ctas_per_sm)
+{
+    if (!ctas_per_sm) return PKV_ERR_INVALID_ARG;
+    if ((block_size != 8 && block_size != 16 && block_size != 32) || (head_dim != 64 && head_dim != 128) ||
+        (group != 1 && group != 2 && group != 4 && group != 8) || (dtype != PKV_F16 && dtype != PKV_BF16))
+        return PKV_ERR_UNSUPPORTED;
+    *ctas_per_sm = 0;
+    SharedArgs a{};
+    a.S = 1;
+    a.max_ctx = long_partitions ? kLongPartTokens : kPartTokens;
+    a.Hq = group;
+    a.Hkv = 1;
+    a.NB = 1;
+    a.block_size = block_size;
+    a.part_tokens = long_partitions ? kLongPartTokens : kPartTokens;
+    a.scale = 1.0f;
+    a.occupancy_out = ctas_per_sm;
+    if (dtype == PKV_F16) return shared_d<__half>(head_dim, group, a);
+    return shared_d<__nv_bfloat16>(head_dim, group, a);
 }

@@ -195,3 +195,22 @@ def test_rejected_calls():
     assert e.value.code == pkv._lib.C["PKV_ERR_UNSUPPORTED"]
     torch.cuda.synchronize()
     assert pkv.pkv_device_status(0) == 0
+
+
+def test_shared_kernel_keeps_three_ctas_per_sm():
+    import ctypes
+    L = pkv._lib.lib()
+    C = pkv._lib.C
+    low = []
+    for dtype in (C["PKV_F16"], C["PKV_BF16"]):
+        for D in (64, 128):
+            for G in (1, 2, 4, 8):
+                for B in (8, 16, 32):
+                    for long_p in (0, 1):
+                        n = ctypes.c_int32(0)
+                        assert L.pkv_debug_shared_occupancy(dtype, D, G, B, long_p, ctypes.byref(n)) == 0
+                        if n.value < 3:
+                            low.append((dtype, D, G, B, long_p, n.value))
+    assert not low, f"below 3 CTAs per SM: {low}"
+    n = ctypes.c_int32(0)
+    assert L.pkv_debug_shared_occupancy(C["PKV_F32"], 128, 4, 16, 0, ctypes.byref(n)) == C["PKV_ERR_UNSUPPORTED"]

@@ -11,11 +11,14 @@ from tests.conftest import ROOT
 pytestmark = pytest.mark.gpu
 
 
-def test_readme_example_runs(cuda_device):
+def test_readme_examples_run(cuda_device):
     with open(os.path.join(ROOT, "README.md")) as f:
-        code = re.search(r"```python\n(.*?)```", f.read(), re.S).group(1)
+        blocks = re.findall(r"```python\n(.*?)```", f.read(), re.S)
+    assert len(blocks) == 2
     scope = {}
-    exec(compile(code, "README.md", "exec"), scope)
+    for i, code in enumerate(blocks):              # the second continues the first
+        exec(compile(code, f"README.md block {i + 1}", "exec"), scope)
     torch.cuda.synchronize()
-    out = scope["out"]
+    out, out4 = scope["out"], scope["out4"]
     assert out.shape == (3, 1, 32, 128) and torch.isfinite(out.float()).all()
+    assert out4.shape == (4, 32, 128) and torch.isfinite(out4.float()).all()

@@ -115,3 +115,39 @@ def test_slot_mapping_matches_the_allocator_model():
         pkv.pkv_slot_mapping(tables, torch.tensor([48, 0, 0], dtype=torch.int32))
     with pytest.raises(pkv.PagedKVError):
         pkv.pkv_slot_mapping(tables, torch.tensor([0, 0, 40], dtype=torch.int32))
+
+
+def test_shared_decode_host_side_rejections(L):
+    """paged_attention_decode_shared's argument checks run before any CUDA call."""
+    from paged_kv_cache_398_b200._lib import C
+    INV, UNS = C["PKV_ERR_INVALID_ARG"], C["PKV_ERR_UNSUPPORTED"]
+    buf = (ctypes.c_uint8 * 8192)()
+    p = ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 256
+    f = ctypes.c_float(0.1)
+
+    def call(S=2, max_ctx=1000, groups=p, ng=1, work=p, nw=3, D=128, B=16, Hq=32, Hkv=8, dtype=2, kn=p, vn=p,
+             ws_bytes=1 << 20):
+        return L.paged_attention_decode_shared(p, p, kn, vn, p, p, p, 64, p, S, max_ctx, groups, ng, p, work, nw,
+                                               512, Hq, Hkv, D, B, 100, f, dtype, p, ws_bytes, None)
+
+    need = L.paged_attention_shared_workspace_bytes(2, 32, 128, 1000)
+    assert need == 2 * 32 * (2 + 1) * 130 * 4      # one record slot per row beyond ceil(1000 / 512)
+    assert call(dtype=C["PKV_F32"]) == UNS          # the tensor-core kernel takes 16-bit inputs
+    assert call(D=96) == UNS and call(B=24) == UNS and call(Hq=24) == UNS
+    assert call(Hq=30) == INV                       # not a multiple of the kv heads
+    assert call(kn=None) == INV                     # k_new without v_new
+    assert call(nw=0) == INV                        # an empty work list
+    assert call(ng=3) == INV                        # more groups than sequences
+    assert call(groups=None) == INV                 # groups missing
+    assert call(work=p + 4) == INV                  # work items are 8-byte pairs
+    assert call(ws_bytes=need - 1) == INV           # workspace too small
+    assert call(S=0) == C["PKV_OK"]                 # an empty batch is a no-op
+    # the plan, on the host: a query of the work list's size
+    t = torch.tensor([[0, 1, 2, 3], [0, 1, 2, 4]], dtype=torch.int32)
+    lens = torch.tensor([60, 61], dtype=torch.int32)
+    g, sh = torch.empty(2, 2, dtype=torch.int32), torch.empty(2, dtype=torch.int32)
+    ng, nw, a, b = (ctypes.c_int32(0) for _ in range(4))
+    assert L.pkv_shared_prefix_plan(t.data_ptr(), 4, lens.data_ptr(), 2, 16, 4, 16, 512, g.data_ptr(),
+                                    ctypes.byref(ng), sh.data_ptr(), None, 0, ctypes.byref(nw), ctypes.byref(a),
+                                    ctypes.byref(b)) == C["PKV_OK"]
+    assert (ng.value, nw.value, a.value, b.value) == (1, 3, 48, 13)

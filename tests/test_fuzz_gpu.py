@@ -82,3 +82,54 @@ def test_random_case_matches_oracle(seed, cuda_device):
     assert np.isfinite(got).all()
     assert not bad.any(), f"case {seed}: {int(bad.sum())} out of tolerance, max abs {err.max():.3e}"
     assert pkv.pkv_device_status(0) == 0
+
+
+def _shared_case(seed):
+    rng = random.Random(10_000 + seed)
+    dtype = rng.choice([torch.float16, torch.bfloat16])
+    D = rng.choice([64, 128])
+    G = rng.choice([1, 2, 4, 8])
+    B = rng.choice([8, 16, 32])
+    Hkv = rng.choice([1, 2, 3])
+    samples = rng.randint(1, 16 // G + 1)          # one more than a group holds, at times: the run splits
+    prompts = rng.randint(1, 4)
+    plo = rng.choice([1, 100, 500])
+    prange = (plo, plo + rng.randint(0, 1600))
+    orange = (1, rng.choice([5, 40, 700]))
+    min_shared = rng.choice([B, 64, 128])
+    return dtype, D, G, B, Hkv, samples, prompts, prange, orange, min_shared
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_shared_prefix_case_matches_oracle(seed, cuda_device):
+    """Shared-prefix decode on random sampling batches: copy-on-write copies,
+    fused slot write, groups that fill or split the 16-row operand, shared
+    lengths on and off partition edges, sequences in no group."""
+    from paged_kv_cache_398_b200.workloads import make_sampling
+    dtype, D, G, B, Hkv, samples, prompts, prange, orange, min_shared = _shared_case(seed)
+    w = make_sampling(prompts, samples, prange, orange, Hkv * G, Hkv, D, dtype, seed=2000 + seed, block_size=B)
+    S = w.num_seqs
+    slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), int(w.context_lens[s]) - 1, B)
+                          for s in range(S)], dtype=torch.int64)
+    k_ref, v_ref = w.k_cache.clone(), w.v_cache.clone()
+    if w.copy_pairs.numel():
+        oracle.block_copy(k_ref, v_ref, w.copy_pairs)
+    oracle.kv_write(k_ref, v_ref, w.k_new, w.v_new, slots)
+    ref = oracle.paged_decode(w.q, k_ref, v_ref, w.block_tables, w.context_lens, w.scale)
+    part = pkv.paged_attention_partition_tokens(S, Hkv, w.max_context_len, dtype)
+    plan = pkv.pkv_shared_prefix_plan(w.block_tables, w.context_lens, B, 16 // G, part, min_shared)
+    g = w.to("cuda")
+    if w.copy_pairs.numel():
+        pkv.block_copy(g.k_cache, g.v_cache, w.copy_pairs)
+    d = plan.to("cuda")
+    out = torch.empty_like(g.q)
+    pkv.paged_attention_decode_shared(out, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale,
+                                      w.max_context_len, d.groups, d.shared_lens, d.work, d.part_tokens,
+                                      k_new=g.k_new, v_new=g.v_new)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(0) == 0
+    assert torch.equal(g.k_cache.cpu(), k_ref) and torch.equal(g.v_cache.cpu(), v_ref)
+    err = np.abs(out.cpu().double().numpy() - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    assert not bad.any(), (f"seed {seed}: {int(bad.sum())} elements out of tolerance, max abs {err.max():.3e}, "
+                           f"groups {plan.groups.tolist()}")

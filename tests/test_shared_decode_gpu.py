@@ -214,3 +214,42 @@ def test_shared_kernel_keeps_three_ctas_per_sm():
     assert not low, f"below 3 CTAs per SM: {low}"
     n = ctypes.c_int32(0)
     assert L.pkv_debug_shared_occupancy(C["PKV_F32"], 128, 4, 16, 0, ctypes.byref(n)) == C["PKV_ERR_UNSUPPORTED"]
+
+
+def test_shared_decode_replays_from_a_cuda_graph():
+    """The shared-prefix step captured once and replayed gives the same bits
+    as eager calls, also after the queries change in place (the plan, the
+    work list and the workspace are device buffers, so nothing is read back
+    or allocated under capture)."""
+    host = make_sampling(6, 4, (300, 1500), (1, 200), 32, 8, 128, torch.bfloat16, seed=41)
+    w = host.to("cuda")
+    plan = make_plan(host).to("cuda")
+    ws = torch.empty(pkv.paged_attention_shared_workspace_bytes(w.num_seqs, w.num_q_heads, w.head_dim,
+                                                                host.max_context_len),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(w.q)
+
+    def step():
+        pkv.paged_attention_decode_shared(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale,
+                                          host.max_context_len, plan.groups, plan.shared_lens, plan.work,
+                                          plan.part_tokens, k_new=w.k_new, v_new=w.v_new, workspace=ws)
+
+    step()                                  # first call on the device: set-up outside capture
+    torch.cuda.synchronize()
+    eager = out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    w.q.copy_(torch.randn(w.q.shape, generator=torch.Generator(device="cuda").manual_seed(3),
+                          device="cuda").to(w.q.dtype))
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = out.clone()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(replayed, out) and not torch.equal(replayed, eager)
+    assert pkv.pkv_device_status(0) == 0

@@ -253,3 +253,25 @@ def test_shared_decode_replays_from_a_cuda_graph():
     torch.cuda.synchronize()
     assert torch.equal(replayed, out) and not torch.equal(replayed, eager)
     assert pkv.pkv_device_status(0) == 0
+
+
+def test_write_then_shared_decode_equals_fused_bitwise():
+    """Without k_new / v_new the call reads new tokens the caller wrote with
+    paged_kv_write; the result is the fused call's, bit for bit."""
+    host = make_sampling(5, 4, (200, 1800), (1, 300), 32, 8, 128, torch.bfloat16, seed=61)
+    plan = make_plan(host)
+    fused = host.to("cuda")
+    out_fused, _ = shared_step(fused, host, plan=plan)
+    sep = host.to("cuda")
+    if sep.copy_pairs.numel():
+        pkv.block_copy(sep.k_cache, sep.v_cache, sep.copy_pairs.cpu())
+    slots = pkv.pkv_slot_mapping(host.block_tables, host.context_lens - 1, host.block_size).cuda()
+    pkv.paged_kv_write(sep.k_new, sep.v_new, sep.k_cache, sep.v_cache, slots)
+    d = plan.to("cuda")
+    out_sep = torch.empty_like(sep.q)
+    pkv.paged_attention_decode_shared(out_sep, sep.q, sep.k_cache, sep.v_cache, sep.block_tables, sep.context_lens,
+                                      sep.scale, sep.max_context_len, d.groups, d.shared_lens, d.work, d.part_tokens)
+    torch.cuda.synchronize()
+    assert torch.equal(out_sep, out_fused)
+    assert torch.equal(sep.k_cache, fused.k_cache) and torch.equal(sep.v_cache, fused.v_cache)
+    assert pkv.pkv_device_status(0) == 0

@@ -235,3 +235,33 @@ def test_work_list_size_query_and_short_buffer():
     w = torch.empty(6, 2, dtype=torch.int32)
     rc = L.pkv_shared_prefix_plan(*args, w.data_ptr(), 6, ctypes.byref(nw), ctypes.byref(a), ctypes.byref(b))
     assert rc == pkv._lib.C["PKV_ERR_INVALID_ARG"] and nw.value == 7
+
+
+def test_plans_of_arbitrary_tables_are_valid():
+    """Property test: any batch of tables and lengths (runs that share random
+    prefixes, invalid ids, lengths anywhere in their rows) gets a plan that
+    satisfies every property the decode relies on."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=200, deadline=None, derandomize=True)
+    @given(st.data())
+    def check(data):
+        bs = data.draw(st.sampled_from([8, 16, 32]))
+        mb = data.draw(st.integers(1, 12))
+        S = data.draw(st.integers(1, 10))
+        rows, base = [], None
+        for _ in range(S):
+            if base is None or data.draw(st.booleans()):
+                base = data.draw(st.lists(st.integers(-1, 40), min_size=mb, max_size=mb))
+            keep = data.draw(st.integers(0, mb))
+            tail = data.draw(st.lists(st.integers(-1, 40), min_size=mb - keep, max_size=mb - keep))
+            rows.append(base[:keep] + tail)
+        t = torch.tensor(rows, dtype=torch.int32)
+        lens = torch.tensor([data.draw(st.integers(1, mb * bs)) for _ in range(S)], dtype=torch.int32)
+        max_group = data.draw(st.integers(1, 16))
+        min_tokens = data.draw(st.sampled_from([0, 1, bs, 64]))
+        pt = data.draw(st.sampled_from([bs, 64, 512]))
+        plan = pkv.pkv_shared_prefix_plan(t, lens, bs, max_group, pt, min_tokens)
+        _check_valid(t, lens, plan, max_group, min_tokens, bs)
+
+    check()

@@ -275,3 +275,14 @@ def test_write_then_shared_decode_equals_fused_bitwise():
     assert torch.equal(out_sep, out_fused)
     assert torch.equal(sep.k_cache, fused.k_cache) and torch.equal(sep.v_cache, fused.v_cache)
     assert pkv.pkv_device_status(0) == 0
+
+
+def test_long_shared_prompt_many_records():
+    """One 40,000-token prompt, 16 samples with one query head per kv head:
+    the group pass covers about 80 partitions, so each row's reduce merges
+    more than 32 records (several passes of its partition loop)."""
+    w = make_sampling(1, 16, (40000, 40000), (1, 600), 2, 2, 64, torch.float16, seed=71, block_size=32)
+    plan = _parity(w, min_shared_tokens=128)
+    assert plan.groups.tolist() == [[0, 16]]
+    assert plan.shared_lens[0].item() == (40000 // 32) * 32
+    assert -(-plan.shared_lens[0].item() // plan.part_tokens) > 32

@@ -1,6 +1,8 @@
-// Tensor-core partition kernel of paged_attention_decode for 16-bit inputs
-// (fp16 / bf16).  Included by decode.cu, which owns the launcher and the
-// split-K reduce kernel.
+// Tensor-core partition kernels of the decode entry points for 16-bit inputs
+// (fp16 / bf16): the body of one partition CTA (partition_tc), the ordinary
+// grid kernel that wraps it, and the shared-prefix kernel that runs it over a
+// work list.  Included by decode.cu and decode_shared.cu, which own the
+// launchers; the split-K reduce is in decode_common.cuh.
 //
 // Per (partition, kv head, sequence) CTA, as in the CUDA-core kernel:
 // 4 warps, each walking its share of the partition's 16-token blocks with

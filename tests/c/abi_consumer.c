@@ -7,10 +7,12 @@
  *                      argument checks that happen before any device work.
  *   abi_consumer gpu   (built with -DWITH_CUDA) one decode step on device 0
  *                      through the C ABI on cudaMalloc'd buffers: block copy,
- *                      slot write, split-K decode.  The result is checked
- *                      against the fp64 oracle library (test infrastructure):
- *                      the cache bit for bit, attention within
- *                      2e-3 + 1e-2 |ref| per element.
+ *                      slot write, split-K decode; then shared-prefix decode
+ *                      of the same step with the forked sample beside its
+ *                      parent.  The results are checked against the fp64
+ *                      oracle library (test infrastructure): the cache bit
+ *                      for bit, attention within 2e-3 + 1e-2 |ref| per
+ *                      element.
  *
  * Exit code 0 when every check passes; otherwise the first failing check is
  * printed and the exit code is 1.
@@ -99,6 +101,25 @@ static int host_checks(void)
     {
         const int64_t bad[2] = {3, 3};  /* a block copied onto itself */
         CHECK(block_copy(NULL, NULL, bad, 1, 2, 128, 16, 8, PKV_BF16, NULL) == PKV_ERR_INVALID_ARG);
+    }
+    {
+        /* shared-prefix plan on the pages' parallel-sampling example: four
+           outputs share prompt blocks 0-5 and own two blocks each */
+        int32_t tabs[4 * 8], lens4[4], groups[8], shared[4], work[2 * 16];
+        int32_t ng = 0, nw = 0, mxs = 0, mxo = 0, j, k;
+        for (j = 0; j < 4; ++j) {
+            for (k = 0; k < 6; ++k) tabs[j * 8 + k] = k;
+            tabs[j * 8 + 6] = 6 + 2 * j;
+            tabs[j * 8 + 7] = 7 + 2 * j;
+            lens4[j] = 6 * 16 + 20;
+        }
+        CHECK(pkv_shared_prefix_plan(tabs, 8, lens4, 4, 16, 4, 16, 512, groups, &ng, shared, work, 16, &nw, &mxs,
+                                     &mxo) == PKV_OK);
+        CHECK(ng == 1 && groups[0] == 0 && groups[1] == 4 && mxs == 96 && mxo == 20);
+        for (j = 0; j < 4; ++j) CHECK(shared[j] == 96);
+        CHECK(nw == 5);                 /* the group's shared partition, then one own partition each */
+        CHECK(work[0] == ~0 && work[1] == 0);
+        CHECK(paged_attention_shared_workspace_bytes(2, 32, 128, 1000) == (size_t)2 * 32 * 3 * 130 * 4);
     }
     CHECK(strcmp(pkv_status_string(PKV_OK), "ok") == 0);
     CHECK(strcmp(pkv_status_string(PKV_ERR_OUT_OF_BLOCKS), "unknown status") != 0);
@@ -237,6 +258,61 @@ static int gpu_checks(void)
     for (e = 0; e < (size_t)S * HQ * D; ++e) {
         const double got = bf16_value(hout[e]);
         CHECK(fabs(got - ref[e]) <= 2e-3 + 1e-2 * fabs(ref[e]));
+    }
+
+    {
+        /* shared-prefix decode of the same step (the new tokens are written),
+           with the fork beside its parent: batch order 0, 3, 1, 2 */
+        const int64_t order2[S] = {0, 3, 1, 2};
+        int32_t tab2[S * MB], len2[S], groups[2 * S], shared[S], work[2 * S * (MB * B / 512 + 1)];
+        int32_t ng = 0, nw = 0, mxs = 0, mxo = 0, part, r;
+        uint16_t* q2 = malloc((size_t)S * HQ * D * 2);
+        void *dq2, *dout2, *dtab2, *dlen2, *dgroups, *dshared, *dwork, *dws2;
+        size_t ws2;
+        CHECK(q2 != NULL);
+        CHECK(pkv_batch_tables(a, order2, S, tab2, MB, -1, len2) == PKV_OK);
+        part = paged_attention_partition_tokens(S, HKV, max_ctx, PKV_BF16);
+        CHECK(part == PKV_PARTITION_TOKENS);
+        CHECK(pkv_shared_prefix_plan(tab2, MB, len2, S, B, PKV_SHARED_MAX_ROWS / (HQ / HKV), 128, part, groups, &ng,
+                                     shared, work, (int32_t)(sizeof(work) / sizeof(work[0]) / 2), &nw, &mxs,
+                                     &mxo) == PKV_OK);
+        CHECK(ng == 1 && groups[0] == 0 && groups[1] == 2 && shared[0] == 688 && shared[2] == 0);
+        for (r = 0; r < S; ++r) memcpy(q2 + (size_t)r * HQ * D, hq + (size_t)order2[r] * HQ * D, (size_t)HQ * D * 2);
+        ws2 = paged_attention_shared_workspace_bytes(S, HQ, D, max_ctx);
+        CUDA_CHECK(cudaMalloc(&dq2, (size_t)S * HQ * D * 2));
+        CUDA_CHECK(cudaMalloc(&dout2, (size_t)S * HQ * D * 2));
+        CUDA_CHECK(cudaMalloc(&dtab2, sizeof(tab2)));
+        CUDA_CHECK(cudaMalloc(&dlen2, sizeof(len2)));
+        CUDA_CHECK(cudaMalloc(&dgroups, sizeof(groups)));
+        CUDA_CHECK(cudaMalloc(&dshared, sizeof(shared)));
+        CUDA_CHECK(cudaMalloc(&dwork, sizeof(work)));
+        CUDA_CHECK(cudaMalloc(&dws2, ws2));
+        CUDA_CHECK(cudaMemcpy(dq2, q2, (size_t)S * HQ * D * 2, cudaMemcpyHostToDevice));
+        CUDA_CHECK(cudaMemcpy(dtab2, tab2, sizeof(tab2), cudaMemcpyHostToDevice));
+        CUDA_CHECK(cudaMemcpy(dlen2, len2, sizeof(len2), cudaMemcpyHostToDevice));
+        CUDA_CHECK(cudaMemcpy(dgroups, groups, sizeof(groups), cudaMemcpyHostToDevice));
+        CUDA_CHECK(cudaMemcpy(dshared, shared, sizeof(shared), cudaMemcpyHostToDevice));
+        CUDA_CHECK(cudaMemcpy(dwork, work, sizeof(work), cudaMemcpyHostToDevice));
+        CHECK(paged_attention_decode_shared(dout2, dq2, NULL, NULL, dk, dv, dtab2, MB, dlen2, S, max_ctx, dgroups, ng,
+                                            dshared, dwork, nw, part, HQ, HKV, D, B, NB,
+                                            (float)(1.0 / sqrt((double)D)), PKV_BF16, dws2, ws2, NULL) == PKV_OK);
+        CUDA_CHECK(cudaDeviceSynchronize());
+        CUDA_CHECK(cudaMemcpy(hout, dout2, (size_t)S * HQ * D * 2, cudaMemcpyDeviceToHost));
+        CHECK(pkv_device_status(0, &flags, 1) == PKV_OK && flags == 0);
+        for (r = 0; r < S; ++r)
+            for (e = 0; e < (size_t)HQ * D; ++e) {
+                const double want = ref[(size_t)order2[r] * HQ * D + e];
+                CHECK(fabs(bf16_value(hout[(size_t)r * HQ * D + e]) - want) <= 2e-3 + 1e-2 * fabs(want));
+            }
+        cudaFree(dq2);
+        cudaFree(dout2);
+        cudaFree(dtab2);
+        cudaFree(dlen2);
+        cudaFree(dgroups);
+        cudaFree(dshared);
+        cudaFree(dwork);
+        cudaFree(dws2);
+        free(q2);
     }
 
     cudaFree(dk);

@@ -62,6 +62,9 @@ extern "C" {
 #define PKV_ERR_DEVICE (-6)        /* a device-side check failed (flags set) */
 #define PKV_ERR_SCRATCH_LIMIT (-7) /* the batch needs more scratch than the
                                       fixed array of the no-alloc variant   */
+#define PKV_ERR_HOST_MEMORY (-8)   /* host memory for the allocator's or the
+                                      plan's own bookkeeping could not be
+                                      allocated; see pkv_alloc_create      */
 
 /* ---- element types ----------------------------------------------------- */
 #define PKV_F32 0
@@ -487,6 +490,13 @@ const char* pkv_status_string(int status);
  *    (src, dst) copy pair.  The last holder (count == 1) writes in place.
  *  - A call that cannot get every block it needs returns
  *    PKV_ERR_OUT_OF_BLOCKS and changes nothing.
+ *  - No C++ exception leaves a call.  If the allocator cannot get host
+ *    memory for its own bookkeeping the call returns PKV_ERR_HOST_MEMORY.
+ *    Creation, adding a sequence, appends, forks, prefix sharing, prompt
+ *    admission and swap-in allocate before they change anything, so such a
+ *    failure leaves the allocator as it was (prompt admission may then cache
+ *    fewer of the prompt's blocks, which only costs later lookups).  After a
+ *    failing free or swap-out, destroy the allocator.
  * Sequence ids are arbitrary int64 values chosen by the caller.
  * One allocator is not thread-safe; use one per thread or lock around it.
  * ======================================================================== */

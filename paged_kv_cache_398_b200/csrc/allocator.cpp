@@ -15,6 +15,7 @@
 #include <algorithm>
 #include <cstring>
 #include <list>
+#include <memory>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -51,6 +52,21 @@ struct BlockKeyHash {
     }
 };
 
+using CacheMap = std::unordered_map<BlockKey, int32_t, BlockKeyHash>;
+
+// Every C entry point that can allocate runs its body through guarded: a
+// failed host allocation becomes PKV_ERR_HOST_MEMORY instead of a C++
+// exception crossing the C ABI.
+template <typename F>
+int guarded(F&& body) noexcept
+{
+    try {
+        return body();
+    } catch (...) {  // std::bad_alloc, or std::length_error for sizes past the address space
+        return PKV_ERR_HOST_MEMORY;
+    }
+}
+
 }  // namespace
 
 struct pkv_allocator {
@@ -60,9 +76,12 @@ struct pkv_allocator {
     std::vector<int32_t> ref;         // reference count per block
     std::unordered_map<int64_t, Seq> seqs;
     int32_t shared = 0;               // blocks with ref > 1
-    // prefix cache: full prompt blocks findable by content
-    std::unordered_map<BlockKey, int32_t, BlockKeyHash> cache;
-    std::vector<BlockKey> key_of;     // per block; toks empty = not cached
+    // prefix cache: full prompt blocks findable by content.  Its buckets are
+    // reserved for every block of the pool at creation, so it never rehashes
+    // and each cached block keeps the iterator of its entry.
+    CacheMap cache;
+    std::vector<CacheMap::iterator> key_it;  // per block, valid while cached[b]
+    std::vector<char> cached;
     std::vector<uint32_t> gen;        // per block; +1 each time it is handed out
     std::list<int32_t> lru;           // cached blocks with ref 0, least recently released first
     std::vector<std::list<int32_t>::iterator> lru_pos;
@@ -80,8 +99,8 @@ struct pkv_allocator {
             b = lru.front();
             lru.pop_front();
             in_lru[b] = 0;
-            cache.erase(key_of[b]);
-            key_of[b].toks.clear();
+            cache.erase(key_it[b]);
+            cached[b] = 0;
             ++evictions;
         }
         ++gen[b];
@@ -101,7 +120,7 @@ struct pkv_allocator {
     {
         if (ref[b]-- == 2) --shared;
         if (ref[b] == 0) {
-            if (!key_of[b].toks.empty()) {  // keep its contents findable until evicted
+            if (cached[b]) {  // keep its contents findable until evicted
                 lru_pos[b] = lru.insert(lru.end(), b);
                 in_lru[b] = 1;
             } else {
@@ -119,7 +138,10 @@ struct pkv_allocator {
         int64_t total = (s.ntok + n + block_size - 1) / block_size;
         return cow + total - (int64_t)s.blocks.size();
     }
-    // caller has checked needs() against the free list
+    // room in s for n more tokens' block ids; the only step of an append that
+    // can fail, so it comes before any change
+    void reserve_for(Seq& s, int64_t n) const { s.blocks.reserve((size_t)((s.ntok + n + block_size - 1) / block_size)); }
+    // caller has checked needs() against the free list and called reserve_for
     void append(Seq& s, int64_t n, int64_t* slots, int64_t* cow_pair, int32_t* cow)
     {
         int32_t did_cow = 0;
@@ -167,32 +189,32 @@ int pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* init
 {
     if (!out || num_blocks < 0 || block_size < 1) return PKV_ERR_INVALID_ARG;
     *out = nullptr;
-    pkv_allocator* a = new (std::nothrow) pkv_allocator();
-    if (!a) return PKV_ERR_INVALID_ARG;
-    a->num_blocks = num_blocks;
-    a->block_size = block_size;
-    a->ref.assign(num_blocks, 0);
-    a->key_of.assign(num_blocks, BlockKey{-1, 0, {}});
-    a->gen.assign(num_blocks, 0);
-    a->lru_pos.resize(num_blocks);
-    a->in_lru.assign(num_blocks, 0);
-    a->free_stack.resize(num_blocks);
-    if (initial_order) {
-        std::vector<char> seen(num_blocks, 0);
-        for (int32_t i = 0; i < num_blocks; ++i) {
-            int32_t b = initial_order[i];
-            if (b < 0 || b >= num_blocks || seen[b]) {
-                delete a;
-                return PKV_ERR_INVALID_ARG;
+    return guarded([&]() -> int {
+        std::unique_ptr<pkv_allocator> a(new pkv_allocator());
+        a->num_blocks = num_blocks;
+        a->block_size = block_size;
+        a->ref.assign(num_blocks, 0);
+        a->cache.reserve((size_t)num_blocks);
+        a->key_it.resize(num_blocks);
+        a->cached.assign(num_blocks, 0);
+        a->gen.assign(num_blocks, 0);
+        a->lru_pos.resize(num_blocks);
+        a->in_lru.assign(num_blocks, 0);
+        a->free_stack.resize(num_blocks);
+        if (initial_order) {
+            std::vector<char> seen(num_blocks, 0);
+            for (int32_t i = 0; i < num_blocks; ++i) {
+                int32_t b = initial_order[i];
+                if (b < 0 || b >= num_blocks || seen[b]) return PKV_ERR_INVALID_ARG;
+                seen[b] = 1;
+                a->free_stack[num_blocks - 1 - i] = b;
             }
-            seen[b] = 1;
-            a->free_stack[num_blocks - 1 - i] = b;
+        } else {
+            for (int32_t i = 0; i < num_blocks; ++i) a->free_stack[num_blocks - 1 - i] = i;
         }
-    } else {
-        for (int32_t i = 0; i < num_blocks; ++i) a->free_stack[num_blocks - 1 - i] = i;
-    }
-    *out = a;
-    return PKV_OK;
+        *out = a.release();
+        return PKV_OK;
+    });
 }
 
 void pkv_alloc_destroy(pkv_allocator* a) { delete a; }
@@ -200,8 +222,10 @@ void pkv_alloc_destroy(pkv_allocator* a) { delete a; }
 int pkv_seq_add(pkv_allocator* a, int64_t seq)
 {
     if (!a || a->find(seq)) return PKV_ERR_INVALID_ARG;
-    a->seqs.emplace(seq, Seq{});
-    return PKV_OK;
+    return guarded([&]() -> int {
+        a->seqs.emplace(seq, Seq{});
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slots_out,
@@ -211,14 +235,18 @@ int pkv_seq_append_tokens(pkv_allocator* a, int64_t seq, int32_t n, int64_t* slo
     Seq* s = a->live(seq);
     if (!s) return PKV_ERR_INVALID_ARG;
     if (a->needs(*s, n) > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
-    a->append(*s, n, slots_out, cow_pair_out, cow_out);
-    return PKV_OK;
+    return guarded([&]() -> int {
+        a->reserve_for(*s, n);
+        a->append(*s, n, slots_out, cow_pair_out, cow_out);
+        return PKV_OK;
+    });
 }
 
 int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
                          int64_t* slots_out, int64_t* cow_pairs_out, int32_t* n_cow_out)
 {
     if (!a || n_seqs < 0 || (n_seqs > 0 && (!seqs || !slots_out))) return PKV_ERR_INVALID_ARG;
+    return guarded([&]() -> int {
     std::vector<Seq*> recs(n_seqs);
     int64_t need = 0;
     for (int32_t i = 0; i < n_seqs; ++i) {
@@ -232,6 +260,7 @@ int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
         if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PKV_ERR_INVALID_ARG;
     }
     if (need > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
+    for (int32_t i = 0; i < n_seqs; ++i) a->reserve_for(*recs[i], 1);  // all-or-nothing: room first
     int32_t ncow = 0;
     for (int32_t i = 0; i < n_seqs; ++i) {
         int64_t pair[2];
@@ -247,6 +276,7 @@ int pkv_batch_append_one(pkv_allocator* a, const int64_t* seqs, int32_t n_seqs,
     }
     if (n_cow_out) *n_cow_out = ncow;
     return PKV_OK;
+    });
 }
 
 int pkv_seq_free(pkv_allocator* a, int64_t seq)
@@ -254,9 +284,11 @@ int pkv_seq_free(pkv_allocator* a, int64_t seq)
     if (!a) return PKV_ERR_INVALID_ARG;
     Seq* s = a->find(seq);
     if (!s) return PKV_ERR_INVALID_ARG;
-    for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
-    a->seqs.erase(seq);
-    return PKV_OK;
+    return guarded([&]() -> int {
+        for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
+        a->seqs.erase(seq);
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_fork(pkv_allocator* a, int64_t parent, int64_t child)
@@ -264,10 +296,12 @@ int pkv_seq_fork(pkv_allocator* a, int64_t parent, int64_t child)
     if (!a) return PKV_ERR_INVALID_ARG;
     const Seq* p = a->live(parent);
     if (!p || a->find(child)) return PKV_ERR_INVALID_ARG;
-    Seq c = *p;
-    for (int32_t b : c.blocks) a->incref(b);
-    a->seqs.emplace(child, std::move(c));
-    return PKV_OK;
+    return guarded([&]() -> int {
+        Seq c = *p;
+        const Seq& added = a->seqs.emplace(child, std::move(c)).first->second;  // the step that can fail
+        for (int32_t b : added.blocks) a->incref(b);
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_share_prefix(pkv_allocator* a, int64_t seq, const int32_t* blocks, int32_t n_blocks,
@@ -280,10 +314,12 @@ int pkv_seq_share_prefix(pkv_allocator* a, int64_t seq, const int32_t* blocks, i
     for (int32_t i = 0; i < n_blocks; ++i) {
         if (blocks[i] < 0 || blocks[i] >= a->num_blocks || a->ref[blocks[i]] < 1) return PKV_ERR_BAD_BLOCK;
     }
-    for (int32_t i = 0; i < n_blocks; ++i) a->incref(blocks[i]);
-    s->blocks.assign(blocks, blocks + n_blocks);
-    s->ntok = n_tokens;
-    return PKV_OK;
+    return guarded([&]() -> int {
+        s->blocks.assign(blocks, blocks + n_blocks);  // the step that can fail
+        for (int32_t i = 0; i < n_blocks; ++i) a->incref(blocks[i]);
+        s->ntok = n_tokens;
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_block_table(const pkv_allocator* a, int64_t seq, int32_t* out, int32_t cap,
@@ -375,46 +411,60 @@ int pkv_seq_append_prompt(pkv_allocator* a, int64_t seq, const int32_t* token_id
     if (!a || n < 0 || (n > 0 && !token_ids)) return PKV_ERR_INVALID_ARG;
     Seq* s = a->live(seq);
     if (!s || !s->blocks.empty() || s->ntok != 0) return PKV_ERR_INVALID_ARG;
-    const int32_t B = a->block_size;
-    const int32_t nfull = n / B;
-    // leading full blocks already cached, walked in order
-    std::vector<int32_t> hit;
-    int32_t parent = -1;
-    uint32_t pgen = 0;
-    int32_t revived = 0;  // hits now resting in the LRU list (not available to others)
-    for (int32_t k = 0; k < nfull; ++k) {
-        BlockKey key{parent, pgen, std::vector<int32_t>(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B)};
-        auto it = a->cache.find(key);
-        if (it == a->cache.end()) break;
-        hit.push_back(it->second);
-        if (a->ref[it->second] == 0) ++revived;
-        parent = it->second;
-        pgen = a->gen[parent];
-    }
-    const int64_t fresh = (int64_t)(n + B - 1) / B - (int64_t)hit.size();
-    if (fresh > a->available() - revived) return PKV_ERR_OUT_OF_BLOCKS;
-    a->lookups += nfull > 0 ? 1 : 0;
-    a->hits += hit.empty() ? 0 : 1;
-    for (int32_t b : hit) {
-        a->incref(b);
-        s->blocks.push_back(b);
-    }
-    const int32_t cached = (int32_t)hit.size() * B;
-    a->hit_tokens += cached;
-    s->ntok = cached;
-    for (int32_t i = 0; i < cached && slots_out; ++i) slots_out[i] = -1;
-    a->append(*s, n - cached, slots_out ? slots_out + cached : nullptr, nullptr, nullptr);
-    // make this prompt's new full blocks findable by the next request
-    for (int32_t k = (int32_t)hit.size(); k < nfull; ++k) {
-        const int32_t b = s->blocks[k];
-        const int32_t par = k == 0 ? -1 : s->blocks[k - 1];
-        BlockKey key{par, par < 0 ? 0u : a->gen[par],
-                     std::vector<int32_t>(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B)};
-        a->key_of[b] = key;
-        a->cache.emplace(std::move(key), b);
-    }
-    if (n_cached_out) *n_cached_out = cached;
-    return PKV_OK;
+    return guarded([&]() -> int {
+        const int32_t B = a->block_size;
+        const int32_t nfull = n / B;
+        // leading full blocks already cached, walked in order with one probe key
+        std::vector<int32_t> hit;
+        hit.reserve((size_t)nfull);
+        BlockKey probe{-1, 0, std::vector<int32_t>((size_t)B)};
+        int32_t revived = 0;  // hits now resting in the LRU list (not available to others)
+        for (int32_t k = 0; k < nfull; ++k) {
+            std::copy(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B, probe.toks.begin());
+            auto it = a->cache.find(probe);
+            if (it == a->cache.end()) break;
+            hit.push_back(it->second);
+            if (a->ref[it->second] == 0) ++revived;
+            probe.parent = it->second;
+            probe.pgen = a->gen[it->second];
+        }
+        const int64_t fresh = (int64_t)(n + B - 1) / B - (int64_t)hit.size();
+        if (fresh > a->available() - revived) return PKV_ERR_OUT_OF_BLOCKS;
+        a->reserve_for(*s, n);
+        a->lookups += nfull > 0 ? 1 : 0;
+        a->hits += hit.empty() ? 0 : 1;
+        for (int32_t b : hit) {
+            a->incref(b);
+            s->blocks.push_back(b);
+        }
+        const int32_t cached = (int32_t)hit.size() * B;
+        a->hit_tokens += cached;
+        s->ntok = cached;
+        for (int32_t i = 0; i < cached && slots_out; ++i) slots_out[i] = -1;
+        a->append(*s, n - cached, slots_out ? slots_out + cached : nullptr, nullptr, nullptr);
+        // make this prompt's new full blocks findable by the next request.  The
+        // first is keyed under the last hit (whose lookup just missed), the rest
+        // under freshly handed-out blocks, so every key is new.  Caching is
+        // best effort: if host memory runs out here, the remaining blocks stay
+        // unfindable (a later miss, never a wrong hit) and the admission stands.
+        try {
+            for (int32_t k = (int32_t)hit.size(); k < nfull; ++k) {
+                const int32_t b = s->blocks[k];
+                const int32_t par = k == 0 ? -1 : s->blocks[k - 1];
+                auto res = a->cache.emplace(
+                    BlockKey{par, par < 0 ? 0u : a->gen[par],
+                             std::vector<int32_t>(token_ids + (int64_t)k * B, token_ids + (int64_t)(k + 1) * B)},
+                    b);
+                if (res.second) {
+                    a->key_it[b] = res.first;
+                    a->cached[b] = 1;
+                }
+            }
+        } catch (...) {
+        }
+        if (n_cached_out) *n_cached_out = cached;
+        return PKV_OK;
+    });
 }
 
 int pkv_prefix_cache_stats(const pkv_allocator* a, pkv_prefix_stats* out)
@@ -438,11 +488,13 @@ int pkv_seq_swap_out(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t
     if (n_out) *n_out = n;
     if (n > cap || (n > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
     if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
-    for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
-    s->blocks.clear();
-    s->swapped = true;
-    s->nswap = n;
-    return PKV_OK;
+    return guarded([&]() -> int {
+        for (auto it = s->blocks.rbegin(); it != s->blocks.rend(); ++it) a->decref(*it);
+        s->blocks.clear();
+        s->swapped = true;
+        s->nswap = n;
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_swap_in(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t cap, int32_t* n_out)
@@ -454,11 +506,14 @@ int pkv_seq_swap_in(pkv_allocator* a, int64_t seq, int32_t* blocks_out, int32_t 
     if (n_out) *n_out = n;
     if (n > cap || (n > 0 && !blocks_out)) return PKV_ERR_INVALID_ARG;
     if (n > a->available()) return PKV_ERR_OUT_OF_BLOCKS;
-    for (int32_t i = 0; i < n; ++i) s->blocks.push_back(a->pop());
-    if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
-    s->swapped = false;
-    s->nswap = 0;
-    return PKV_OK;
+    return guarded([&]() -> int {
+        s->blocks.reserve((size_t)n);  // the step that can fail, before any change
+        for (int32_t i = 0; i < n; ++i) s->blocks.push_back(a->pop());
+        if (n > 0) std::memcpy(blocks_out, s->blocks.data(), sizeof(int32_t) * n);
+        s->swapped = false;
+        s->nswap = 0;
+        return PKV_OK;
+    });
 }
 
 int pkv_seq_is_swapped(const pkv_allocator* a, int64_t seq, int32_t* out)

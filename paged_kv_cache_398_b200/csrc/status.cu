@@ -123,6 +123,7 @@ const char* pkv_status_string(int status)
         case PKV_ERR_BAD_BLOCK: return "bad block id";
         case PKV_ERR_DEVICE: return "device-side check failed";
         case PKV_ERR_SCRATCH_LIMIT: return "batch needs more scratch than the fixed no-alloc array";
+        case PKV_ERR_HOST_MEMORY: return "host memory could not be allocated";
         default: return "unknown status";
     }
 }

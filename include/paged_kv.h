@@ -270,7 +270,8 @@ int paged_attention_decode_mq(void* out, const void* q, const void* k_new, const
  *  max_shared_len_out  max of shared_lens_out (0 if no group)
  *  max_own_len_out  max over sequences of context_lens[s] - shared_lens_out[s]
  * Groups have at least 2 members and never overlap.  The result depends only
- * on the arguments.
+ * on the arguments.  PKV_ERR_HOST_MEMORY if the work list's host scratch
+ * cannot be allocated.
  */
 #define PKV_SHARED_MAX_ROWS 16
 int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -108,7 +108,7 @@ extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_b
     try {
         items.reserve((size_t)num_seqs + (size_t)ng * 4);
     } catch (...) {
-        return PKV_ERR_INVALID_ARG;  // no memory for the list: nothing is written
+        return PKV_ERR_HOST_MEMORY;  // no memory for the list: the outputs are not written
     }
     try {
         for (int32_t g = 0; g < ng; ++g) {
@@ -122,7 +122,7 @@ extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_b
                 items.push_back({std::min(part_tokens, own - p * part_tokens), s, p});
         }
     } catch (...) {
-        return PKV_ERR_INVALID_ARG;
+        return PKV_ERR_HOST_MEMORY;
     }
     std::stable_sort(items.begin(), items.end(), [](const Item& l, const Item& r) { return l.tokens > r.tokens; });
     *num_work_out = (int32_t)items.size();

@@ -63,7 +63,12 @@ extern "C" int block_copy(void* k_cache, void* v_cache, const int64_t* pairs, in
     if (!pkv::aligned16(k_cache) || !pkv::aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
 
     // Reject every list whose result would depend on the copy order.
-    std::vector<uint8_t> role(num_blocks, 0);  // bit0: a src, bit1: a dst
+    std::vector<uint8_t> role;  // bit0: a src, bit1: a dst
+    try {
+        role.assign((size_t)num_blocks, 0);
+    } catch (...) {  // no C++ exception leaves a C call
+        return PKV_ERR_HOST_MEMORY;
+    }
     for (int32_t i = 0; i < num_pairs; ++i) {
         const int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
         if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || s == d) return PKV_ERR_INVALID_ARG;

@@ -77,7 +77,12 @@ int swap_blocks(void* k_cache, void* v_cache, const int64_t* block_ids, int32_t 
     if (!k_cache || !v_cache || !block_ids || !host_k || !host_v) return PKV_ERR_INVALID_ARG;
     if (!pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) || !pkv::aligned16(host_k) || !pkv::aligned16(host_v))
         return PKV_ERR_INVALID_ARG;
-    std::vector<uint8_t> seen(to_host ? 0 : num_blocks, 0);
+    std::vector<uint8_t> seen;
+    try {
+        seen.assign(to_host ? 0 : (size_t)num_blocks, 0);
+    } catch (...) {  // no C++ exception leaves a C call
+        return PKV_ERR_HOST_MEMORY;
+    }
     for (int32_t i = 0; i < n; ++i) {
         const int64_t b = block_ids[i];
         if (b < 0 || b >= num_blocks) return PKV_ERR_INVALID_ARG;

@@ -284,8 +284,9 @@ int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_s
 /*
  * paged_attention_decode_shared -- one decode step (one new token per
  * sequence, optionally fused with its slot write) with a plan from
- * pkv_shared_prefix_plan.  Computes exactly what paged_attention_decode_mq
- * with q_len 1 computes:
+ * pkv_shared_prefix_plan.  Computes the attention paged_attention_decode_mq
+ * with q_len 1 computes, within its tolerance (the bits equal it where no
+ * group forms; a group's shared partitions round differently):
  *
  *   out[s][i][:] = sum_{t < ctx_s} softmax_t(scale * q[s][i] . K_s[t]) * V_s[t]
  *

@@ -108,3 +108,37 @@ def test_multi_query_step_layout():
             pos = int(st.lens_host[s]) - QL + j
             assert int(st.slots[s * QL + j]) == slot_for_position(st.tables_host[s].tolist(), pos, 16)
     assert st.pairs.shape == (0, 2)
+
+
+def test_packed_step_inputs_alias_one_buffer():
+    """The step's inputs live in one packed buffer at 256-byte offsets (one
+    H2D copy per step); a second buffer of the same layout binds the same way
+    (the end-to-end loop alternates two)."""
+    g = torch.Generator().manual_seed(3)
+    S, Hq, Hkv, D, MB = 5, 8, 2, 64, 7
+    st = types.SimpleNamespace(q_len=1, inputs=bench.STEP_INPUTS)
+    st.q = torch.randn(S, Hq, D, generator=g).to(torch.bfloat16)
+    st.k_new = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    st.v_new = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    st.slots = torch.arange(S, dtype=torch.int64) * 3
+    st.block_tables = torch.randint(0, 50, (S, MB), generator=g, dtype=torch.int32)
+    st.context_lens = torch.randint(1, 100, (S,), generator=g, dtype=torch.int32)
+    st.out = torch.empty_like(st.q)
+    orig = {n: getattr(st, n).clone() for n in bench.STEP_INPUTS}
+    bench.pack_step_inputs(st, "cpu")
+    base = st.in_dev.data_ptr()
+    for name in bench.STEP_INPUTS:
+        t = getattr(st, name)
+        assert torch.equal(t, orig[name]) and (t.data_ptr() - base) % 256 == 0
+        assert base <= t.data_ptr() < base + st.in_dev.numel()
+    assert torch.equal(st.in_host, st.in_dev)
+    assert st.q4.shape == (S, 1, Hq, D) and st.k_rows.shape == (S, Hkv, D)
+    # a second buffer with the same layout
+    other = torch.zeros_like(st.in_dev)
+    out2 = torch.empty_like(st.out)
+    b = bench.step_bindings(st, bench.input_views(st, other), out2)
+    other.copy_(st.in_host)
+    for name in bench.STEP_INPUTS:
+        assert torch.equal(b[name], orig[name])
+        assert b[name].data_ptr() - other.data_ptr() == getattr(st, name).data_ptr() - base
+    assert b["out4"].data_ptr() == out2.data_ptr() and b["q4"].data_ptr() == b["q"].data_ptr()

@@ -142,3 +142,17 @@ def test_packed_step_inputs_alias_one_buffer():
         assert torch.equal(b[name], orig[name])
         assert b[name].data_ptr() - other.data_ptr() == getattr(st, name).data_ptr() - base
     assert b["out4"].data_ptr() == out2.data_ptr() and b["q4"].data_ptr() == b["q"].data_ptr()
+
+
+def test_repeated_step_reference_equals_one_step_where_no_source_is_written():
+    """On the prefix workload no new token lands in a block another sequence
+    reads, so the repeated step's reference is the one-step reference."""
+    w = make_workload(4, device="cpu", num_seqs=6, max_ctx=600)
+    seqs = [0, 2, 5]
+    once = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs)
+    again = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs, repeated=True)
+    r1, r2 = [], []
+    bench.oracle_step_timed(once, 2, keep=r1)
+    bench.oracle_step_timed(again, 2, keep=r2)
+    assert np.array_equal(np.stack(r1), np.stack(r2))
+    assert len(again.meta["pre_writes"][0]) == len(seqs)   # only the sampled sequences write into these blocks

@@ -50,3 +50,26 @@ def test_two_gloo_ranks_reduce_like_the_bench():
 def test_single_rank_reduce_is_identity():
     import bench
     assert bench.reduce_over_ranks(None, torch.device("cpu"), [3.0], [4.0, 5.0]) == [3.0, 4.0, 5.0]
+
+
+def test_reference_arm_prints_on_rank_zero_only():
+    """`bench.py --impl reference` under N ranks: rank 0 times the oracle and
+    prints one JSON line; every other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+
+    from tests.conftest import ROOT
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--reference-seqs", "2", "--workload", "2"]
+    outs = {}
+    for rank in (0, 1):
+        env = dict(os.environ, RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE="2")
+        r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stderr
+        outs[rank] = [l for l in r.stdout.splitlines() if l.strip()]
+    assert outs[1] == []
+    assert len(outs[0]) == 1
+    line = json.loads(outs[0][0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"

@@ -8,6 +8,7 @@
 // allocation).  A launch carries up to kPairsPerLaunch pairs; grid.y walks
 // the pairs, grid.z picks the key or the value cache, and each thread moves
 // kUnroll 16-byte chunks with all loads issued before the stores.
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -62,22 +63,28 @@ extern "C" int block_copy(void* k_cache, void* v_cache, const int64_t* pairs, in
     if (!k_cache || !v_cache || !pairs) return PKV_ERR_INVALID_ARG;
     if (!pkv::aligned16(k_cache) || !pkv::aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
 
-    // Reject every list whose result would depend on the copy order.
-    std::vector<uint8_t> role;  // bit0: a src, bit1: a dst
+    // Reject every list whose result would depend on the copy order: a dst
+    // named twice, or a dst that is also a src.  Sorting the ids keeps the
+    // check's cost in the number of pairs, not the size of the pool.
+    std::vector<int64_t> srcs, dsts;
     try {
-        role.assign((size_t)num_blocks, 0);
+        srcs.resize((size_t)num_pairs);
+        dsts.resize((size_t)num_pairs);
     } catch (...) {  // no C++ exception leaves a C call
         return PKV_ERR_HOST_MEMORY;
     }
     for (int32_t i = 0; i < num_pairs; ++i) {
         const int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
         if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks || s == d) return PKV_ERR_INVALID_ARG;
-        if (role[d] & 2) return PKV_ERR_INVALID_ARG;
-        role[s] |= 1;
-        role[d] |= 2;
+        srcs[i] = s;
+        dsts[i] = d;
     }
-    for (int32_t i = 0; i < num_pairs; ++i) {
-        if (role[pairs[2 * i + 1]] & 1) return PKV_ERR_INVALID_ARG;
+    std::sort(srcs.begin(), srcs.end());
+    std::sort(dsts.begin(), dsts.end());
+    if (std::adjacent_find(dsts.begin(), dsts.end()) != dsts.end()) return PKV_ERR_INVALID_ARG;
+    for (size_t i = 0, j = 0; i < dsts.size(); ++i) {  // merge walk: is any dst also a src?
+        while (j < srcs.size() && srcs[j] < dsts[i]) ++j;
+        if (j < srcs.size() && srcs[j] == dsts[i]) return PKV_ERR_INVALID_ARG;
     }
 
     const int64_t block_chunks = (int64_t)(block_bytes / 16);

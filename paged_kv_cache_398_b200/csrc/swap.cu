@@ -12,6 +12,7 @@
 // Block ids are checked on the host and passed by value.  Consecutive
 // threads move consecutive 16-byte chunks of a block, and each thread issues
 // its loads before its stores.
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -77,19 +78,18 @@ int swap_blocks(void* k_cache, void* v_cache, const int64_t* block_ids, int32_t 
     if (!k_cache || !v_cache || !block_ids || !host_k || !host_v) return PKV_ERR_INVALID_ARG;
     if (!pkv::aligned16(k_cache) || !pkv::aligned16(v_cache) || !pkv::aligned16(host_k) || !pkv::aligned16(host_v))
         return PKV_ERR_INVALID_ARG;
-    std::vector<uint8_t> seen;
-    try {
-        seen.assign(to_host ? 0 : (size_t)num_blocks, 0);
-    } catch (...) {  // no C++ exception leaves a C call
-        return PKV_ERR_HOST_MEMORY;
-    }
     for (int32_t i = 0; i < n; ++i) {
-        const int64_t b = block_ids[i];
-        if (b < 0 || b >= num_blocks) return PKV_ERR_INVALID_ARG;
-        if (!to_host) {  // two host slots into one block: order-dependent
-            if (seen[b]) return PKV_ERR_INVALID_ARG;
-            seen[b] = 1;
+        if (block_ids[i] < 0 || block_ids[i] >= num_blocks) return PKV_ERR_INVALID_ARG;
+    }
+    if (!to_host) {  // two host slots into one block: order-dependent.  Sorted, in time of n, not of the pool.
+        std::vector<int64_t> ids;
+        try {
+            ids.assign(block_ids, block_ids + n);
+        } catch (...) {  // no C++ exception leaves a C call
+            return PKV_ERR_HOST_MEMORY;
         }
+        std::sort(ids.begin(), ids.end());
+        if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PKV_ERR_INVALID_ARG;
     }
     void* dk = mapped_device_pointer(host_k);
     void* dv = mapped_device_pointer(host_v);

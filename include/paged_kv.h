@@ -344,11 +344,12 @@ int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32_t group, i
 /*
  * paged_attention_decode_noalloc -- paged_attention_decode without a
  * caller-supplied workspace, for callers that cannot allocate device memory
- * when they decode.  Examples: code that runs while a stream is being
- * captured into a CUDA graph (allocating is not allowed there), runtimes
- * whose device memory is a fixed arena handed out at start-up, and embedders
- * that must never call the CUDA allocator.  It has no counterpart in the
- * pages; it is an interface convenience of this library.
+ * when they decode: runtimes whose device memory is one fixed arena handed
+ * out at start-up (nothing is left to allocate from), and embedders that
+ * must never call the CUDA allocator (cudaMalloc and cudaFree can
+ * synchronise the device and take a process-wide lock, which a latency-
+ * bound decode loop cannot afford).  It has no counterpart in the pages; it
+ * is an interface convenience of this library.
  *
  * The arguments and the result are those of paged_attention_decode.  The
  * split-K scratch comes from one fixed array of PKV_NOALLOC_SCRATCH_BYTES
@@ -357,14 +358,21 @@ int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32_t group, i
  * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
  * routine.
  *
- *  - Limit: if paged_attention_workspace_bytes(num_seqs, num_q_heads,
- *    head_dim, max_context_len) exceeds PKV_NOALLOC_SCRATCH_BYTES, the call
- *    returns PKV_ERR_SCRATCH_LIMIT and enqueues nothing.  Example that fits:
- *    128 sequences x 32 query heads x 8192 tokens at head_dim 128 need 34 MB.
- *  - First call on a device: it resolves the array's device address
- *    (cudaGetSymbolAddress) and sets the decode kernels' shared-memory
- *    limit, once per device, with that device current.  Make that first call
- *    before any stream capture.
+ *  - Errors: a call that paged_attention_decode would reject for any
+ *    workspace gets the same code here.  A valid call whose
+ *    paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim,
+ *    max_context_len) exceeds PKV_NOALLOC_SCRATCH_BYTES returns
+ *    PKV_ERR_SCRATCH_LIMIT and enqueues nothing.  Example that fits: 128
+ *    sequences x 32 query heads x 8192 tokens at head_dim 128 need 34 MB.
+ *  - Set-up: the first call on a device resolves the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and keeps it.  Like
+ *    every decode entry point, the first call of each launch shape (dtype,
+ *    head_dim, query heads per kv head, block size and partition size) also
+ *    sets that kernel's shared-memory limit.  Make those first calls before
+ *    any stream capture.
+ *  - Lifetime: the address is kept for the life of the process, like the
+ *    status word's.  Do not use the library across a cudaDeviceReset (or any
+ *    other destruction of the device's primary context).
  *  - Sharing: all calls on one device share the one array, which keeps the
  *    last call's contents.  Nothing in it needs to start at zero: each call
  *    writes every scratch entry before reading it.  Calls that overlap on

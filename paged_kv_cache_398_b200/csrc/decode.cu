@@ -557,12 +557,14 @@ int dispatch_d(int D, int G, const DecodeArgs& a)
     return PKV_ERR_UNSUPPORTED;
 }
 
-// Host-side checks and dispatch shared by the decode entry points.
-int decode_entry(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                 const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
-                 int32_t num_seqs, int32_t q_len, int32_t max_context_len, int32_t num_q_heads,
-                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
-                 int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
+// Host-side checks of a decode call's shape and pointers (everything but
+// the workspace), shared by the decode entry points.  PKV_OK with
+// num_seqs == 0 means there is nothing to launch.
+int decode_check(const void* out, const void* q, const void* k_new, const void* v_new, const void* k_cache,
+                 const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                 const int32_t* context_lens, int32_t num_seqs, int32_t q_len, int32_t max_context_len,
+                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                 int32_t num_blocks, float scale, int32_t dtype)
 {
     if (pkv::dtype_bytes(dtype) == 0) return PKV_ERR_UNSUPPORTED;
     if (num_seqs < 0 || q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
@@ -581,6 +583,21 @@ int decode_entry(void* out, const void* q, const void* k_new, const void* v_new,
         ((uintptr_t)out % pkv::dtype_bytes(dtype)) || ((uintptr_t)block_tables & 3u) ||
         ((uintptr_t)context_lens & 3u) || (k_new && (!pkv::aligned16(k_new) || !pkv::aligned16(v_new))))
         return PKV_ERR_INVALID_ARG;
+    return PKV_OK;
+}
+
+// Host-side checks and dispatch shared by the decode entry points.
+int decode_entry(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                 const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                 int32_t num_seqs, int32_t q_len, int32_t max_context_len, int32_t num_q_heads,
+                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                 int32_t dtype, void* workspace, size_t workspace_bytes, void* stream)
+{
+    const int checked = decode_check(out, q, k_new, v_new, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                     context_lens, num_seqs, q_len, max_context_len, num_q_heads, num_kv_heads,
+                                     head_dim, block_size, num_blocks, scale, dtype);
+    if (checked != PKV_OK || num_seqs == 0) return checked;
+    const int G = num_q_heads / num_kv_heads;
     const size_t need =
         paged_attention_mq_workspace_bytes(num_seqs, q_len, num_q_heads, head_dim, max_context_len);
     if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
@@ -733,6 +750,11 @@ extern "C" int paged_attention_decode_noalloc(void* out, const void* q, const vo
                                               int32_t num_blocks, float scale, int32_t dtype, void* stream)
 {
     const pkv::NvtxRange nvtx("paged_attention_decode_noalloc");
+    // a call that is invalid for any workspace gets the same code as from paged_attention_decode
+    const int checked = decode_check(out, q, nullptr, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                     context_lens, num_seqs, 1, max_context_len, num_q_heads, num_kv_heads,
+                                     head_dim, block_size, num_blocks, scale, dtype);
+    if (checked != PKV_OK || num_seqs == 0) return checked;
     const size_t need = paged_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len);
     if (need > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;

@@ -1,10 +1,11 @@
 """paged_attention_decode_noalloc: decode without a caller-supplied workspace.
 
-Some callers cannot allocate device memory at the moment they decode: code
-running while a stream is captured into a CUDA graph, runtimes that hand out
-a fixed device arena at start-up, and embedders that must never call the
-CUDA allocator.  For them the library offers an entry point that takes its
-split-K scratch from a fixed array in the library's own device memory.
+Some callers cannot allocate device memory at the moment they decode:
+runtimes that hand out all device memory as one fixed arena at start-up, and
+embedders that must never call the CUDA allocator (it can synchronise the
+device and take a process-wide lock).  For them the library offers an entry
+point that takes its split-K scratch from a fixed array in the library's own
+device memory.
 
 These tests call it through the C ABI (ctypes, raw pointers) and check its
 output against the workspace-taking entry point, within the tolerance the
@@ -97,3 +98,38 @@ def test_noalloc_rejects_batches_beyond_the_limit():
                                           ctypes.c_float(0.1), C["PKV_BF16"], None)
     assert rc == C["PKV_ERR_SCRATCH_LIMIT"]
     assert b"scratch" in L.pkv_status_string(rc)
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    """After a first call of the same shape (which resolves the array's
+    address and sets the kernel's attributes), a call leaves the device's
+    free memory and torch's allocated bytes unchanged."""
+    L = lib()
+    w = make_workload(4, num_seqs=24, device="cuda").to("cuda")
+    need = L.paged_attention_workspace_bytes(w.num_seqs, w.num_q_heads, w.head_dim, w.max_context_len)
+    assert need > 0                                     # the call does use the scratch array
+    out = torch.empty_like(w.q)
+    assert _abi_decode(L, w, out, noalloc=True) == C["PKV_OK"]
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    torch0 = torch.cuda.memory_allocated()
+    for _ in range(3):
+        assert _abi_decode(L, w, out, noalloc=True) == C["PKV_OK"]
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_allocated() == torch0
+
+
+def test_noalloc_invalid_arguments_get_the_workspace_entry_points_code():
+    """A call that is invalid for any workspace returns the same code from
+    both entry points, even when its shape would also exceed the array."""
+    L = lib()
+    dummy = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    p = dummy.data_ptr()
+    S, Hq, ctx = 1024, 64, 8192                         # far beyond the array
+    for D, Hkv, expect in ((96, 8, "PKV_ERR_UNSUPPORTED"),       # unsupported head_dim
+                           (128, 7, "PKV_ERR_INVALID_ARG")):     # Hq not a multiple of Hkv
+        common = [p, p, p, p, p, 512, p, S, ctx, Hq, Hkv, D, 16, 10, ctypes.c_float(0.1), C["PKV_BF16"]]
+        assert L.paged_attention_decode_noalloc(*common, None) == C[expect]
+        assert L.paged_attention_decode(*common, None, 0, None) == C[expect]

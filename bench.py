@@ -40,7 +40,7 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 METRIC = "paged decode attention: effective KV GB/s (% of HBM peak), seq-steps/s"
-WORKLOAD_NAMES = {2: "7b", 3: "13b", 4: "8b_gqa_prefix", 5: "8b_gqa_sampling"}
+WORKLOAD_NAMES = {1: "tiny", 2: "7b", 3: "13b", 4: "8b_gqa_prefix", 5: "8b_gqa_sampling"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -59,9 +59,12 @@ def decode_source_hash() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str, num_seqs: int, path: str, block_size: int):
+def recorded_traffic(workload: str, num_seqs: int, path: str, block_size: int, q_len: int):
     """DRAM bytes per decode call from the committed ncu record, or None if
-    there is none for this workload or the decode sources changed since."""
+    there is none for this step or the decode sources changed since.  The
+    record is captured on a smaller cut of the same recipe that takes the
+    same kernel instantiation, and scaled to the full batch by its
+    algorithmic bytes (its "scaling" key says how)."""
     try:
         with open(TRAFFIC_RECORD) as f:
             rec = json.load(f)
@@ -69,8 +72,8 @@ def recorded_traffic(workload: str, num_seqs: int, path: str, block_size: int):
         return None
     if rec.get("source_sha256") != decode_source_hash():
         return None
-    if (rec.get("workload"), rec.get("num_seqs"), rec.get("path"), rec.get("block_size")) != \
-            (workload, num_seqs, path, block_size):
+    if (rec.get("workload"), rec.get("applies_to_num_seqs"), rec.get("path"), rec.get("block_size"),
+            rec.get("q_len", 1)) != (workload, num_seqs, path, block_size, q_len):
         return None
     return rec.get("dram_bytes_per_call")
 
@@ -202,10 +205,11 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
     e = w.q.element_size()
     ctx = lens.to(torch.int64)
     nblk = (ctx + w.block_size - 1) // w.block_size
-    st.kv_bytes = int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * e
-    uniq_blocks = len(set(tables[tables >= 0].tolist())) if number in (4, 5) else int(nblk.sum())
-    st.kv_unique_bytes = uniq_blocks * w.num_kv_heads * w.block_size * w.head_dim * 2 * e  # upper bound
-    st.decode_bytes = (st.kv_bytes + 2 * S * q_len * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S)
+    per_token = w.num_kv_heads * w.head_dim * 2 * e            # K and V of one position, all kv heads
+    st.kv_bytes = int(ctx.sum()) * per_token                    # logical: every sequence's own context
+    st.kv_unique_bytes = unique_live_tokens(tables, lens, w.block_size) * per_token
+    other = 2 * S * q_len * w.num_q_heads * w.head_dim * e + 4 * int(nblk.sum()) + 4 * S   # Q, out, tables, lens
+    st.decode_bytes = st.kv_bytes + other
     st.write_bytes = 2 * 2 * S * q_len * w.num_kv_heads * w.head_dim * e + 8 * S * q_len
     st.copy_bytes = 2 * 2 * pairs.shape[0] * w.num_kv_heads * w.block_size * w.head_dim * e
     st.part_tokens = pkv.paged_attention_partition_tokens(S, w.num_kv_heads, st.max_ctx, w.dtype)
@@ -221,10 +225,32 @@ def build_step(number: int, device, rank: int = 0, num_seqs=None, block_size: in
         x = st.plan.shared_lens.to(torch.int64)
         first = st.plan.groups[:, 0].to(torch.int64)
         tokens = int(x[first].sum()) + int((ctx - x).sum())
-        st.shared_bytes = (tokens * w.num_kv_heads * w.head_dim * 2 * e + 2 * S * w.num_q_heads * w.head_dim * e
-                           + 4 * int(nblk.sum()) + 4 * S + 4 * S + 8 * first.numel()
-                           + 8 * st.plan.work.shape[0] + st.write_bytes)
+        st.plan_bytes = 4 * S + 8 * first.numel() + 8 * st.plan.work.shape[0]   # shared_lens, groups, work list
+        st.shared_bytes = tokens * per_token + other + st.plan_bytes + st.write_bytes
+    # the decode call's bytes (roofline): the K/V it must read counted once per
+    # physical block's live tokens (unique), or once per sequence (logical)
+    extra = {"fused": st.write_bytes, "shared": st.write_bytes + getattr(st, "plan_bytes", 0), "separate": 0}[path]
+    st.call_bytes_unique = st.kv_unique_bytes + other + extra
+    st.call_bytes_logical = st.kv_bytes + other + extra
     return st
+
+
+def unique_live_tokens(tables, lens, block_size: int) -> int:
+    """Token-exact count of the K/V positions a step must read at least once:
+    each physical block the batch's tables reach counts its live tokens once
+    (the most any sequence holding it uses), however many sequences share it."""
+    lens = lens.to(torch.int64)
+    nblk = (lens + block_size - 1) // block_size
+    mb = tables.shape[1]
+    idx = torch.arange(mb, dtype=torch.int64)
+    live = idx[None, :] < nblk[:, None]                                  # [S, MB] entries in use
+    used = (lens[:, None] - idx[None, :] * block_size).clamp(0, block_size)
+    ids = tables.to(torch.int64)[live]
+    if ids.numel() == 0:
+        return 0
+    per_block = torch.zeros(int(ids.max()) + 1, dtype=torch.int64)
+    per_block.scatter_reduce_(0, ids, used[live], reduce="amax")
+    return int(per_block.sum())
 
 
 STEP_INPUTS = ("q", "k_new", "v_new", "slots", "block_tables", "context_lens")
@@ -396,70 +422,100 @@ def sampled_steps(steps: int, samples: int = 60):
 # clocks
 # ----------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of this GPU, sampled every
+    `period_s` on a host thread through NVML (or, without the Python NVML
+    binding, from `nvidia-smi -lms`, at its coarser period).  summary()
+    covers the samples that fall inside the given wall-clock windows."""
 
-    def __init__(self, device_index: int):
+    REASONS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
+    SMI_FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
         p = torch.cuda.get_device_properties(device_index)
-        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0".upper()
-        self.samples = []
-        self.proc = None
+        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        self.period = period_s
+        self.samples = []          # (monotonic time, sm MHz, power W, reasons bit mask)
+        self.max_mhz = None
+        self.source = None
+        self._stop = threading.Event()
+        self.thread = self.proc = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(self.bus)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h, reasons), daemon=True)
         except Exception:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            try:
+                self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.SMI_FIELDS}",
+                                              "--format=csv,noheader,nounits", "-lms", "20"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                return
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
         self.thread.start()
 
-    def _read(self):
+    def _poll_nvml(self, nvml, h, reasons):
+        while not self._stop.is_set():
+            try:
+                t = time.monotonic()
+                sm = float(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM))
+                pw = nvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = int(reasons(h)) if reasons else 0
+                self.samples.append((t, sm, pw, rs))
+            except Exception:
+                return
+            self._stop.wait(self.period)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 5 or not parts[0].upper().endswith(self.bus[-7:]):   # "BB:DD.F" of this GPU
                 continue
-            if not parts[0].upper().endswith(self.bus[-7:]):   # "BB:DD.F" of this GPU
+            try:
+                self.max_mhz = float(parts[2])
+                self.samples.append((time.monotonic(), float(parts[1]), float(parts[3]), int(parts[4], 16)))
+            except ValueError:
                 continue
-            self.samples.append((time.monotonic(), parts))
 
     def stop(self):
+        self._stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
 
-    def summary(self, t0, t1):
-        win = [p for t, p in self.samples if t0 <= t <= t1]
-        where = "timed region"
+    def summary(self, windows, label: str):
+        """Median SM clock, peak power and every slowdown reason seen in the samples inside `windows`."""
+        win = [x for x in self.samples if any(a <= x[0] <= b for a, b in windows)]
         if not win:
-            win = [p for _, p in self.samples]
-            where = "whole run (no sample fell inside the timed region)"
-        if not win:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(p[1]) for p in win if num(p[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for p in win for n, v in zip(names, p[5:9]) if v.strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": num(win[0][2]), "power_w_max": max((num(p[3]) or 0) for p in win),
-                "reasons": reasons, "samples": len(win), "window": where}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "window": label, "source": self.source or "unavailable"}
+        mask = 0
+        for x in win:
+            mask |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in win), "sm_min_mhz": min(x[1] for x in win),
+                "sm_max_mhz": self.max_mhz, "power_w_max": max(x[2] for x in win),
+                "reasons": [n for n, bit in self.REASONS if mask & bit], "samples": len(win),
+                "period_ms": self.period * 1e3 if self.source == "nvml" else 20.0,
+                "window": label, "source": self.source}
 
 
 # ----------------------------------------------------------------------------
 # the oracle on the host cores
 # ----------------------------------------------------------------------------
-def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False):
+def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False, q=None, k_new=None, v_new=None):
     """The listed sequences' blocks (plus copy sources) copied to the host and
     relabelled 0..n-1, with their tables, as an oracle input.
 
@@ -470,9 +526,15 @@ def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False):
     token into its siblings' blocks.  meta["pre_writes"] then holds the new
     token of every sequence of the batch, sampled or not, whose slot lies in
     these blocks, for oracle_step_timed to apply once (copies + those writes)
-    before the step it times."""
+    before the step it times.
+
+    q / k_new / v_new: the step's own tensors when they are not the
+    workload's (multi-query steps: [S, q_len, heads, D])."""
     from paged_kv_cache_398_b200.workloads import DecodeWorkload
     B = w.block_size
+    q = w.q if q is None else q
+    k_new = w.k_new if k_new is None else k_new
+    v_new = w.v_new if v_new is None else v_new
     need = []
     for s in seqs:
         need += tables[s, :-(-int(lens[s]) // B)].tolist()
@@ -486,7 +548,7 @@ def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False):
     for r, s in enumerate(seqs):
         n = -(-int(lens[s]) // B)
         sbt[r, :n] = torch.tensor([remap[b] for b in tables[s, :n].tolist()], dtype=torch.int32)
-    sel = torch.tensor(seqs, dtype=torch.int64, device=w.q.device)
+    sel = torch.tensor(seqs, dtype=torch.int64, device=q.device)
     meta = {}
     if repeated:
         writers, slots = [], []
@@ -496,41 +558,51 @@ def sub_workload(w, tables, lens, pairs, seqs, repeated: bool = False):
             if b in remap:
                 writers.append(s)
                 slots.append(remap[b] * B + pos % B)
-        wsel = torch.tensor(writers, dtype=torch.int64, device=w.q.device)
-        meta["pre_writes"] = (torch.tensor(slots, dtype=torch.int64), w.k_new[wsel].cpu(), w.v_new[wsel].cpu())
+        wsel = torch.tensor(writers, dtype=torch.int64, device=q.device)
+        meta["pre_writes"] = (torch.tensor(slots, dtype=torch.int64), k_new[wsel].cpu(), v_new[wsel].cpu())
     return DecodeWorkload(
         name=w.name + "-sample", dtype=w.dtype, num_seqs=len(seqs), num_q_heads=w.num_q_heads,
         num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, block_size=B, num_blocks=len(ids),
         context_lens=lens[seqs].contiguous(), block_tables=sbt,
         copy_pairs=torch.tensor([(remap[a], remap[b]) for a, b in sub_pairs], dtype=torch.int64).reshape(-1, 2),
-        q=w.q[sel].cpu(), k_cache=w.k_cache[idx].cpu(), v_cache=w.v_cache[idx].cpu(),
-        k_new=w.k_new[sel].cpu(), v_new=w.v_new[sel].cpu(), scale=w.scale, seed=w.seed, meta=meta)
+        q=q[sel].cpu(), k_cache=w.k_cache[idx].cpu(), v_cache=w.v_cache[idx].cpu(),
+        k_new=k_new[sel].cpu(), v_new=v_new[sel].cpu(), scale=w.scale, seed=w.seed, meta=meta)
 
 
 def oracle_step_timed(sub, threads: int, keep=None):
     """Run the oracle's copy + write + decode on `sub`; returns wall seconds.
-    With `keep` (a list), the fp64 outputs [Hq, D] of the sequences are
-    appended to it."""
+    With `keep` (a list), the fp64 outputs of the sequences ([Hq, D], or
+    [q_len, Hq, D] for a multi-query step) are appended to it."""
     import concurrent.futures as cf
 
     import oracle
     from oracle.allocator_model import slot_for_position
     B = sub.block_size
-    slots = torch.tensor([slot_for_position(sub.block_tables[s].tolist(), int(sub.context_lens[s]) - 1, B)
-                          for s in range(sub.num_seqs)], dtype=torch.int64)
+    mq = sub.q.dim() == 4                      # [n, q_len, Hq, D]: q_len new tokens per sequence
+    ql = sub.q.shape[1] if mq else 1
+    slots = torch.tensor([slot_for_position(sub.block_tables[s].tolist(), int(sub.context_lens[s]) - ql + j, B)
+                          for s in range(sub.num_seqs) for j in range(ql)], dtype=torch.int64)
+    k_rows = sub.k_new.reshape(-1, *sub.k_new.shape[-2:])
+    v_rows = sub.v_new.reshape(-1, *sub.v_new.shape[-2:])
     k, v = sub.k_cache.clone(), sub.v_cache.clone()
     if "pre_writes" in sub.meta:                 # the step's earlier repetition (untimed)
         pre_slots, pre_k, pre_v = sub.meta["pre_writes"]
         if sub.copy_pairs.numel():
             oracle.block_copy(k, v, sub.copy_pairs)
         oracle.kv_write(k, v, pre_k, pre_v, pre_slots)
+
+    def one(s):
+        if mq:
+            return oracle.paged_decode_mq(sub.q[s:s + 1], k, v, sub.block_tables[s:s + 1],
+                                          sub.context_lens[s:s + 1], sub.scale)[0]
+        return oracle.paged_decode_seq(s, sub.q, k, v, sub.block_tables, sub.context_lens, sub.scale)
+
     t0 = time.perf_counter()
     if sub.copy_pairs.numel():
         oracle.block_copy(k, v, sub.copy_pairs)
-    oracle.kv_write(k, v, sub.k_new, sub.v_new, slots)
+    oracle.kv_write(k, v, k_rows, v_rows, slots)
     with cf.ThreadPoolExecutor(max_workers=threads) as ex:
-        outs = list(ex.map(lambda s: oracle.paged_decode_seq(s, sub.q, k, v, sub.block_tables, sub.context_lens,
-                                                             sub.scale), range(sub.num_seqs)))
+        outs = list(ex.map(one, range(sub.num_seqs)))
     t = time.perf_counter() - t0
     if keep is not None:
         keep.extend(outs)
@@ -559,17 +631,28 @@ def pick_sample(lens, work_seconds_target: float, per_token_s: float):
     return seqs
 
 
-def cpu_baseline(st, threads: int):
-    lens, tables, pairs = st.lens_host, st.tables_host, st.pairs
-    probe = sub_workload(st.w, tables, lens, pairs, [0])
+def step_sub_workload(st, seqs, repeated: bool = False):
+    """The oracle input for the listed sequences of a built step (its own Q
+    and new K/V, which may be multi-query)."""
+    return sub_workload(st.w, st.tables_host, st.lens_host, st.pairs, seqs, repeated=repeated,
+                        q=st.q, k_new=st.k_new, v_new=st.v_new)
+
+
+def cpu_baseline(st, threads: int, target_s: float = 30.0):
+    """The oracle on the host cores, on the leading sequences of the step
+    whose single-thread work adds up to about target_s seconds.  Returns its
+    throughput and, under "refs", its fp64 outputs for the parity check."""
+    lens = st.lens_host
+    probe = step_sub_workload(st, [0])
     t1 = oracle_step_timed(probe, 1)
     per_tok = t1 / max(1, int(lens[0]))
-    seqs = pick_sample(lens, 30.0, per_tok)
-    sub = sub_workload(st.w, tables, lens, pairs, seqs, repeated=True)
+    seqs = pick_sample(lens, target_s, per_tok)
+    sub = step_sub_workload(st, seqs, repeated=True)
     refs = []
     t = oracle_step_timed(sub, threads, keep=refs)
     return {"value": sample_kv_bytes(sub) / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": (f"{len(seqs)} of {len(lens)} sequences (all {sub.num_q_heads} query heads): "
+            "sample": (f"{len(seqs)} of {len(lens)} sequences (all {sub.num_q_heads} query heads"
+                       f"{f', {st.q_len} new tokens each' if st.q_len > 1 else ''}): "
                        f"copy + slot write + decode by the fp64 C oracle, {t:.2f} s wall on {threads} threads"),
             "seconds": t, "seqs": seqs, "refs": refs}
 
@@ -584,10 +667,12 @@ def parity_on_sample(st, base, atol: float = 2e-3, rtol: float = 1e-2):
     ref = np.stack(base["refs"])
     err = np.abs(got - ref)
     big = np.abs(ref) > 1e-3
+    shape = " x ".join(str(n) for n in ref.shape[1:])
     return {"max_abs_err": float(err.max()), "max_rel_err": float((err[big] / np.abs(ref[big])).max()),
             "out_of_tolerance": int((err > atol + rtol * np.abs(ref)).sum()), "elements": int(err.size),
             "tolerance": f"|gpu - oracle| <= {atol:g} + {rtol:g} |oracle| per element",
-            "sample": f"{len(base['seqs'])} sequences x {ref.shape[1]} query heads x {ref.shape[2]}"}
+            "sample": f"{len(base['seqs'])} of {st.out.shape[0]} sequences, each {shape} "
+                      f"({'new tokens x ' if ref.ndim == 4 else ''}query heads x head_dim)"}
 
 
 # ----------------------------------------------------------------------------
@@ -705,8 +790,129 @@ def rank_seed(number: int, rank: int) -> int:
     return 398000 + number + 1000 * rank
 
 
+def time_step(st, steps: int, warmup: int, dev, barrier):
+    """`warmup` untimed steps, then `steps` timed ones between a barrier and a
+    device synchronise on both sides (CUDA events around all of them, and
+    around each call of the evenly spread sampled steps), then the
+    end-to-end loop (host inputs in, host output out, every step) for the
+    same number of steps.  Returns the times and the wall-clock windows of
+    the two timed loops (for the clock record)."""
+    for _ in range(warmup):
+        run_step(st)
+    barrier()
+    sampled = sampled_steps(steps)
+    evs = {i: tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for i in sampled}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    w0 = time.monotonic()
+    start.record()
+    for i in range(steps):
+        run_step(st, evs.get(i))
+    end.record()
+    barrier()
+    w1 = time.monotonic()
+    r = {"ms": start.elapsed_time(end),
+         "dec_ms": [ev[2].elapsed_time(ev[3]) for ev in evs.values()],
+         "copy_ms": [ev[0].elapsed_time(ev[1]) for ev in evs.values()] if st.pairs.shape[0] else None,
+         "write_ms": [ev[1].elapsed_time(ev[2]) for ev in evs.values()] if st.path == "separate" else None}
+
+    # ---- end to end: host inputs in, host output out, every step ------------
+    # the step's inputs (q, new K/V, slots, tables, lengths) sit packed in one
+    # pinned host buffer and go over in one copy; the output comes back in one.
+    # The copies of neighbouring steps overlap the kernels (e2e_steps_pipelined).
+    h_out = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
+    r["h2d"] = st.in_host.numel()
+    r["d2h"] = h_out[0].numel() * h_out[0].element_size()
+    e2e_steps_pipelined(st, max(1, warmup), dev, h_out)
+    barrier()
+    w2 = time.monotonic()
+    e0, e1 = e2e_steps_pipelined(st, steps, dev, h_out)
+    barrier()
+    w3 = time.monotonic()
+    r["e2e_ms"] = e0.elapsed_time(e1)
+    r["windows"] = [(w0, w1), (w2, w3)]
+    return r
+
+
+E2E_HOW = ("every step: packed inputs from pinned host memory in one H2D copy, output to pinned host memory in "
+           "one D2H copy; two input and output buffers, copies on their own streams overlapping the "
+           "neighbouring steps' kernels")
+
+ROOFLINE_KERNEL = {"fused": "paged_attention_decode_mq with fused slot write (partition kernel + split-K reduce)",
+                   "shared": "paged_attention_decode_shared with fused slot write "
+                             "(group and own passes in one launch + split-K reduce)",
+                   "separate": "paged_attention_decode (partition kernel + split-K reduce)"}
+
+
+def launches_per_step(st) -> int:
+    return {"fused": st.launches_fused, "separate": st.launches_separate,
+            "shared": getattr(st, "launches_shared", None)}[st.path]
+
+
+def roofline_of(st, dec_mean_ms: float, peak: float, peak_kind: str) -> dict:
+    """The decode call against the HBM roofline.  achieved = the bytes the
+    call must move (each physical block's live K/V tokens once, Q, out,
+    tables, lengths, and the fused new K/V in and out) / its mean duration."""
+    achieved = st.call_bytes_unique / (dec_mean_ms / 1e3) / 1e9
+    logical = st.call_bytes_logical / (dec_mean_ms / 1e3) / 1e9
+    return {"kernel": ROOFLINE_KERNEL[st.path], "bound": "hbm", "achieved": achieved, "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+            "algorithmic_bytes_per_launch": st.call_bytes_unique,
+            "logical_bytes_per_launch": st.call_bytes_logical, "frac_logical": logical / peak,
+            "decode_ms_mean": dec_mean_ms}
+
+
+# The north star's other configurations, measured after the headline in the
+# same run: (key, workload, new tokens per sequence, path, timed steps).
+# q_len 16 on the MHA batches is the multi-query (draft verification) shape.
+ENTRIES = (
+    ("tiny", 1, 1, "separate", 2000),
+    ("7b", 2, 1, "fused", 2000),
+    ("7b_q16", 2, 16, "fused", 1000),
+    ("13b", 3, 1, "fused", 1000),
+    ("13b_q16", 3, 16, "fused", 600),
+    ("8b_gqa_sampling", 5, 1, "shared", 300),
+    ("8b_gqa_sampling_ordinary", 5, 1, "fused", 200),
+)
+
+
+def measure_entry(spec, dev, threads: int, clocks, peak: float, peak_kind: str, barrier, warmup: int = 20,
+                  oracle_s: float = 6.0):
+    key, number, q_len, path, steps = spec
+    st = build_step(number, dev, 0, None, 16, None, q_len, path)
+    st.path = path
+    torch.cuda.synchronize(dev)
+    base = cpu_baseline(st, threads, target_s=oracle_s)   # the oracle's input is taken before any product step
+    r = time_step(st, steps, warmup, dev, barrier)
+    S = st.w.num_seqs
+    dec_mean = statistics.mean(r["dec_ms"])
+    entry = {
+        "workload": WORKLOAD_NAMES[number], "num_seqs": S, "num_q_heads": st.w.num_q_heads,
+        "num_kv_heads": st.w.num_kv_heads, "head_dim": st.w.head_dim, "q_len": q_len, "path": path,
+        "dtype": str(st.w.dtype).replace("torch.", ""), "context_tokens": int(st.lens_host.sum()),
+        "partition_tokens": st.part_tokens, "steps": steps, "warmup": warmup,
+        "value": st.kv_bytes * steps / (r["ms"] / 1e3) / 1e9, "unit": "GB/s",
+        "ms_per_step": r["ms"] / steps,
+        "seq_steps_per_s": S * steps / (r["ms"] / 1e3),
+        "new_tokens_per_s": S * q_len * steps / (r["ms"] / 1e3),
+        "kv_bytes_logical": st.kv_bytes, "kv_bytes_unique": st.kv_unique_bytes,
+        "e2e": {"value": st.kv_bytes * steps / (r["e2e_ms"] / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"] / steps},
+        "roofline": roofline_of(st, dec_mean, peak, peak_kind),
+        "parity": parity_on_sample(st, base),
+        "clocks": clocks.summary(r["windows"], "this entry's timed and end-to-end loops"),
+        "gpu_launches": launches_per_step(st) * steps,
+        "l2": f"{st.kv_unique_bytes / 1e6:.0f} MB of unique K/V per step vs 126 MB of L2, no flush",
+    }
+    if st.plan is not None:
+        entry["shared_prefix"] = {"groups": int(st.plan.groups.shape[0]), "work_items": int(st.plan.work.shape[0])}
+    del st
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args):
-    import paged_kv_cache_398_b200 as pkv
+    import paged_kv_cache_398_b200 as pkv  # noqa: F401  (loads the library before any timing)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -730,47 +936,14 @@ def run_ours(args):
     threads = cpu_threads()
     # the oracle sample is copied off the device before the first product step
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and st.q_len == 1:
-        base = cpu_baseline(st, threads)   # (multi-query parity is covered by the GPU tests)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(st, threads)
 
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
-    for _ in range(args.warmup):
-        run_step(st)
-    barrier()
-
-    sampled = sampled_steps(args.steps)
-    evs = {i: tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for i in sampled}
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    t_wall0 = time.monotonic()
-    start.record()
-    for i in range(args.steps):
-        run_step(st, evs.get(i))
-    end.record()
-    barrier()
-    t_wall1 = time.monotonic()
-    ms = start.elapsed_time(end)
-    dec_ms = [ev[2].elapsed_time(ev[3]) for ev in evs.values()]
-    copy_ms = [ev[0].elapsed_time(ev[1]) for ev in evs.values()] if st.pairs.shape[0] else None
-    write_ms = [ev[1].elapsed_time(ev[2]) for ev in evs.values()] if st.path == "separate" else None
-
-    # ---- end to end: host inputs in, host output out, every step ------------
-    # the step's inputs (q, new K/V, slots, tables, lengths) sit packed in one
-    # pinned host buffer and go over in one copy; the output comes back in one.
-    # The copies of neighbouring steps overlap the kernels (e2e_steps_pipelined).
-    h_out = [torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory() for _ in range(2)]
-    h2d = st.in_host.numel()
-    d2h = h_out[0].numel() * h_out[0].element_size()
-    e2e_steps_pipelined(st, max(1, args.warmup), dev, h_out)
-    e2e_steps = args.steps
-    barrier()
-    e0, e1 = e2e_steps_pipelined(st, e2e_steps, dev, h_out)
-    barrier()
-    t_wall2 = time.monotonic()
-    e2e_ms = e0.elapsed_time(e1)
-    clocks.stop()
+    time.sleep(0.05)
+    r = time_step(st, args.steps, args.warmup, dev, barrier)
+    ms, e2e_ms = r["ms"], r["e2e_ms"]
     swap = measure_swap(st, dev) if not args.no_swap else None
 
     ms_max, e2e_max, kv_total, uniq_total = reduce_over_ranks(
@@ -779,18 +952,21 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
+        clocks.stop()
         return 0
 
     peak, peak_kind = hbm_peak()
+    entries = None
+    if world == 1 and not args.no_workloads:
+        entries = {spec[0]: measure_entry(spec, dev, threads, clocks, peak, peak_kind, barrier)
+                   for spec in ENTRIES}
+    clocks.stop()
+
     S = st.w.num_seqs
     value = kv_total * args.steps / (ms_max / 1e3) / 1e9
-    dec_mean = statistics.mean(dec_ms)
-    # the fused call also moves the new tokens' K/V (read and written once);
-    # the shared-prefix call reads each group's shared blocks once
-    call_bytes = (st.shared_bytes if st.path == "shared" else
-                  st.decode_bytes + (st.write_bytes if st.path == "fused" else 0))
-    achieved = call_bytes / (dec_mean / 1e3) / 1e9
-    clk = clocks.summary(t_wall0, t_wall1)
+    dec_mean = statistics.mean(r["dec_ms"])
+    roof = roofline_of(st, dec_mean, peak, peak_kind)
+    roof["traffic"] = recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path, st.w.block_size, st.q_len)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -808,30 +984,19 @@ def run_ours(args):
         "seq_steps_per_s": S * world * args.steps / (ms_max / 1e3),
         "new_tokens_per_s": S * st.q_len * world * args.steps / (ms_max / 1e3),
         "unique_kv_gbps": uniq_total * args.steps / (ms_max / 1e3) / 1e9,
-        "kernel_ms": {"decode_mean": dec_mean, "decode_min": min(dec_ms),
-                      "kv_write_mean": statistics.mean(write_ms) if write_ms else None,
-                      "block_copy_mean": statistics.mean(copy_ms) if copy_ms else None,
-                      "sampled_steps": len(dec_ms),
+        "kernel_ms": {"decode_mean": dec_mean, "decode_min": min(r["dec_ms"]),
+                      "kv_write_mean": statistics.mean(r["write_ms"]) if r["write_ms"] else None,
+                      "block_copy_mean": statistics.mean(r["copy_ms"]) if r["copy_ms"] else None,
+                      "sampled_steps": len(r["dec_ms"]),
                       "how": "CUDA events around each call on its stream, in evenly spread timed steps"},
-        "roofline": {"kernel": {"fused": "paged_attention_decode_mq with fused slot write "
-                                         "(partition kernel + split-K reduce)",
-                                "shared": "paged_attention_decode_shared with fused slot write "
-                                          "(group and own passes in one launch + split-K reduce)",
-                                "separate": "paged_attention_decode (partition kernel + split-K reduce)"}[st.path],
-                     "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic(WORKLOAD_NAMES[args.workload], S, st.path, st.w.block_size),
-                     "algorithmic_bytes_per_launch": call_bytes},
+        "roofline": roof,
         "cpu_baseline": ({k: v for k, v in base.items() if k in ("value", "unit", "cores", "kind", "sample")}
                          if base else None),
         "parity": parity_on_sample(st, base) if base else None,
-        "e2e": {"value": kv_total * e2e_steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_steps,
-                "how": "every step: packed inputs from pinned host memory in one H2D copy, output to pinned "
-                       "host memory in one D2H copy; two input and output buffers, copies on their own "
-                       "streams overlapping the neighbouring steps' kernels"},
-        "gpu_launches": {"fused": st.launches_fused, "separate": st.launches_separate,
-                         "shared": getattr(st, "launches_shared", None)}[st.path] * args.steps,
+        "e2e": {"value": kv_total * args.steps / (e2e_max / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": e2e_max / args.steps, "how": E2E_HOW},
+        "gpu_launches": launches_per_step(st) * args.steps,
         "path": st.path,
         "host_alloc_us_per_step": st.host_alloc_us,
         "host_alloc_us_per_step_steady": st.host_step_us,
@@ -844,10 +1009,11 @@ def run_ours(args):
                          {"admit_us_per_request": st.admit_us_per_request, "hit_tokens": st.prefix["hit_tokens"],
                           "blocks_shared": st.prefix["hit_tokens"] // st.w.block_size,
                           "cached_blocks": st.prefix["cached_blocks"]}),
-        "clocks": clk,
+        "clocks": clocks.summary(r["windows"], "the timed loop and the end-to-end loop"),
         "swap": swap,
         "fragmentation": fragmentation_report(st.lens_host),
-        "wall_s_timed": t_wall1 - t_wall0,
+        "workloads": entries,
+        "wall_s_timed": r["windows"][0][1] - r["windows"][0][0],
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -862,6 +1028,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-swap", action="store_true", help="skip the swap-out / swap-in measurement")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations (the line's workloads object)")
     ap.add_argument("--block-size", type=int, default=16, choices=[8, 16, 32],
                     help="tokens per block (the pages use 16)")
     ap.add_argument("--path", choices=["fused", "separate", "shared"], default="fused",

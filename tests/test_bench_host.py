@@ -156,3 +156,44 @@ def test_repeated_step_reference_equals_one_step_where_no_source_is_written():
     bench.oracle_step_timed(again, 2, keep=r2)
     assert np.array_equal(np.stack(r1), np.stack(r2))
     assert len(again.meta["pre_writes"][0]) == len(seqs)   # only the sampled sequences write into these blocks
+
+
+def test_unique_live_tokens_counts_each_block_once_token_exact():
+    """Brute force over (sequence, block) on a small sampling batch: shared
+    prompt blocks count once, a partial block counts the most tokens any
+    holder uses, and entries past a sequence's blocks are ignored."""
+    w = make_workload(5, device="cpu", num_prompts=6, max_prompt=300, max_output=40, pad_random=True)
+    B = w.block_size
+    live = {}
+    for s in range(w.num_seqs):
+        n = int(w.context_lens[s])
+        for i in range(-(-n // B)):
+            b = int(w.block_tables[s, i])
+            live[b] = max(live.get(b, 0), min(B, n - i * B))
+    assert bench.unique_live_tokens(w.block_tables, w.context_lens, B) == sum(live.values())
+    # without sharing it is the plain sum of the lengths
+    w2 = make_workload(2, device="cpu", num_seqs=5, max_ctx=200)
+    assert bench.unique_live_tokens(w2.block_tables, w2.context_lens, B) == int(w2.context_lens.sum())
+
+
+def test_multi_query_oracle_sample_equals_the_whole_batch_oracle():
+    """The bench's per-sequence oracle step for q_len new tokens (slot write
+    of all of them, then causal multi-query decode) equals the oracle run
+    on the whole batch at once."""
+    QL = 3
+    w = make_workload(2, device="cpu", num_seqs=4, max_ctx=120, min_ctx=QL)
+    g = torch.Generator().manual_seed(3)
+    S, Hq, Hkv, D = w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim
+    q = torch.randn(S, QL, Hq, D, generator=g).to(w.dtype)
+    kn = torch.randn(S, QL, Hkv, D, generator=g).to(w.dtype)
+    vn = torch.randn(S, QL, Hkv, D, generator=g).to(w.dtype)
+    seqs = [0, 2, 3]
+    sub = bench.sub_workload(w, w.block_tables, w.context_lens, w.copy_pairs, seqs, q=q, k_new=kn, v_new=vn)
+    refs = []
+    bench.oracle_step_timed(sub, 2, keep=refs)
+    k, v = w.k_cache.clone(), w.v_cache.clone()
+    slots = torch.tensor([int(w.block_tables[s, p // 16]) * 16 + p % 16
+                          for s in range(S) for p in range(int(w.context_lens[s]) - QL, int(w.context_lens[s]))])
+    oracle.kv_write(k, v, kn.reshape(-1, Hkv, D), vn.reshape(-1, Hkv, D), slots)
+    full = oracle.paged_decode_mq(q, k, v, w.block_tables, w.context_lens, w.scale)
+    assert np.array_equal(np.stack(refs), full[seqs])

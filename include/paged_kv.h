@@ -110,8 +110,12 @@ int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_
  * PKV_LONG_MIN_PAIRS_PER_SM x the device's multiprocessor count.  Such a
  * batch fills the GPU with (sequence, kv head) pairs alone, and halving its
  * thread-block count saves more fixed per-block cost than the longer
- * blocks add to the tail.  The choice depends only on these launch values,
- * so calls with the same shape always split the same way.
+ * blocks add to the tail.  A multi-query launch of more than 8 query rows
+ * per kv head (q_len * num_q_heads / num_kv_heads > 8, the 16-row form)
+ * always uses PKV_PARTITION_TOKENS_LONG: every partition ends with 16 rows
+ * of output or split-K records, so fewer, longer partitions write and merge
+ * less.  The choice depends only on these launch values, so calls with the
+ * same shape always split the same way.
  */
 #define PKV_PARTITION_TOKENS 512
 #define PKV_PARTITION_TOKENS_LONG 1024
@@ -127,6 +131,18 @@ int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_
  */
 int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,
                                          int32_t dtype);
+
+/*
+ * paged_attention_mq_partition_tokens -- the same for a
+ * paged_attention_decode_mq launch of q_len new tokens per sequence (rule
+ * above; q_len 1 gives paged_attention_partition_tokens).  Returns
+ * PKV_PARTITION_TOKENS, PKV_PARTITION_TOKENS_LONG, or a negative PKV_ERR_*
+ * code: PKV_ERR_INVALID_ARG for a bad shape (num_q_heads not a multiple of
+ * num_kv_heads included), PKV_ERR_CUDA with no CUDA device where the rule
+ * needs the multiprocessor count.
+ */
+int32_t paged_attention_mq_partition_tokens(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                            int32_t num_kv_heads, int32_t max_context_len, int32_t dtype);
 
 /*
  * paged_attention_workspace_bytes -- size of the workspace that
@@ -309,8 +325,13 @@ int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_s
  *                 256-byte aligned (never NULL)
  *  All other arguments are those of paged_attention_decode_mq with q_len 1.
  * The plan is a promise about the tables: the members of a group hold the
- * same blocks for positions [0, x).  The call checks what it can see
- * cheaply: a work item naming a group or sequence outside the batch or a
+ * same blocks for positions [0, x).  A plan made before a table changed (a
+ * copy-on-write repoint, an eviction) breaks it.  The group pass checks it
+ * on the device: each covered member's table entries over the partition's
+ * blocks are compared with the first member's.  A member that differs
+ * raises PKV_DEV_BAD_PLAN and gets no result: the reduce leaves its output
+ * rows unwritten, and the other members' rows are still computed.  The call
+ * also checks: a work item naming a group or sequence outside the batch or a
  * partition past max_context_len, a group with more than
  * PKV_SHARED_MAX_ROWS rows, or one whose x does not fit the cache or
  * max_context_len raises PKV_DEV_BAD_PLAN and is skipped; a member whose own

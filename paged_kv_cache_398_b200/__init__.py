@@ -22,7 +22,8 @@ from .allocator import TABLE_KEEP_TAIL, BlockAllocator, OutOfBlocks
 from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, SHARED_MAX_ROWS, SharedPrefixPlan,
                       block_copy, paged_attention_decode, paged_attention_decode_mq, paged_attention_decode_noalloc,
                       paged_attention_decode_shared, paged_attention_mq_workspace_bytes,
-                      paged_attention_partition_tokens, paged_attention_shared_workspace_bytes,
+                      paged_attention_mq_partition_tokens, paged_attention_partition_tokens,
+                      paged_attention_shared_workspace_bytes,
                       paged_attention_workspace_bytes, paged_kv_write, pkv_device_status, pkv_shared_prefix_plan,
                       pkv_slot_mapping, swap_blocks_in, swap_blocks_out)
 
@@ -31,7 +32,8 @@ __all__ = [
     "LibraryMissing", "OutOfBlocks",
     "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_decode_mq",
     "paged_attention_decode_noalloc", "paged_attention_decode_shared", "paged_attention_mq_workspace_bytes",
-    "paged_attention_partition_tokens", "paged_attention_shared_workspace_bytes", "paged_attention_workspace_bytes",
+    "paged_attention_mq_partition_tokens", "paged_attention_partition_tokens",
+    "paged_attention_shared_workspace_bytes", "paged_attention_workspace_bytes",
     "SHARED_MAX_ROWS", "SharedPrefixPlan", "pkv_shared_prefix_plan",
     "paged_kv_write", "pkv_device_status", "pkv_slot_mapping", "swap_blocks_in", "swap_blocks_out",
 ]

@@ -43,6 +43,7 @@ _SIGS = {
     "paged_kv_write": ([P, P, P, P, P, I32, I32, I32, I32, I32, I32, P], ctypes.c_int),
     "paged_attention_workspace_bytes": ([I32, I32, I32, I32], SZ),
     "paged_attention_partition_tokens": ([I32, I32, I32, I32], I32),
+    "paged_attention_mq_partition_tokens": ([I32, I32, I32, I32, I32, I32], I32),
     "pkv_debug_decode_occupancy": ([I32, I32, I32, I32, I32, I32, P], I32),
     "pkv_debug_shared_occupancy": ([I32, I32, I32, I32, I32, P], I32),
     "paged_attention_decode": ([P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32, I32,

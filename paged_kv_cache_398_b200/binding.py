@@ -86,6 +86,18 @@ def paged_attention_partition_tokens(num_seqs: int, num_kv_heads: int, max_conte
     return rc
 
 
+def paged_attention_mq_partition_tokens(num_seqs: int, q_len: int, num_q_heads: int, num_kv_heads: int,
+                                        max_context_len: int, dtype: torch.dtype) -> int:
+    """Split-K partition size (tokens) of a paged_attention_decode_mq launch
+    of q_len new tokens per sequence: PARTITION_TOKENS or PARTITION_TOKENS_LONG."""
+    if dtype not in _DTYPE:
+        raise PagedKVError("dtype", C["PKV_ERR_UNSUPPORTED"])
+    rc = int(lib().paged_attention_mq_partition_tokens(num_seqs, q_len, num_q_heads, num_kv_heads,
+                                                       max_context_len, _DTYPE[dtype]))
+    check("paged_attention_mq_partition_tokens", min(rc, 0))
+    return rc
+
+
 def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
                            max_context_len: int, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> torch.Tensor:

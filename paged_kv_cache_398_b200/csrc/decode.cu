@@ -8,7 +8,8 @@
 // Design (B200, sm_100a):
 //  * Work unit = (partition p, kv head h, sequence s): one CTA.  A partition
 //    is PKV_PARTITION_TOKENS tokens, or PKV_PARTITION_TOKENS_LONG on large
-//    batches of long contexts (part_tokens_for).  The G = Hq / Hkv query
+//    batches of long contexts and on launches of more than 8 query rows per
+//    kv head (mq_part_tokens_for).  The G = Hq / Hkv query
 //    heads that share kv head h are computed together, so each K/V block is
 //    read from HBM once per kv head, not once per query head.
 //  * fp16 / bf16 run the tensor-core kernel of decode_tc.cuh (tiled TMA,
@@ -430,7 +431,7 @@ struct DecodeArgs {
     int32_t Hkv;
     int32_t NB;
     int32_t block_size;
-    int32_t part_tokens;  // kPartTokens or kLongPartTokens (part_tokens_for)
+    int32_t part_tokens;  // kPartTokens or kLongPartTokens (mq_part_tokens_for)
     float scale;
     void* ws;
     cudaStream_t stream;
@@ -605,7 +606,7 @@ int decode_entry(void* out, const void* q, const void* k_new, const void* v_new,
     int* status = pkv::status_word_for_current_device();
     if (!status) return PKV_ERR_CUDA;
     int part_tokens = kPartTokens;
-    const int rc = part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, &part_tokens);
+    const int rc = mq_part_tokens_for(dtype, num_seqs, q_len * G, num_kv_heads, max_context_len, &part_tokens);
     if (rc != PKV_OK) return rc;
     const DecodeArgs a{out,           q,        k_new,          v_new,        k_cache,      v_cache,
                        block_tables,  max_blocks_per_seq,       context_lens, num_seqs,     q_len,
@@ -627,6 +628,19 @@ extern "C" size_t paged_attention_mq_workspace_bytes(int32_t num_seqs, int32_t q
     const size_t parts = ((size_t)max_context_len + kPartTokens - 1) / kPartTokens;
     if (parts <= 1) return 0;
     return (size_t)num_seqs * q_len * num_q_heads * parts * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+extern "C" int32_t paged_attention_mq_partition_tokens(int32_t num_seqs, int32_t q_len, int32_t num_q_heads,
+                                                       int32_t num_kv_heads, int32_t max_context_len, int32_t dtype)
+{
+    if (num_seqs < 0 || q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+        max_context_len < 1)
+        return PKV_ERR_INVALID_ARG;
+    if (dtype != PKV_F32 && dtype != PKV_F16 && dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+    int part_tokens = kPartTokens;
+    const int rc = mq_part_tokens_for(dtype, num_seqs, q_len * (num_q_heads / num_kv_heads), num_kv_heads,
+                                      max_context_len, &part_tokens);
+    return rc != PKV_OK ? rc : part_tokens;
 }
 
 extern "C" int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,

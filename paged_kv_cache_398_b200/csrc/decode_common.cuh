@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(128)
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         M = fmaxf(M, m);
     }
+    // a poison record (m = +inf, written by the shared-prefix group pass for
+    // a member whose table broke the plan's promise): leave the row unwritten
+    if (M == INFINITY) return;
     float L = 0.0f;
     float o[kPer];
 #pragma unroll
@@ -312,6 +315,18 @@ int part_tokens_for(int32_t dtype, int32_t num_seqs, int32_t num_kv_heads, int32
     if (rc != PKV_OK) return rc;
     if ((int64_t)num_seqs * num_kv_heads >= (int64_t)PKV_LONG_MIN_PAIRS_PER_SM * sms) *out = kLongPartTokens;
     return PKV_OK;
+}
+
+// The same for a launch of `rows` query rows per kv head (q_len x G): more
+// than 8 (the 16-row form) always takes the long partitions.
+inline int mq_part_tokens_for(int32_t dtype, int32_t num_seqs, int32_t rows, int32_t num_kv_heads,
+                              int32_t max_context_len, int* out)
+{
+    if (dtype != PKV_F32 && rows > 8) {
+        *out = kLongPartTokens;
+        return PKV_OK;
+    }
+    return part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, out);
 }
 
 }  // namespace

@@ -436,8 +436,12 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
         pkv::fence_mbar_init();
     }
     if constexpr (kPlan == kPlanGroup) {
-        // the group pass stages nothing: the staging barrier's word carries the cover bits
-        if (threadIdx.x == 0) *reinterpret_cast<volatile uint32_t*>(new_bar) = cover;
+        // the group pass stages nothing: the staging barrier's two words carry
+        // the cover bits and the members whose tables disagree with the leader's
+        if (threadIdx.x == 0) {
+            reinterpret_cast<volatile uint32_t*>(new_bar)[0] = cover;
+            reinterpret_cast<volatile uint32_t*>(new_bar)[1] = 0u;
+        }
         __syncthreads();
         cover = *reinterpret_cast<volatile uint32_t*>(new_bar);
     } else {
@@ -489,6 +493,27 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
             qa[ks][3] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
     }
+    if constexpr (kPlan == kPlanGroup) {
+        // The plan promises that every covered member's table holds the
+        // leader's block ids over [0, x); a plan made before a table changed
+        // (a copy-on-write repoint, an eviction) breaks that.  Check this
+        // partition's slice of each member against the leader's (s_blk).
+        // The loads go out after the first tile copies, so their latency
+        // hides behind those.  A member that differs is marked; the merge
+        // then gives it a poison record instead of its split-K record.
+        uint32_t bad = 0u;
+        const int checks = (nq - 1) * nbp;  // members 1..nq-1; blk0 + nbp <= ceil(x / B) <= mb
+        for (int idx = threadIdx.x; idx < checks; idx += kWarps * 32) {
+            const int j = 1 + idx / nbp, i = idx % nbp;
+            if ((cover >> j) & 1u) {
+                const int32_t b = pkv::ld_early(block_tables + (int64_t)(s + j) * mb + blk0 + i);
+                if (b != s_blk[i]) bad |= 1u << j;
+            }
+        }
+        bad = __reduce_or_sync(0xffffffffu, bad);
+        if (lane == 0 && bad != 0u) atomicOr(reinterpret_cast<uint32_t*>(new_bar) + 1, bad);
+    }
+
     // Multi-query: positions row ra (rb) may see are < lim_a (lim_b); a row
     // holding no query sees nothing.  (A single query sees the whole context,
     // so that path masks against ctx alone.)
@@ -846,8 +871,23 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
         slot = (x_own + part_tokens - 1) / part_tokens + p;
         nparts = split_parts(x_own, ctx, part_tokens);
     }
+    uint32_t mismatch = 0u;  // group pass: members whose tables differ from the leader's
+    if constexpr (kPlan == kPlanGroup) {
+        mismatch = reinterpret_cast<volatile uint32_t*>(new_bar)[1];
+        if (threadIdx.x == 0 && mismatch != 0u) pkv::raise_flag(status, PKV_DEV_BAD_PLAN);
+    }
     for (int r = warp; r < rows; r += kWarps) {
         if (kPlan == kPlanGroup && !((cover >> (r / G)) & 1u)) continue;  // a member computed elsewhere
+        if (kPlan == kPlanGroup && ((mismatch >> (r / G)) & 1u)) {
+            // poison record (m = +inf, which no score produces): the reduce
+            // leaves this member's output row unwritten
+            if (lane == 0) {
+                const int64_t orow = ((int64_t)row0 + r / G) * num_q_heads + h * G + r % G;
+                ws_ml[(orow * max_parts + slot) * 2] = INFINITY;
+                ws_ml[(orow * max_parts + slot) * 2 + 1] = 0.0f;
+            }
+            continue;
+        }
         float mw[kWarps];
         float M = -INFINITY;
 #pragma unroll

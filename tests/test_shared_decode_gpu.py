@@ -171,6 +171,39 @@ def test_inconsistent_plans_are_flagged_and_stay_in_bounds():
     _parity(w)
 
 
+def test_stale_plan_member_table_is_flagged_and_its_row_left_unwritten():
+    """A plan made before one member's table changed inside the shared range
+    (a copy-on-write repoint after planning): the group pass finds the
+    member's block id differing from the leader's, raises PKV_DEV_BAD_PLAN
+    and the member's output row is never written; every other row is the
+    oracle's attention.  ("Copy-on-Write: Sharing KV Cache": a shared block
+    is copied before it diverges, so a table can change under a plan.)"""
+    import dataclasses
+    w = make_sampling(3, 4, (300, 600), (1, 100), 32, 8, 128, torch.bfloat16, seed=23)
+    plan = make_plan(w)
+    assert plan.groups.shape[0] == 3
+    first, n = plan.groups[1].tolist()
+    member = first + 2
+    assert n == 4 and int(plan.shared_lens[member]) >= 6 * w.block_size
+    used = set(w.block_tables[w.block_tables >= 0].tolist()) | set(w.copy_pairs.flatten().tolist())
+    spare = next(b for b in range(w.num_blocks) if b not in used)
+    bt = w.block_tables.clone()
+    bt[member, 5] = spare                        # block 5 of the shared range, repointed after planning
+    moved = dataclasses.replace(w, block_tables=bt)
+    g = moved.to("cuda")
+    out = torch.full_like(g.q, float("nan"))
+    shared_step(g, moved, plan=plan, out=out)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(0) & BAD_PLAN
+    assert torch.isnan(out[member].float()).all()
+    ref, _, _ = oracle_step(moved, oracle_slots(moved))
+    others = [s for s in range(w.num_seqs) if s != member]
+    assert_close(out[torch.tensor(others, device="cuda")], ref[others], "rows of the other sequences")
+    # the same batch with a fresh plan: every row, the moved member included
+    pkv.pkv_device_status(0, clear=True)
+    _parity(moved)
+
+
 def test_rejected_calls():
     w = make_sampling(2, 4, (300, 400), (1, 50), 32, 8, 128, torch.bfloat16, seed=31).to("cuda")
     host = make_sampling(2, 4, (300, 400), (1, 50), 32, 8, 128, torch.bfloat16, seed=31)

@@ -81,6 +81,17 @@ def test_host_side_rejections(L):
     assert L.paged_attention_partition_tokens(-1, 8, 100, C["PKV_BF16"]) == INV
     assert L.paged_attention_partition_tokens(4, 0, 100, C["PKV_BF16"]) == INV
     assert L.paged_attention_partition_tokens(4, 8, 100, 7) == UNS
+    # multi-query: more than 8 query rows per kv head (the 16-row form) always take the long partitions
+    MQ = L.paged_attention_mq_partition_tokens
+    assert MQ(64, 16, 40, 40, 600, C["PKV_F16"]) == C["PKV_PARTITION_TOKENS_LONG"]      # 16 rows
+    assert MQ(8, 3, 16, 4, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS_LONG"]        # 3 x 4 = 12 rows
+    assert MQ(8, 2, 16, 4, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS"]             # 8 rows: the short rule
+    assert MQ(8, 1, 32, 8, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS"]
+    assert MQ(8, 16, 16, 16, 9000, C["PKV_F32"]) == C["PKV_PARTITION_TOKENS"]           # fp32 keeps the short ones
+    assert MQ(8, 16, 40, 7, 100, C["PKV_F16"]) == INV                                  # Hq not a multiple of Hkv
+    assert MQ(8, 0, 40, 40, 100, C["PKV_F16"]) == INV
+    assert MQ(8, 16, 40, 40, 0, C["PKV_F16"]) == INV
+    assert MQ(8, 16, 40, 40, 100, 7) == UNS
     # order-dependent copy lists are rejected on the host
     dummy = ctypes.c_void_p(p)
     for pairs in ([[1, 1]], [[1, 2], [3, 2]], [[1, 2], [2, 3]], [[0, 8]], [[-1, 2]]):

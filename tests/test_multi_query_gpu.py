@@ -77,7 +77,7 @@ def _both_paths(w, q_len):
     return (out_a, a.k_cache, a.v_cache), (out_b, b.k_cache, b.v_cache)
 
 
-MQ_LENS = [4, 15, 16, 17, 18, 33, 511, 512, 513, 514, 1024, 1026, 4099]
+MQ_LENS = [4, 15, 16, 17, 18, 33, 511, 512, 513, 514, 1024, 1026, 2049, 4099]
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])

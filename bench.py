@@ -390,6 +390,14 @@ def run_step(st, ev=None):
         pkv.paged_kv_write(st.k_rows, st.v_rows, st.k_cache, st.v_cache, st.slots)
     if ev is not None:
         ev[2].record()
+    run_decode(st)
+    if ev is not None:
+        ev[3].record()
+
+
+def run_decode(st):
+    """The step's decode call alone (the call run_step makes after its copies and write)."""
+    import paged_kv_cache_398_b200 as pkv
     if st.path == "separate" and st.q_len == 1:
         pkv.paged_attention_decode(st.out, st.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                    st.w.scale, st.max_ctx, workspace=st.workspace)
@@ -405,8 +413,6 @@ def run_step(st, ev=None):
         pkv.paged_attention_decode_mq(st.out4, st.q4, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                                       st.w.scale, st.max_ctx, k_new=st.k_new4, v_new=st.v_new4,
                                       workspace=st.workspace)
-    if ev is not None:
-        ev[3].record()
 
 
 def sampled_steps(steps: int, samples: int = 60):
@@ -815,7 +821,22 @@ def time_step(st, steps: int, warmup: int, dev, barrier):
     r = {"ms": start.elapsed_time(end),
          "dec_ms": [ev[2].elapsed_time(ev[3]) for ev in evs.values()],
          "copy_ms": [ev[0].elapsed_time(ev[1]) for ev in evs.values()] if st.pairs.shape[0] else None,
-         "write_ms": [ev[1].elapsed_time(ev[2]) for ev in evs.values()] if st.path == "separate" else None}
+         "write_ms": [ev[1].elapsed_time(ev[2]) for ev in evs.values()] if st.path == "separate" else None,
+         "decode_loop_ms": None}
+    if not decode_only_step(st):
+        # the roofline's duration: the decode call alone, timed over a loop of
+        # its own (repeating it reads what the step reads; the cache is as the
+        # timed steps left it)
+        for _ in range(warmup):
+            run_decode(st)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            run_decode(st)
+        b.record()
+        barrier()
+        r["decode_loop_ms"] = a.elapsed_time(b)
 
     # ---- end to end: host inputs in, host output out, every step ------------
     # the step's inputs (q, new K/V, slots, tables, lengths) sit packed in one
@@ -850,16 +871,19 @@ def launches_per_step(st) -> int:
             "shared": getattr(st, "launches_shared", None)}[st.path]
 
 
+def decode_only_step(st) -> bool:
+    """Whether a step is the decode call alone (no copy-on-write pairs, write fused)."""
+    return st.path in ("fused", "shared") and st.pairs.shape[0] == 0
+
+
 def decode_call_ms(st, r, steps: int):
-    """Mean duration of the step's decode call, and how it was measured.  A
-    step that is the decode call alone (no copy-on-write pairs, write fused)
-    gives it as the timed loop's event time / steps.  Otherwise it is the
-    mean over the sampled steps' events around the call, which costs the
-    call its programmatic early launch and so reads a few us long."""
-    if st.path in ("fused", "shared") and st.pairs.shape[0] == 0:
+    """Mean duration of the step's decode call, and how it was measured: the
+    timed loop's CUDA-event time / steps when the step is the call alone, else
+    the same over a loop of the decode call alone run right after it."""
+    if decode_only_step(st):
         return r["ms"] / steps, "CUDA events around the timed loop / steps (the step is the decode call alone)"
-    return (statistics.mean(r["dec_ms"]),
-            f"CUDA events around the call in {len(r['dec_ms'])} evenly spread timed steps")
+    return (r["decode_loop_ms"] / steps,
+            "CUDA events around a loop of the decode call alone (same steps), after the timed loop")
 
 
 def roofline_of(st, dec_mean_ms: float, peak: float, peak_kind: str, how: str = "") -> dict:

@@ -30,7 +30,7 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _cuda(name: str, t: torch.Tensor, dtype=None, ndim=None) -> torch.Tensor:
-    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
@@ -41,9 +41,17 @@ def _cuda(name: str, t: torch.Tensor, dtype=None, ndim=None) -> torch.Tensor:
     return t
 
 
-def _stream(device: torch.device, stream) -> ctypes.c_void_p:
-    s = torch.cuda.current_stream(device) if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+# torch's current stream as a raw handle, without building a Stream object
+# (about 3 us a call otherwise); the public call where torch lacks it.
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(device: torch.device, stream) -> int:
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_current_stream is not None:
+        return _raw_current_stream(device.index if device.index is not None else torch.cuda.current_device())
+    return torch.cuda.current_stream(device).cuda_stream
 
 
 def _cache_shape(k_cache, v_cache):
@@ -119,9 +127,10 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         raise ValueError("q/out must be [S, Hq, D] with the cache's head_dim")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables/context_lens must have one row per sequence")
-    need = paged_attention_workspace_bytes(S, Hq, D, max_context_len)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:   # a given workspace's size is checked by the library
+        need = paged_attention_workspace_bytes(S, Hq, D, max_context_len)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr, ws_bytes = 0, 0
     if workspace is not None:
         _cuda("workspace", workspace)
@@ -168,9 +177,10 @@ def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, context_le
         if tuple(k_new.shape) != (S, QL, Hkv, D) or tuple(v_new.shape) != (S, QL, Hkv, D):
             raise ValueError("k_new/v_new must be [S, q_len, Hkv, D]")
         kn, vn = k_new.data_ptr(), v_new.data_ptr()
-    need = paged_attention_mq_workspace_bytes(S, QL, Hq, D, max_context_len)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None:   # a given workspace's size is checked by the library
+        need = paged_attention_mq_workspace_bytes(S, QL, Hq, D, max_context_len)
+        if need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr, ws_bytes = 0, 0
     if workspace is not None:
         _cuda("workspace", workspace)

@@ -165,6 +165,53 @@ def test_workload_parity_full_size_sampled(number):
     assert pkv.pkv_device_status(0) == 0
 
 
+@pytest.mark.parametrize("number", [2, 3])
+def test_workload_16_new_tokens_full_size_sampled(number):
+    """The 7B and 13B batches at full size with 16 new tokens per sequence
+    (the multi-query step of the bench's q_len 16 entries): one fused call
+    writes every new token's K/V and attends causally.  The cache update is
+    checked everywhere, the attention on sampled sequences (the longest among
+    them) against the oracle.  Such launches take the long partitions."""
+    import dataclasses
+    from paged_kv_cache_398_b200.workloads import _randn
+    QL = 16
+    base = make_workload(number, device="cuda", min_ctx=QL)
+    S, Hq, Hkv, D = base.num_seqs, base.num_q_heads, base.num_kv_heads, base.head_dim
+    gd = torch.Generator(device="cuda").manual_seed(70 + number)
+    host = dataclasses.replace(base, q=_randn((S, QL, Hq, D), base.dtype, gd, "cuda"),
+                               k_new=_randn((S, QL, Hkv, D), base.dtype, gd, "cuda"),
+                               v_new=_randn((S, QL, Hkv, D), base.dtype, gd, "cuda"))
+    assert pkv.paged_attention_mq_partition_tokens(S, QL, Hq, Hkv, host.max_context_len, host.dtype) == \
+        pkv.PARTITION_TOKENS_LONG
+    w = host.to("cuda")
+    order = torch.argsort(host.context_lens, descending=True).tolist()
+    gen = torch.Generator().manual_seed(number)
+    seqs = sorted(set([order[0], order[1], order[-1]] + torch.randperm(S, generator=gen)[:2].tolist()))
+    sub = _sub_workload(w, seqs)                   # taken before the product step
+    slots = torch.tensor([slot_for_position(host.block_tables[s].tolist(), int(host.context_lens[s]) - QL + j, B)
+                          for s in range(S) for j in range(QL)], dtype=torch.int64)
+    k_expect, v_expect = w.k_cache.clone(), w.v_cache.clone()
+    sd = slots.cuda()
+    k_expect[sd // B, :, sd % B, :] = w.k_new.reshape(S * QL, Hkv, D)
+    v_expect[sd // B, :, sd % B, :] = w.v_new.reshape(S * QL, Hkv, D)
+    out = torch.empty_like(w.q)
+    pkv.paged_attention_decode_mq(out, w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale,
+                                  host.max_context_len, k_new=w.k_new, v_new=w.v_new)
+    torch.cuda.synchronize()
+    assert torch.equal(w.k_cache, k_expect) and torch.equal(w.v_cache, v_expect)
+    del k_expect, v_expect
+
+    n = len(seqs)
+    sub_slots = torch.tensor([slot_for_position(sub.block_tables[r].tolist(), int(sub.context_lens[r]) - QL + j, B)
+                              for r in range(n) for j in range(QL)], dtype=torch.int64)
+    k_ref, v_ref = sub.k_cache.clone(), sub.v_cache.clone()
+    oracle.kv_write(k_ref, v_ref, sub.k_new.reshape(n * QL, Hkv, D).contiguous(),
+                    sub.v_new.reshape(n * QL, Hkv, D).contiguous(), sub_slots)
+    ref = oracle.paged_decode_mq(sub.q, k_ref, v_ref, sub.block_tables, sub.context_lens, sub.scale)
+    assert_close(out[torch.tensor(seqs, device="cuda")], ref, f"{w.name}, 16 new tokens")
+    assert pkv.pkv_device_status(0) == 0
+
+
 # ---------------------------------------------------------------------------
 # shapes and edges: every dtype, head dim and group size; lengths on and
 # around block and partition boundaries; the longest context
@@ -406,6 +453,13 @@ def test_partition_rule_on_this_device():
     assert pkv.paged_attention_partition_tokens(256, 8, 8130, bf16) == pkv.PARTITION_TOKENS_LONG
     assert pkv.paged_attention_partition_tokens(64, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS
     assert pkv.paged_attention_partition_tokens(24, 32, 1986, torch.float16) == pkv.PARTITION_TOKENS
+    # multi-query: more than 8 rows per kv head take the long partitions on any batch; up to 8 keep the rule above
+    mq = pkv.paged_attention_mq_partition_tokens
+    assert mq(64, 16, 40, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(2, 4, 32, 8, 300, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(pairs - 1, 2, 4, 1, 4096, bf16) == pkv.PARTITION_TOKENS
+    assert mq(pairs, 2, 4, 1, 4096, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(256, 1, 32, 8, 8130, bf16) == pkv.paged_attention_partition_tokens(256, 8, 8130, bf16)
 
 
 @pytest.mark.parametrize("block_size,dtype,D,G", [

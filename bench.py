@@ -247,10 +247,13 @@ def unique_live_tokens(tables, lens, block_size: int) -> int:
     live = idx[None, :] < nblk[:, None]                                  # [S, MB] entries in use
     used = (lens[:, None] - idx[None, :] * block_size).clamp(0, block_size)
     ids = tables.to(torch.int64)[live]
+    used = used[live]
+    keep = ids >= 0                       # an invalid id reads nothing the call counts
+    ids, used = ids[keep], used[keep]
     if ids.numel() == 0:
         return 0
     per_block = torch.zeros(int(ids.max()) + 1, dtype=torch.int64)
-    per_block.scatter_reduce_(0, ids, used[live], reduce="amax")
+    per_block.scatter_reduce_(0, ids, used, reduce="amax")
     return int(per_block.sum())
 
 
@@ -445,6 +448,7 @@ class ClockSampler:
         self.samples = []          # (monotonic time, sm MHz, power W, reasons bit mask)
         self.max_mhz = None
         self.source = None
+        self.nvml = None
         self._stop = threading.Event()
         self.thread = self.proc = None
 
@@ -457,6 +461,7 @@ class ClockSampler:
             reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
                               getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
             self.source = "nvml"
+            self.nvml = pynvml
             self.thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h, reasons), daemon=True)
         except Exception:
             try:
@@ -502,6 +507,13 @@ class ClockSampler:
                 self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
+            self.thread = None
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            self.nvml = None
 
     def summary(self, windows, label: str):
         """Median SM clock, peak power and every slowdown reason seen in the samples inside `windows`."""

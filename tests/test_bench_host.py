@@ -197,3 +197,19 @@ def test_multi_query_oracle_sample_equals_the_whole_batch_oracle():
     oracle.kv_write(k, v, kn.reshape(-1, Hkv, D), vn.reshape(-1, Hkv, D), slots)
     full = oracle.paged_decode_mq(q, k, v, w.block_tables, w.context_lens, w.scale)
     assert np.array_equal(np.stack(refs), full[seqs])
+
+
+def test_clock_summary_covers_only_the_timed_windows():
+    """The clock record: median SM clock, minimum, peak power and every
+    slowdown reason of the samples inside the given windows only."""
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.period, c.max_mhz, c.source = 0.002, 1965.0, "nvml"
+    c.samples = [(0.0, 900.0, 100.0, 0x8),            # outside: hw_slowdown must not be reported
+                 (1.0, 1965.0, 250.0, 0x0), (1.1, 1900.0, 300.0, 0x4), (1.2, 1950.0, 280.0, 0x0),
+                 (5.0, 1800.0, 260.0, 0x20)]          # in the second window: sw_thermal_slowdown
+    r = c.summary([(0.9, 1.3), (4.9, 5.1)], "test")
+    assert r["samples"] == 4 and r["sm_mhz"] == 1925.0 and r["sm_min_mhz"] == 1800.0
+    assert r["power_w_max"] == 300.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    empty = c.summary([(2.0, 3.0)], "none")
+    assert empty["samples"] == 0 and empty["sm_mhz"] is None

@@ -162,3 +162,26 @@ def test_shared_decode_host_side_rejections(L):
                                     ctypes.byref(ng), sh.data_ptr(), None, 0, ctypes.byref(nw), ctypes.byref(a),
                                     ctypes.byref(b)) == C["PKV_OK"]
     assert (ng.value, nw.value, a.value, b.value) == (1, 3, 48, 13)
+
+
+def test_copy_and_swap_list_checks_cost_the_list_not_the_pool(L):
+    """block_copy and swap_blocks_in check their id lists by sorting them, so
+    a check on a pool of 2^20 blocks costs microseconds, not a pool-sized
+    scan.  The lists here are rejected (a dst that is also a src; an id
+    named twice), which happens on the host before any CUDA call."""
+    import time
+    from paged_kv_cache_398_b200._lib import C
+    INV = C["PKV_ERR_INVALID_ARG"]
+    NB = 1 << 20
+    fake = ctypes.c_void_p(1 << 20)                     # 16-byte aligned; never dereferenced
+    pairs = torch.tensor([[i, NB - 1 - i] for i in range(7)] + [[100, 3]], dtype=torch.int64)  # 3 is a src
+    ids = torch.tensor(list(range(0, NB, NB // 15)) + [0], dtype=torch.int64)                   # 0 twice
+    args_c = (fake, fake, ctypes.c_void_p(pairs.data_ptr()), pairs.shape[0], 8, 128, 16, NB, 2, None)
+    args_s = (fake, fake, ctypes.c_void_p(ids.data_ptr()), ids.shape[0], fake, fake, 8, 128, 16, NB, 2, None)
+    assert L.block_copy(*args_c) == INV and L.swap_blocks_in(*args_s) == INV
+    for fn, args in ((L.block_copy, args_c), (L.swap_blocks_in, args_s)):
+        t0 = time.perf_counter()
+        for _ in range(200):
+            assert fn(*args) == INV
+        per_call = (time.perf_counter() - t0) / 200
+        assert per_call < 50e-6, f"{fn.__name__}: {per_call * 1e6:.1f} us a check"

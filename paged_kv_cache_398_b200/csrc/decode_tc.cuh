@@ -271,7 +271,6 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
     using C = TcCfg<D>;
     constexpr int part_tokens = PT;
     static_assert(PT == kPartTokens || PT == kLongPartTokens, "partition sizes");
-    static_assert(kPlan != kPlanGroup || kMQ, "the group pass uses the 16-row form");
     static_assert(kPlan != kPlanOwn || !kMQ, "a sequence's own pass has one query");
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
     constexpr int kRows = kMQ ? 16 : 8;  // operand rows that can hold queries
@@ -641,8 +640,9 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
                 // some token of this block lies past a row's last visible
                 // position: ctx - 1 for one query, the row's own token's
                 // position for several; padding rows keep ctx (finite scores)
-                const int lim0 = qd < rows ? first_new + qd / G + 1 : ctx;
-                const int lim1 = qd + 1 < rows ? first_new + (qd + 1) / G + 1 : ctx;
+                // (the group pass: every row sees all of [0, x) -- no causal limit)
+                const int lim0 = kPlan != kPlanGroup && qd < rows ? first_new + qd / G + 1 : ctx;
+                const int lim1 = kPlan != kPlanGroup && qd + 1 < rows ? first_new + (qd + 1) / G + 1 : ctx;
                 if (pos0 + ra >= lim0) x[0] = -INFINITY;
                 if (pos0 + ra >= lim1) x[1] = -INFINITY;
                 if (pos0 + ra + 8 >= lim0) x[2] = -INFINITY;
@@ -977,11 +977,21 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
         return;
     }
     if (w.x < 0) {
-        partition_tc<T, D, G, true, B, PT, kPlanGroup>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, nullptr, nullptr,
-                                                        k_cache_w, v_cache_w, block_tables, mb, context_lens, max_ctx,
-                                                        1, num_q_heads, num_kv_heads, num_blocks, scale_log2,
-                                                        max_parts, status, plan_groups, shared_lens, num_seqs, w.y, h,
-                                                        ~w.x);
+        // a group of at most 8 rows (members x G) runs the transposed 8-column
+        // form, a larger one the 16-row form (either checks the group again)
+        const int n = pkv::ld_early(plan_groups + 2 * (int64_t)(~w.x) + 1);
+        if (n * G <= 8)
+            partition_tc<T, D, G, false, B, PT, kPlanGroup>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, nullptr, nullptr,
+                                                             k_cache_w, v_cache_w, block_tables, mb, context_lens,
+                                                             max_ctx, 1, num_q_heads, num_kv_heads, num_blocks,
+                                                             scale_log2, max_parts, status, plan_groups, shared_lens,
+                                                             num_seqs, w.y, h, ~w.x);
+        else
+            partition_tc<T, D, G, true, B, PT, kPlanGroup>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, nullptr, nullptr,
+                                                            k_cache_w, v_cache_w, block_tables, mb, context_lens,
+                                                            max_ctx, 1, num_q_heads, num_kv_heads, num_blocks,
+                                                            scale_log2, max_parts, status, plan_groups, shared_lens,
+                                                            num_seqs, w.y, h, ~w.x);
     } else {
         partition_tc<T, D, G, false, B, PT, kPlanOwn>(&tm_k, &tm_v, out, ws_acc, ws_ml, q, k_new, v_new, k_cache_w,
                                                        v_cache_w, block_tables, mb, context_lens, max_ctx, 1,

@@ -65,6 +65,9 @@ def _parity(w, min_shared_tokens=128):
     (torch.bfloat16, 32, 128, 16, 2, 2),   # 8 query heads per kv head: groups of 2
     (torch.float16, 16, 128, 8, 4, 8),     # 2 per kv head: 8 samples
     (torch.bfloat16, 8, 128, 8, 2, 3),     # groups smaller than the operand allows
+    (torch.bfloat16, 16, 128, 32, 8, 2),   # 2 samples x 4 heads = 8 rows: the transposed 8-column group pass
+    (torch.float16, 16, 64, 4, 4, 5),      # 5 samples x 1 head = 5 rows (8-column form)
+    (torch.float16, 32, 128, 16, 8, 3),    # 3 samples x 2 heads = 6 rows (8-column form), block size 32
 ])
 def test_shared_decode_matches_oracle(dtype, B, D, Hq, Hkv, samples):
     w = make_sampling(5, samples, (1, 1400), (1, 300), Hq, Hkv, D, dtype, seed=70 + B + samples, block_size=B)
@@ -73,6 +76,16 @@ def test_shared_decode_matches_oracle(dtype, B, D, Hq, Hkv, samples):
     expect = sum(1 for p in w.meta["prompt_lens"] if (p // B) * B >= 128)
     assert plan.groups.shape[0] == expect
     assert all(n == samples for _, n in plan.groups.tolist())
+
+
+def test_groups_of_both_forms_in_one_launch():
+    """A family of 12 samples at 2 query heads per kv head splits into a
+    group of 8 (16 rows: the 16-row form) and one of 4 (8 rows: the
+    8-column form); both forms run in the same launch."""
+    w = make_sampling(3, 12, (600, 1400), (1, 200), 8, 4, 128, torch.bfloat16, seed=91)
+    plan = _parity(w)
+    sizes = sorted(n for _, n in plan.groups.tolist())
+    assert sizes == [4, 4, 4, 8, 8, 8]
 
 
 def test_shared_lengths_on_partition_edges():

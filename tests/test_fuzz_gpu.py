@@ -38,9 +38,34 @@ def _case(seed):
     return dtype, D, G, B, Hkv, S, q_len, fused, lens, rng.random() < 0.5
 
 
+def _mq_case(seed):
+    """Many new tokens per sequence on one or two query heads per kv head:
+    the 16-row form, its long partitions and both write paths."""
+    rng = random.Random(20_000 + seed)
+    dtype = rng.choice([torch.float16, torch.bfloat16])
+    D = rng.choice([64, 128])
+    G = rng.choice([1, 1, 2])
+    B = rng.choice([8, 16, 16, 32])
+    Hkv = rng.choice([1, 2, 3])
+    S = rng.randint(1, 5)
+    q_len = rng.randint(5, 16 // G)
+    fused = rng.random() < 0.5
+    lens = [max(q_len, rng.choice([rng.randint(1, 60), rng.randint(500, 1100), rng.randint(1000, 3100)]))
+            for _ in range(S)]
+    return dtype, D, G, B, Hkv, S, q_len, fused, lens, rng.random() < 0.5
+
+
 @pytest.mark.parametrize("seed", range(40))
 def test_random_case_matches_oracle(seed, cuda_device):
-    dtype, D, G, B, Hkv, S, q_len, fused, lens, pad_random = _case(seed)
+    _check_case(seed, *_case(seed))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_many_new_tokens_case_matches_oracle(seed, cuda_device):
+    _check_case(500 + seed, *_mq_case(seed))
+
+
+def _check_case(seed, dtype, D, G, B, Hkv, S, q_len, fused, lens, pad_random):
     w = make_custom(lens, Hkv * G, Hkv, D, dtype, seed=1000 + seed, block_size=B, pad_random=pad_random,
                     q_len=q_len if q_len > 1 else None, spare_blocks=5)
     mq = q_len > 1

@@ -298,6 +298,26 @@ int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_blocks_per_s
                            int32_t* max_shared_len_out, int32_t* max_own_len_out);
 
 /*
+ * pkv_shared_prefix_order -- host only.  A batch order in which sequences
+ * whose tables start with the same physical blocks are adjacent, for a
+ * serving loop whose batch interleaves requests that share a cached prefix
+ * ("Prefix Caching") or samples of several prompts: pkv_shared_prefix_plan
+ * groups only runs of consecutive sequences.  The order sorts the sequences
+ * by the ids of their shareable blocks (those wholly below their last
+ * position, up to the first negative entry) lexicographically, and is
+ * stable: sequences with equal rows keep their batch order.
+ *
+ *  block_tables, context_lens  as pkv_shared_prefix_plan (host int32)
+ *  order_out      host, int64 [num_seqs]: position i of the reordered batch
+ *                 holds sequence order_out[i] (a permutation of 0..num_seqs-1)
+ * Returns PKV_OK, PKV_ERR_INVALID_ARG (a length outside [1,
+ * max_blocks_per_seq * block_size], bad sizes, null pointers) or
+ * PKV_ERR_HOST_MEMORY.
+ */
+int pkv_shared_prefix_order(const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t block_size, int64_t* order_out);
+
+/*
  * paged_attention_decode_shared -- one decode step (one new token per
  * sequence, optionally fused with its slot write) with a plan from
  * pkv_shared_prefix_plan.  Computes the attention paged_attention_decode_mq

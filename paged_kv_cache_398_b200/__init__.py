@@ -24,7 +24,8 @@ from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, SHARE
                       paged_attention_decode_shared, paged_attention_mq_workspace_bytes,
                       paged_attention_mq_partition_tokens, paged_attention_partition_tokens,
                       paged_attention_shared_workspace_bytes,
-                      paged_attention_workspace_bytes, paged_kv_write, pkv_device_status, pkv_shared_prefix_plan,
+                      paged_attention_workspace_bytes, paged_kv_write, pkv_device_status, pkv_shared_prefix_order,
+                      pkv_shared_prefix_plan,
                       pkv_slot_mapping, swap_blocks_in, swap_blocks_out)
 
 __all__ = [
@@ -34,6 +35,6 @@ __all__ = [
     "paged_attention_decode_noalloc", "paged_attention_decode_shared", "paged_attention_mq_workspace_bytes",
     "paged_attention_mq_partition_tokens", "paged_attention_partition_tokens",
     "paged_attention_shared_workspace_bytes", "paged_attention_workspace_bytes",
-    "SHARED_MAX_ROWS", "SharedPrefixPlan", "pkv_shared_prefix_plan",
+    "SHARED_MAX_ROWS", "SharedPrefixPlan", "pkv_shared_prefix_order", "pkv_shared_prefix_plan",
     "paged_kv_write", "pkv_device_status", "pkv_slot_mapping", "swap_blocks_in", "swap_blocks_out",
 ]

@@ -55,6 +55,7 @@ _SIGS = {
     "paged_attention_decode_shared": ([P, P, P, P, P, P, P, I32, P, I32, I32, P, I32, P, P, I32, I32, I32, I32, I32,
                                        I32, I32, ctypes.c_float, I32, P, SZ, P], ctypes.c_int),
     "pkv_shared_prefix_plan": ([P, I32, P, I32, I32, I32, I32, I32, P, P, P, P, I32, P, P, P], ctypes.c_int),
+    "pkv_shared_prefix_order": ([P, I32, P, I32, I32, P], ctypes.c_int),
     "paged_attention_decode_noalloc": ([P, P, P, P, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
                                         ctypes.c_float, I32, P], ctypes.c_int),
     "block_copy": ([P, P, P, I32, I32, I32, I32, I32, I32, P], ctypes.c_int),

@@ -241,6 +241,23 @@ def pkv_shared_prefix_plan(block_tables, context_lens, block_size: int, max_grou
                             int(part_tokens), int(mx_shared.value), int(mx_own.value))
 
 
+def pkv_shared_prefix_order(block_tables, context_lens, block_size: int) -> torch.Tensor:
+    """A batch order (int64 permutation) that puts sequences whose HOST int32
+    block_tables [S, MB] start with the same blocks next to each other, so
+    that pkv_shared_prefix_plan on the reordered batch can group them."""
+    bt = torch.as_tensor(block_tables, dtype=torch.int32).contiguous()
+    cl = torch.as_tensor(context_lens, dtype=torch.int32).contiguous()
+    if bt.device.type != "cpu" or cl.device.type != "cpu" or bt.dim() != 2 or cl.dim() != 1 or \
+            bt.shape[0] != cl.shape[0]:
+        raise ValueError("block_tables [S, MB] and context_lens [S] must be host int32 tensors")
+    S = cl.shape[0]
+    order = torch.empty(S, dtype=torch.int64)
+    check("pkv_shared_prefix_order", lib().pkv_shared_prefix_order(
+        bt.data_ptr() if S else None, max(bt.shape[1], 1), cl.data_ptr() if S else None, S, int(block_size),
+        order.data_ptr() if S else None))
+    return order
+
+
 def paged_attention_shared_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int,
                                            max_context_len: int) -> int:
     return int(lib().paged_attention_shared_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len))

@@ -19,6 +19,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <numeric>
 #include <vector>
 
 #include "paged_kv.h"
@@ -132,5 +133,38 @@ extern "C" int pkv_shared_prefix_plan(const int32_t* block_tables, int32_t max_b
         work_out[2 * k] = items[k].a;
         work_out[2 * k + 1] = items[k].p;
     }
+    return PKV_OK;
+}
+
+// A batch order that puts sequences whose tables start with the same blocks
+// next to each other: the rows' shareable blocks (valid ids wholly below the
+// sequence's last position) in lexicographic order, stable, so a common
+// prefix makes a contiguous run and siblings keep their batch order.
+extern "C" int pkv_shared_prefix_order(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       const int32_t* context_lens, int32_t num_seqs, int32_t block_size,
+                                       int64_t* order_out)
+{
+    if (num_seqs < 0 || max_blocks_per_seq < 1 || block_size < 1) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (!block_tables || !context_lens || !order_out) return PKV_ERR_INVALID_ARG;
+    const int64_t cap = (int64_t)max_blocks_per_seq * block_size;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (context_lens[s] < 1 || context_lens[s] > cap) return PKV_ERR_INVALID_ARG;
+    std::vector<int32_t> idx, len;
+    try {
+        idx.resize((size_t)num_seqs);
+        len.resize((size_t)num_seqs);
+    } catch (...) {  // no C++ exception leaves a C call
+        return PKV_ERR_HOST_MEMORY;
+    }
+    auto row = [&](int32_t s) { return block_tables + (int64_t)s * max_blocks_per_seq; };
+    for (int32_t s = 0; s < num_seqs; ++s) len[s] = valid_entries(row(s), (context_lens[s] - 1) / block_size);
+    std::iota(idx.begin(), idx.end(), 0);
+    std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) {
+        const int32_t n = std::min(len[a], len[b]);
+        const int32_t k = common_entries(row(a), row(b), n);
+        return k < n ? row(a)[k] < row(b)[k] : len[a] < len[b];  // a row that is a prefix of the other first
+    });
+    for (int32_t i = 0; i < num_seqs; ++i) order_out[i] = idx[i];
     return PKV_OK;
 }

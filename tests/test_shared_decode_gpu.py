@@ -88,6 +88,26 @@ def test_groups_of_both_forms_in_one_launch():
     assert sizes == [4, 4, 4, 8, 8, 8]
 
 
+def test_interleaved_batch_reordered_for_sharing():
+    """A batch whose families are interleaved (as a serving loop may admit
+    them): pkv_shared_prefix_order brings each family's samples together, and
+    shared-prefix decode of the reordered batch finds every group and
+    matches the oracle."""
+    import dataclasses
+    w = make_sampling(5, 4, (300, 1500), (1, 200), 32, 8, 128, torch.bfloat16, seed=77)
+    grouped = make_plan(w).groups.shape[0]
+    perm = torch.randperm(w.num_seqs, generator=torch.Generator().manual_seed(8))
+
+    def take(src, idx):
+        return dataclasses.replace(src, block_tables=src.block_tables[idx], context_lens=src.context_lens[idx],
+                                   q=src.q[idx], k_new=src.k_new[idx], v_new=src.v_new[idx])
+    shuffled = take(w, perm)
+    assert make_plan(shuffled).groups.shape[0] < grouped
+    order = pkv.pkv_shared_prefix_order(shuffled.block_tables, shuffled.context_lens, shuffled.block_size)
+    plan = _parity(take(shuffled, order))
+    assert plan.groups.shape[0] == grouped
+
+
 def test_shared_lengths_on_partition_edges():
     # prompts whose shared part ends just before, on and after a partition boundary
     dtype, B = torch.bfloat16, 16

@@ -265,3 +265,75 @@ def test_plans_of_arbitrary_tables_are_valid():
         _check_valid(t, lens, plan, max_group, min_tokens, bs)
 
     check()
+
+
+# ---------------------------------------------------------------------------
+# pkv_shared_prefix_order: a batch order that makes sharing sequences adjacent
+# ---------------------------------------------------------------------------
+def test_order_regroups_an_interleaved_batch():
+    """Samples of several prompts, shuffled through the batch: the plan of
+    the shuffled batch finds (almost) nothing; reordered by
+    pkv_shared_prefix_order, it finds every group the unshuffled batch has."""
+    from paged_kv_cache_398_b200.workloads import make_sampling
+    w = make_sampling(6, 4, (300, 900), (1, 60), 8, 2, 64, torch.float16, seed=17)
+    plan = pkv.pkv_shared_prefix_plan(w.block_tables, w.context_lens, B, 4, 512)
+    perm = torch.randperm(w.num_seqs, generator=torch.Generator().manual_seed(3))
+    bt, cl = w.block_tables[perm], w.context_lens[perm]
+    shuffled = pkv.pkv_shared_prefix_plan(bt, cl, B, 4, 512)
+    order = pkv.pkv_shared_prefix_order(bt, cl, B)
+    assert sorted(order.tolist()) == list(range(w.num_seqs))
+    again = pkv.pkv_shared_prefix_plan(bt[order], cl[order], B, 4, 512)
+    assert shuffled.groups.shape[0] < plan.groups.shape[0]
+    assert again.groups.shape[0] == plan.groups.shape[0]
+    assert int(again.shared_lens.sum()) == int(plan.shared_lens.sum())
+    _check_valid(bt[order], cl[order], again, 4, 128)
+
+
+def test_order_makes_every_common_prefix_contiguous():
+    """Brute force on random small tables: after the reordering, the
+    sequences whose shareable blocks start with any given prefix sit at
+    consecutive positions, and sequences with equal rows keep their batch
+    order."""
+    rng = random.Random(5)
+    for _ in range(300):
+        S = rng.randint(1, 9)
+        lens = [rng.randint(1, 5 * B) for _ in range(S)]
+        rows = [[rng.choice([0, 1, 2, rng.randint(3, 40)]) for _ in range(5)] for _ in range(S)]
+        for r in rows:                                  # now and then a hole (-1) inside a row
+            if rng.random() < 0.2:
+                r[rng.randint(0, 4)] = -1
+        bt, cl = _tables(rows), torch.tensor(lens, dtype=torch.int32)
+        order = pkv.pkv_shared_prefix_order(bt, cl, B).tolist()
+        assert sorted(order) == list(range(S))
+
+        def key(s):                                   # shareable blocks: valid ids below the last position
+            k = []
+            for b in rows[s][:(lens[s] - 1) // B]:
+                if b < 0:
+                    break
+                k.append(b)
+            return k
+        keys = [key(s) for s in order]
+        for L in range(1, 6):
+            seen = {}
+            for pos, k in enumerate(keys):
+                if len(k) >= L:
+                    seen.setdefault(tuple(k[:L]), []).append(pos)
+            for positions in seen.values():
+                # no sequence without the prefix sits between two that hold it
+                assert positions == list(range(positions[0], positions[-1] + 1))
+        for i in range(S - 1):
+            if keys[i] == keys[i + 1]:
+                assert order[i] < order[i + 1]
+
+
+def test_order_rejects_bad_arguments():
+    L = pkv._lib.lib()
+    C = pkv._lib.C
+    bt, cl = _tables([[0, 1], [0, 2]]), torch.tensor([20, 40], dtype=torch.int32)
+    assert pkv.pkv_shared_prefix_order(bt[:0], cl[:0], B).numel() == 0
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pkv_shared_prefix_order(bt, torch.tensor([20, 33], dtype=torch.int32), B)   # past the table
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pkv_shared_prefix_order(bt, torch.tensor([0, 20], dtype=torch.int32), B)    # empty sequence
+    assert L.pkv_shared_prefix_order(None, 2, None, 2, B, None) == C["PKV_ERR_INVALID_ARG"]

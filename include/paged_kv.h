@@ -329,9 +329,9 @@ int pkv_shared_prefix_order(const int32_t* block_tables, int32_t max_blocks_per_
  * but in two passes, run by one launch over the plan's work list.  The group
  * pass reads the blocks of positions [0, x) of a group once, through the
  * first member's table, and attends all members' query heads to them
- * together (members x (num_q_heads / num_kv_heads) rows of one 16-row
- * tensor-core operand).  Each sequence's own pass reads its positions
- * [x, ctx), and the split-K reduce merges both.
+ * together (members x (num_q_heads / num_kv_heads) rows: at most 8 in the
+ * 8-column tensor-core form, up to 16 in the 16-row form).  Each sequence's
+ * own pass reads its positions [x, ctx), and the split-K reduce merges both.
  *
  *  groups         device, int32 [num_groups][2], as groups_out; may be NULL
  *                 when num_groups is 0

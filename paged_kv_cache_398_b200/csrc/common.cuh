@@ -51,9 +51,13 @@ inline size_t dtype_bytes(int32_t dtype)
 
 // Launch configuration whose kernel may be staged while the previous kernel
 // on the stream finishes (programmatic dependent launch).  The kernel must
-// call grid_dependency_wait() before it reads anything a previous kernel may
-// have written.  After a non-kernel stream operation the launch simply
-// waits, as an ordinary one would.
+// call grid_dependency_wait() before it reads anything the previous kernel
+// writes.  After a non-kernel stream operation the launch simply waits, as an
+// ordinary one would.  The previous kernel releases it at the exit of its
+// last CTA, or earlier where that kernel calls grid_dependency_launch(); the
+// partition kernels call it only after their own grid_dependency_wait(), so
+// whatever was written before them is complete, and visible at L2, by the
+// time a kernel they release starts.
 inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
@@ -91,6 +95,15 @@ inline void pdl_attribute(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr)
 __device__ __forceinline__ void grid_dependency_wait()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel on the stream, when it was launched as a dependent,
+// to start before this grid ends (its grid_dependency_wait() still waits for
+// this grid's completion).  Once every CTA has called it or exited, that
+// kernel's CTAs can take SM slots this grid's tail leaves free.
+__device__ __forceinline__ void grid_dependency_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // A read-only 32-bit global load kept where it is written (volatile asm): a

@@ -118,6 +118,15 @@ __device__ __forceinline__ int split_parts(int x, int ctx, int part_tokens)
 // launch).  One warp per (sequence, query head); each lane owns
 // head_dim / 32 consecutive outputs and issues the vector loads of up to 8
 // partitions before it consumes them.
+//
+// The tensor-core partition kernels release this kernel early
+// (grid_dependency_launch), so a warp decides whether its row needs a merge
+// before it waits for them: the lengths are inputs of the call, complete
+// before the partition kernel started, and are read at L2.  Rows that fit
+// one partition (most of them in a batch of short contexts) then cost
+// nothing after the partition grid ends.  CTA 0 waits in any case, so that
+// this grid never completes before the partition grid does: a kernel that
+// waits for this one also waits for that one.
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
     decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_acc,
@@ -129,19 +138,20 @@ __global__ void __launch_bounds__(128)
     constexpr int kPer = D / 32;
     using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
     constexpr int kUnroll = 8;
-    pkv::grid_dependency_wait();  // the partition kernel's results are visible after this
+    if (blockIdx.x == 0) pkv::grid_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (row >= (int64_t)num_seqs * q_len * num_q_heads) return;   // row = (s * q_len + j) * Hq + i
     const int s = (int)(row / ((int64_t)q_len * num_q_heads));
-    const SeqRange sr = seq_range(context_lens, s, mb, block_size, max_ctx, part_tokens, false, nullptr);
+    const SeqRange sr = seq_range_of(__ldcg(context_lens + s), mb, block_size, max_ctx, part_tokens, false, nullptr);
     if (sr.bad || sr.ctx < q_len) return;   // zero rows: written
     // partitions: ceil(ctx / pt), or the group's and the sequence's own when
     // its positions are split (paged_attention_decode_shared)
     const int nparts =
-        shared_lens ? split_parts(shared_split(__ldg(shared_lens + s), sr.ctx, block_size), sr.ctx, part_tokens)
+        shared_lens ? split_parts(shared_split(__ldcg(shared_lens + s), sr.ctx, block_size), sr.ctx, part_tokens)
                     : sr.nparts;
     if (nparts <= 1) return;   // single partition: written by the partition kernel
+    pkv::grid_dependency_wait();  // the partition kernel's results are visible after this
     const float* ml = ws_ml + row * max_parts * 2;
     const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
     constexpr int kStride = D / kPer;  // Vec elements per partition

@@ -278,6 +278,10 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     pkv::grid_dependency_wait();  // inputs written by the previous kernel are visible after this
+    // the split-K reduce may launch now: its CTAs whose rows need no merge
+    // finish inside this grid's tail (after this grid's own wait, so the
+    // lengths they read before theirs are complete)
+    pkv::grid_dependency_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool report = p == 0 && h == 0 && threadIdx.x == 0;
     constexpr int part_blocks = part_tokens / B;

@@ -156,6 +156,45 @@ __global__ void __launch_bounds__(128)
     const Vec* acc = reinterpret_cast<const Vec*>(ws_acc + row * max_parts * D) + lane;
     constexpr int kStride = D / kPer;  // Vec elements per partition
 
+    if (nparts <= kUnroll) {
+        // every record load of the row is issued before any is used: one
+        // round trip to L2 (the same arithmetic, in the same order, as below)
+        Vec a[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (u < nparts) a[u] = acc[(int64_t)u * kStride];
+        }
+        const float m = lane < nparts ? ml[lane * 2] : -INFINITY;
+        const float lv = lane < nparts ? ml[lane * 2 + 1] : 0.0f;
+        float M = m;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        M = fmaxf(-INFINITY, M);
+        if (M == INFINITY) return;  // a poison record: see below
+        float w = 0.0f, lw = 0.0f;
+        if (lane < nparts) {
+            w = exp2f(m - M);
+            lw = lv * w;
+        }
+        float L = 0.0f;
+        float o[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) o[e] = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (u < nparts) {  // warp-uniform
+                const float wj = __shfl_sync(0xffffffffu, w, u);
+                L += __shfl_sync(0xffffffffu, lw, u);
+                const float* av = reinterpret_cast<const float*>(&a[u]);
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) o[e] = fmaf(av[e], wj, o[e]);
+            }
+        }
+        const float inv = 1.0f / L;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) pkv::store_out(out + row * D + lane * kPer + e, o[e] * inv);
+        return;
+    }
     float M = -INFINITY;
     for (int p0 = 0; p0 < nparts; p0 += 32) {
         const int pp = p0 + lane;

@@ -197,3 +197,35 @@ def test_fused_decode_step_replays_from_a_cuda_graph():
     step()
     torch.cuda.synchronize()
     assert torch.equal(replayed, out) and not torch.equal(replayed, eager)
+
+
+@pytest.mark.parametrize("G,q_len", [(1, 16), (4, 1)])
+def test_back_to_back_fused_calls_when_every_row_fits_one_partition(G, q_len):
+    """max_context_len far above every length: the split-K reduce is launched
+    but no row needs it, so all of its CTAs but the first leave before they
+    wait for the partition kernel.  A second fused call issued right behind
+    rewrites the very slots the first one reads (same lengths, other new
+    tokens); each call must still attend to its own new tokens only."""
+    import dataclasses
+    Hkv, D, dtype, max_ctx = 4, 128, torch.float16, 4096
+    lens = [max(n, q_len) for n in (1, 17, 200, 333, 480, 500)]   # one partition of 512 or 1024 tokens each
+    w1 = make_custom(lens, Hkv * G, Hkv, D, dtype, seed=77 + G, q_len=q_len,
+                     max_blocks_per_seq=max_ctx // B)
+    g = torch.Generator().manual_seed(5 + G)
+    w2 = dataclasses.replace(w1, q=torch.randn(w1.q.shape, generator=g).to(dtype),
+                             k_new=torch.randn(w1.k_new.shape, generator=g).to(dtype),
+                             v_new=torch.randn(w1.v_new.shape, generator=g).to(dtype))
+    ref1, k_ref1, v_ref1 = oracle_mq(w1, q_len)
+    ref2, k_ref2, v_ref2 = oracle_mq(dataclasses.replace(w2, k_cache=k_ref1, v_cache=v_ref1), q_len)
+    assert pkv.paged_attention_mq_workspace_bytes(w1.num_seqs, q_len, w1.num_q_heads, D, max_ctx) > 0
+    a = w1.to("cuda")
+    q2, kn2, vn2 = w2.q.cuda(), w2.k_new.cuda(), w2.v_new.cuda()
+    out1, out2 = torch.empty_like(a.q), torch.empty_like(a.q)
+    for out, q, kn, vn in ((out1, a.q, a.k_new, a.v_new), (out2, q2, kn2, vn2)):
+        pkv.paged_attention_decode_mq(out, q, a.k_cache, a.v_cache, a.block_tables, a.context_lens, a.scale,
+                                      max_ctx, k_new=kn, v_new=vn)
+    torch.cuda.synchronize()
+    assert torch.equal(a.k_cache.cpu(), k_ref2) and torch.equal(a.v_cache.cpu(), v_ref2)
+    assert_close(out1, ref1, "first call")
+    assert_close(out2, ref2, "second call")
+    assert pkv.pkv_device_status(0) == 0

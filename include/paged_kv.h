@@ -21,7 +21,13 @@
  *    host memory, read before the call returns.
  *  - Streams.  `stream` is a cudaStream_t passed as void*; NULL means the
  *    legacy default stream.  Device calls only enqueue work and return
- *    without synchronising.
+ *    without synchronising.  The decode kernels are launched with
+ *    programmatic stream serialisation and release the next kernel on the
+ *    stream before they finish.  An ordinary launch after them still waits
+ *    for all of them; a kernel that the caller launches with programmatic
+ *    serialisation itself must call cudaGridDependencySynchronize() (PTX
+ *    griddepcontrol.wait) before it reads what the decode call wrote, as
+ *    any such kernel must.
  *  - Cache layout.  k_cache and v_cache are each
  *    [num_blocks][num_kv_heads][block_size][head_dim], row-major, in the
  *    element type `dtype`.  Every (block, kv head) tile is therefore one

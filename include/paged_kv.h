@@ -111,20 +111,24 @@ int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_
 /*
  * Split-K partitions.  Decode splits each sequence into partitions of
  * PKV_PARTITION_TOKENS tokens, one thread block each, and merges them.  A
- * launch uses PKV_PARTITION_TOKENS_LONG instead when it is fp16 / bf16,
- * max_context_len >= PKV_LONG_MIN_CONTEXT, and num_seqs * num_kv_heads >=
- * PKV_LONG_MIN_PAIRS_PER_SM x the device's multiprocessor count.  Such a
- * batch fills the GPU with (sequence, kv head) pairs alone, and halving its
- * thread-block count saves more fixed per-block cost than the longer
- * blocks add to the tail.  A multi-query launch of more than 8 query rows
- * per kv head (q_len * num_q_heads / num_kv_heads > 8, the 16-row form)
- * always uses PKV_PARTITION_TOKENS_LONG: every partition ends with 16 rows
- * of output or split-K records, so fewer, longer partitions write and merge
- * less.  The choice depends only on these launch values, so calls with the
- * same shape always split the same way.
+ * launch of fp16 / bf16 with num_seqs * num_kv_heads >=
+ * PKV_LONG_MIN_PAIRS_PER_SM x the device's multiprocessor count (a "large
+ * batch": its (sequence, kv head) pairs alone fill the GPU) and
+ * max_context_len >= PKV_LONG_MIN_CONTEXT uses PKV_PARTITION_TOKENS_WIDE
+ * instead: fewer thread blocks, and fewer of them past a shorter sequence's
+ * end, save more fixed per-block cost than the longer blocks add to the
+ * tail.  A multi-query launch of more than 8 query rows per kv head
+ * (q_len * num_q_heads / num_kv_heads > 8, the 16-row form) uses
+ * PKV_PARTITION_TOKENS_WIDE on a large batch of any context length and
+ * PKV_PARTITION_TOKENS_LONG otherwise: every partition ends with 16 rows of
+ * output or split-K records, so fewer, longer partitions write and merge
+ * less.  Shared-prefix decode follows the one-query rule.  The choice
+ * depends only on these launch values, so calls with the same shape always
+ * split the same way.
  */
 #define PKV_PARTITION_TOKENS 512
 #define PKV_PARTITION_TOKENS_LONG 1024
+#define PKV_PARTITION_TOKENS_WIDE 2048
 #define PKV_LONG_MIN_CONTEXT 4096
 #define PKV_LONG_MIN_PAIRS_PER_SM 12
 
@@ -132,7 +136,7 @@ int paged_kv_write(const void* k_new, const void* v_new, void* k_cache, void* v_
  * paged_attention_partition_tokens -- the partition size, in tokens, that
  * paged_attention_decode and paged_attention_decode_mq use for this launch
  * shape on the current device (rule above).  Returns PKV_PARTITION_TOKENS,
- * PKV_PARTITION_TOKENS_LONG, or a negative PKV_ERR_* code (no CUDA device:
+ * PKV_PARTITION_TOKENS_WIDE, or a negative PKV_ERR_* code (no CUDA device:
  * PKV_ERR_CUDA).
  */
 int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,
@@ -142,7 +146,8 @@ int32_t paged_attention_partition_tokens(int32_t num_seqs, int32_t num_kv_heads,
  * paged_attention_mq_partition_tokens -- the same for a
  * paged_attention_decode_mq launch of q_len new tokens per sequence (rule
  * above; q_len 1 gives paged_attention_partition_tokens).  Returns
- * PKV_PARTITION_TOKENS, PKV_PARTITION_TOKENS_LONG, or a negative PKV_ERR_*
+ * PKV_PARTITION_TOKENS, PKV_PARTITION_TOKENS_LONG, PKV_PARTITION_TOKENS_WIDE,
+ * or a negative PKV_ERR_*
  * code: PKV_ERR_INVALID_ARG for a bad shape (num_q_heads not a multiple of
  * num_kv_heads included), PKV_ERR_CUDA with no CUDA device where the rule
  * needs the multiprocessor count.
@@ -382,8 +387,9 @@ int paged_attention_decode_shared(void* out, const void* q, const void* k_new, c
  * pkv_debug_shared_occupancy -- test hook: resident thread blocks per SM of
  * paged_attention_decode_shared's kernel for this instantiation (fp16 /
  * bf16), as the CUDA occupancy calculator reports it with the kernel's
- * shared memory.  Launches nothing.  Returns PKV_ERR_UNSUPPORTED for shapes
- * the call does not build.
+ * shared memory; long_partitions != 0 selects the PKV_PARTITION_TOKENS_WIDE
+ * variant, 0 the PKV_PARTITION_TOKENS one.  Launches nothing.  Returns
+ * PKV_ERR_UNSUPPORTED for shapes the call does not build.
  */
 int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32_t group, int32_t block_size,
                                int32_t long_partitions, int32_t* ctas_per_sm);
@@ -518,7 +524,9 @@ int pkv_last_cuda_error(void);
  * current device (cudaOccupancyMaxActiveBlocksPerMultiprocessor, with the
  * kernel's own shared memory).  group = num_q_heads / num_kv_heads; q_len > 1
  * selects the multi-query kernel; long_partitions != 0 the
- * PKV_PARTITION_TOKENS_LONG variant (fp16 / bf16).  Enqueues nothing.  A
+ * PKV_PARTITION_TOKENS_WIDE variant (fp16 / bf16), 0 the other one
+ * (PKV_PARTITION_TOKENS, or PKV_PARTITION_TOKENS_LONG for more than 8 rows
+ * per kv head).  Enqueues nothing.  A
  * tensor-core kernel is built for 3 per SM (its shared memory and 168
  * registers); fewer means a build lost a third of the bytes in flight.
  */

@@ -19,8 +19,8 @@ The native library ``libpaged_kv.so`` is built in-tree by
 
 from ._lib import LibraryMissing, PagedKVError
 from .allocator import TABLE_KEEP_TAIL, BlockAllocator, OutOfBlocks
-from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, SHARED_MAX_ROWS, SharedPrefixPlan,
-                      block_copy, paged_attention_decode, paged_attention_decode_mq, paged_attention_decode_noalloc,
+from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, PARTITION_TOKENS_WIDE, SHARED_MAX_ROWS,
+                      SharedPrefixPlan, block_copy, paged_attention_decode, paged_attention_decode_mq, paged_attention_decode_noalloc,
                       paged_attention_decode_shared, paged_attention_mq_workspace_bytes,
                       paged_attention_mq_partition_tokens, paged_attention_partition_tokens,
                       paged_attention_shared_workspace_bytes,
@@ -29,8 +29,8 @@ from .binding import (BLOCK_SIZE, PARTITION_TOKENS, PARTITION_TOKENS_LONG, SHARE
                       pkv_slot_mapping, swap_blocks_in, swap_blocks_out)
 
 __all__ = [
-    "BLOCK_SIZE", "PARTITION_TOKENS", "PARTITION_TOKENS_LONG", "TABLE_KEEP_TAIL", "BlockAllocator",
-    "LibraryMissing", "OutOfBlocks",
+    "BLOCK_SIZE", "PARTITION_TOKENS", "PARTITION_TOKENS_LONG", "PARTITION_TOKENS_WIDE", "TABLE_KEEP_TAIL",
+    "BlockAllocator", "LibraryMissing", "OutOfBlocks",
     "PagedKVError", "block_copy", "paged_attention_decode", "paged_attention_decode_mq",
     "paged_attention_decode_noalloc", "paged_attention_decode_shared", "paged_attention_mq_workspace_bytes",
     "paged_attention_mq_partition_tokens", "paged_attention_partition_tokens",

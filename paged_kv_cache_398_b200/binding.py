@@ -20,6 +20,7 @@ _DTYPE = {torch.float32: C["PKV_F32"], torch.float16: C["PKV_F16"], torch.bfloat
 BLOCK_SIZE = 16
 PARTITION_TOKENS = C["PKV_PARTITION_TOKENS"]
 PARTITION_TOKENS_LONG = C["PKV_PARTITION_TOKENS_LONG"]
+PARTITION_TOKENS_WIDE = C["PKV_PARTITION_TOKENS_WIDE"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -86,7 +87,7 @@ def paged_attention_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: i
 def paged_attention_partition_tokens(num_seqs: int, num_kv_heads: int, max_context_len: int,
                                      dtype: torch.dtype) -> int:
     """Split-K partition size (tokens) a decode launch of this shape uses on
-    the current CUDA device: PARTITION_TOKENS or PARTITION_TOKENS_LONG."""
+    the current CUDA device: PARTITION_TOKENS or PARTITION_TOKENS_WIDE."""
     if dtype not in _DTYPE:
         raise PagedKVError("dtype", C["PKV_ERR_UNSUPPORTED"])
     rc = int(lib().paged_attention_partition_tokens(num_seqs, num_kv_heads, max_context_len, _DTYPE[dtype]))
@@ -97,7 +98,8 @@ def paged_attention_partition_tokens(num_seqs: int, num_kv_heads: int, max_conte
 def paged_attention_mq_partition_tokens(num_seqs: int, q_len: int, num_q_heads: int, num_kv_heads: int,
                                         max_context_len: int, dtype: torch.dtype) -> int:
     """Split-K partition size (tokens) of a paged_attention_decode_mq launch
-    of q_len new tokens per sequence: PARTITION_TOKENS or PARTITION_TOKENS_LONG."""
+    of q_len new tokens per sequence: PARTITION_TOKENS, PARTITION_TOKENS_LONG or
+    PARTITION_TOKENS_WIDE."""
     if dtype not in _DTYPE:
         raise PagedKVError("dtype", C["PKV_ERR_UNSUPPORTED"])
     rc = int(lib().paged_attention_mq_partition_tokens(num_seqs, q_len, num_q_heads, num_kv_heads,

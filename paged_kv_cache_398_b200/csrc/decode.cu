@@ -7,9 +7,10 @@
 //
 // Design (B200, sm_100a):
 //  * Work unit = (partition p, kv head h, sequence s): one CTA.  A partition
-//    is PKV_PARTITION_TOKENS tokens, or PKV_PARTITION_TOKENS_LONG on large
-//    batches of long contexts and on launches of more than 8 query rows per
-//    kv head (mq_part_tokens_for).  The G = Hq / Hkv query
+//    is PKV_PARTITION_TOKENS tokens, or PKV_PARTITION_TOKENS_WIDE on large
+//    batches of long contexts; launches of more than 8 query rows per kv
+//    head take PKV_PARTITION_TOKENS_WIDE on large batches and
+//    PKV_PARTITION_TOKENS_LONG otherwise (mq_part_tokens_for).  The G = Hq / Hkv query
 //    heads that share kv head h are computed together, so each K/V block is
 //    read from HBM once per kv head, not once per query head.
 //  * fp16 / bf16 run the tensor-core kernel of decode_tc.cuh (tiled TMA,
@@ -431,7 +432,7 @@ struct DecodeArgs {
     int32_t Hkv;
     int32_t NB;
     int32_t block_size;
-    int32_t part_tokens;  // kPartTokens or kLongPartTokens (mq_part_tokens_for)
+    int32_t part_tokens;  // mq_part_tokens_for
     float scale;
     void* ws;
     cudaStream_t stream;
@@ -456,14 +457,17 @@ int launch(const DecodeArgs& a)
         // per (multi-query, partition size), each setting its shared-memory
         // limit once per device
         using C = TcCfg<D>;
-        const bool mq = a.q_len * G > 8, wide = a.part_tokens == kLongPartTokens;  // 16-row form past 8 rows
+        // the 8-column form takes kPartTokens or kWidePartTokens, the 16-row form
+        // (past 8 rows) kLongPartTokens or kWidePartTokens (mq_part_tokens_for)
+        const bool mq = a.q_len * G > 8, wide = a.part_tokens == kWidePartTokens;
+        if (!wide && a.part_tokens != (mq ? kLongPartTokens : kPartTokens)) return PKV_ERR_UNSUPPORTED;
         const int smem = C::smem_bytes(mq ? 16 : 0);  // staging room for several new tokens' rows
         static std::atomic<bool> cfg_s[64] = {}, cfg_sw[64] = {}, cfg_m[64] = {}, cfg_mw[64] = {};
         auto with_kernel = [&](auto&& f) {
             if (!mq && !wide) return f(decode_partition_tc_kernel<T, D, G, false, B, kPartTokens>, cfg_s);
-            if (!mq) return f(decode_partition_tc_kernel<T, D, G, false, B, kLongPartTokens>, cfg_sw);
-            if (!wide) return f(decode_partition_tc_kernel<T, D, G, true, B, kPartTokens>, cfg_m);
-            return f(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens>, cfg_mw);
+            if (!mq) return f(decode_partition_tc_kernel<T, D, G, false, B, kWidePartTokens>, cfg_sw);
+            if (!wide) return f(decode_partition_tc_kernel<T, D, G, true, B, kLongPartTokens>, cfg_m);
+            return f(decode_partition_tc_kernel<T, D, G, true, B, kWidePartTokens>, cfg_mw);
         };
         if (a.occupancy_out) {
             return with_kernel(
@@ -666,12 +670,12 @@ extern "C" int pkv_debug_decode_occupancy(int32_t dtype, int32_t head_dim, int32
     DecodeArgs a{};
     a.S = 1;
     a.q_len = q_len;
-    a.max_ctx = long_partitions ? kLongPartTokens : kPartTokens;
+    a.part_tokens = long_partitions ? kWidePartTokens : q_len * group > 8 ? kLongPartTokens : kPartTokens;
+    a.max_ctx = a.part_tokens;
     a.Hq = group;
     a.Hkv = 1;
     a.NB = 1;
     a.block_size = block_size;
-    a.part_tokens = long_partitions ? kLongPartTokens : kPartTokens;
     a.scale = 1.0f;
     a.occupancy_out = ctas_per_sm;
     switch (dtype) {

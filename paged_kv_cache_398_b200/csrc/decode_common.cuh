@@ -20,9 +20,10 @@ namespace {
 
 constexpr int kTile = 16;                          // tokens per compute tile
 constexpr int kPartTokens = PKV_PARTITION_TOKENS;          // partition of an ordinary launch
-constexpr int kLongPartTokens = PKV_PARTITION_TOKENS_LONG;  // large batches of long contexts (fp16 / bf16)
+constexpr int kLongPartTokens = PKV_PARTITION_TOKENS_LONG;  // 16-row launches that are not large batches
+constexpr int kWidePartTokens = PKV_PARTITION_TOKENS_WIDE;  // large batches (fp16 / bf16)
 constexpr int kPartTiles = kPartTokens / kTile;             // tiles per ordinary partition
-constexpr int kMaxPartBlocks = kLongPartTokens / 8;         // blocks per partition, at most
+constexpr int kMaxPartBlocks = kWidePartTokens / 8;         // blocks per partition, at most
 constexpr int kWarps = 4;
 constexpr int kStages = 2;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
@@ -345,34 +346,49 @@ int sm_count(int* out)
     return PKV_OK;
 }
 
+// A batch whose (sequence, kv head) pairs alone fill every SM several times
+// over keeps the GPU busy with long partitions.
+int large_batch(int32_t num_seqs, int32_t num_kv_heads, bool* out)
+{
+    int sms = 0;
+    const int rc = sm_count(&sms);
+    if (rc != PKV_OK) return rc;
+    *out = (int64_t)num_seqs * num_kv_heads >= (int64_t)PKV_LONG_MIN_PAIRS_PER_SM * sms;
+    return PKV_OK;
+}
+
 // Partition size of a launch.  A partition CTA has a fixed cost besides its
 // stream of tiles: the prologue, the merge of its warps, its split-K record,
 // and the CTAs past a shorter sequence's end that start only to exit.  On a
-// large batch of long contexts, partitions of kLongPartTokens halve the CTA
-// count and that cost; a batch of (sequence, kv head) pairs that alone fills
-// every SM several times over keeps the GPU busy, and contexts of at least
-// PKV_LONG_MIN_CONTEXT tokens still split into several partitions.  Smaller
-// or shorter batches keep kPartTokens for parallelism and a short tail.
-// The choice depends only on the launch shape, so it is the same for every
-// call with that shape (bitwise-repeatable results).  fp32 keeps kPartTokens.
+// large batch of long contexts, partitions of kWidePartTokens cut the CTA
+// count and that cost, and contexts of at least PKV_LONG_MIN_CONTEXT tokens
+// still split into several partitions.  Smaller or shorter batches keep
+// kPartTokens for parallelism and a short tail.  The choice depends only on
+// the launch shape, so it is the same for every call with that shape
+// (bitwise-repeatable results).  fp32 keeps kPartTokens.
 int part_tokens_for(int32_t dtype, int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int* out)
 {
     *out = kPartTokens;
     if (dtype == PKV_F32 || max_context_len < PKV_LONG_MIN_CONTEXT) return PKV_OK;
-    int sms = 0;
-    const int rc = sm_count(&sms);
+    bool large = false;
+    const int rc = large_batch(num_seqs, num_kv_heads, &large);
     if (rc != PKV_OK) return rc;
-    if ((int64_t)num_seqs * num_kv_heads >= (int64_t)PKV_LONG_MIN_PAIRS_PER_SM * sms) *out = kLongPartTokens;
+    if (large) *out = kWidePartTokens;
     return PKV_OK;
 }
 
-// The same for a launch of `rows` query rows per kv head (q_len x G): more
-// than 8 (the 16-row form) always takes the long partitions.
+// The same for a launch of `rows` query rows per kv head (q_len x G).  More
+// than 8 (the 16-row form): kWidePartTokens on a large batch of any context
+// length, else kLongPartTokens (every partition ends with 16 rows of output
+// or records, so even a small batch splits into fewer, longer partitions).
 inline int mq_part_tokens_for(int32_t dtype, int32_t num_seqs, int32_t rows, int32_t num_kv_heads,
                               int32_t max_context_len, int* out)
 {
     if (dtype != PKV_F32 && rows > 8) {
-        *out = kLongPartTokens;
+        bool large = false;
+        const int rc = large_batch(num_seqs, num_kv_heads, &large);
+        if (rc != PKV_OK) return rc;
+        *out = large ? kWidePartTokens : kLongPartTokens;
         return PKV_OK;
     }
     return part_tokens_for(dtype, num_seqs, num_kv_heads, max_context_len, out);

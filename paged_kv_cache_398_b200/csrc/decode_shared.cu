@@ -61,11 +61,12 @@ template <typename T, int D, int G, int B>
 int launch_shared(const SharedArgs& a)
 {
     using C = TcCfg<D>;
-    const bool wide = a.part_tokens == kLongPartTokens;
+    const bool wide = a.part_tokens == kWidePartTokens;  // part_tokens_for: kPartTokens or kWidePartTokens
+    if (!wide && a.part_tokens != kPartTokens) return PKV_ERR_UNSUPPORTED;
     const int smem = C::smem_bytes(0);  // neither pass stages new tokens' rows
     static std::atomic<bool> cfg_n[64] = {}, cfg_w[64] = {};
     if (a.occupancy_out) {
-        return wide ? occupancy_of(decode_shared_tc_kernel<T, D, G, B, kLongPartTokens>, smem, cfg_w, a.occupancy_out)
+        return wide ? occupancy_of(decode_shared_tc_kernel<T, D, G, B, kWidePartTokens>, smem, cfg_w, a.occupancy_out)
                     : occupancy_of(decode_shared_tc_kernel<T, D, G, B, kPartTokens>, smem, cfg_n, a.occupancy_out);
     }
     const int slots = shared_record_slots(a.max_ctx, a.part_tokens);
@@ -99,7 +100,7 @@ int launch_shared(const SharedArgs& a)
         }
         return pkv::check_launch();
     };
-    rc = wide ? run(decode_shared_tc_kernel<T, D, G, B, kLongPartTokens>, cfg_w)
+    rc = wide ? run(decode_shared_tc_kernel<T, D, G, B, kWidePartTokens>, cfg_w)
               : run(decode_shared_tc_kernel<T, D, G, B, kPartTokens>, cfg_n);
     if (rc != PKV_OK) return rc;
     // 2. merge (always: a sequence split at x has records only)
@@ -219,12 +220,12 @@ extern "C" int pkv_debug_shared_occupancy(int32_t dtype, int32_t head_dim, int32
     *ctas_per_sm = 0;
     SharedArgs a{};
     a.S = 1;
-    a.max_ctx = long_partitions ? kLongPartTokens : kPartTokens;
+    a.max_ctx = long_partitions ? kWidePartTokens : kPartTokens;
     a.Hq = group;
     a.Hkv = 1;
     a.NB = 1;
     a.block_size = block_size;
-    a.part_tokens = long_partitions ? kLongPartTokens : kPartTokens;
+    a.part_tokens = long_partitions ? kWidePartTokens : kPartTokens;
     a.scale = 1.0f;
     a.occupancy_out = ctas_per_sm;
     if (dtype == PKV_F16) return shared_d<__half>(head_dim, group, a);

@@ -239,8 +239,8 @@ __device__ __forceinline__ float softmax_row(float* x, float& m, float& l)
 // k_new / v_new non-null: the new tokens' K/V rows [S][q_len][Hkv][D] are
 // written to their slots (through the block table) by the CTA whose
 // partition holds them, and patched into the staged tiles before use.
-// PT: partition size in tokens (kPartTokens, or kLongPartTokens for large
-// batches of long contexts).
+// PT: partition size in tokens (kPartTokens, kLongPartTokens or
+// kWidePartTokens: part_tokens_for / mq_part_tokens_for).
 // kPlan (paged_attention_decode_shared; kPlanNone otherwise):
 //  kPlanGroup: z is group g of plan_groups = (first sequence, n).
 //              Its members' queries (one new token each, q_len = 1) are
@@ -270,7 +270,7 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
 {
     using C = TcCfg<D>;
     constexpr int part_tokens = PT;
-    static_assert(PT == kPartTokens || PT == kLongPartTokens, "partition sizes");
+    static_assert(PT == kPartTokens || PT == kLongPartTokens || PT == kWidePartTokens, "partition sizes");
     static_assert(kPlan != kPlanOwn || !kMQ, "a sequence's own pass has one query");
     static_assert(G >= 1 && G <= 8, "G query heads fill rows 0..G-1 of the 16-row operand");
     constexpr int kRows = kMQ ? 16 : 8;  // operand rows that can hold queries
@@ -285,7 +285,8 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool report = p == 0 && h == 0 && threadIdx.x == 0;
     constexpr int part_blocks = part_tokens / B;
-    static_assert(part_blocks <= kWarps * 32 && part_blocks <= kMaxPartBlocks, "one table entry per thread");
+    constexpr int kEntries = (part_blocks + kWarps * 32 - 1) / (kWarps * 32);  // table entries per thread
+    static_assert(kEntries <= 2 && part_blocks <= kMaxPartBlocks, "at most two table entries per thread");
 
     // s: the sequence whose block table the CTA walks; row0: the query /
     // output row of its first query token; ctx: positions attended (the
@@ -295,7 +296,9 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
     // member j as computed here.
     int s, row0, nq, ctx, part0, blk0, slot, nparts, x_own = 0;
     uint32_t cover = 0u;
-    int32_t blk_raw = -1;
+    int32_t blk_raw[kEntries];  // this thread's entries of the partition's table slice
+#pragma unroll
+    for (int e = 0; e < kEntries; ++e) blk_raw[e] = -1;
     if constexpr (kPlan == kPlanGroup) {
         const int g = z;
         const int first = pkv::ld_early(plan_groups + 2 * (int64_t)g);
@@ -318,8 +321,11 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
         blk0 = p * part_blocks;
         slot = p;
         nparts = 2;  // records, never the final output
-        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
-            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+#pragma unroll
+        for (int e = 0; e < kEntries; ++e) {
+            const int i = (int)threadIdx.x + e * kWarps * 32;
+            if (i < part_blocks && blk0 + i < mb) blk_raw[e] = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + i);
+        }
         // members: covered when their own split is x (warp 0, one lane each)
         if (warp == 0) {
             bool cov = false, stray = false;
@@ -363,8 +369,11 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
         blk0 = part0 / B;
         x_own = x;  // slot and nparts follow from it after the loop
         slot = nparts = 0;
-        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
-            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+#pragma unroll
+        for (int e = 0; e < kEntries; ++e) {
+            const int i = (int)threadIdx.x + e * kWarps * 32;
+            if (i < part_blocks && blk0 + i < mb) blk_raw[e] = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + i);
+        }
     } else {
         // The context length and this thread's entry of the partition's table
         // slice are loaded together: the entry depends only on (s, p), so the
@@ -373,8 +382,11 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
         // own blocks are loaded but never used.
         s = z;
         blk0 = p * part_blocks;
-        if ((int)threadIdx.x < part_blocks && blk0 + (int)threadIdx.x < mb)
-            blk_raw = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + threadIdx.x);
+#pragma unroll
+        for (int e = 0; e < kEntries; ++e) {
+            const int i = (int)threadIdx.x + e * kWarps * 32;
+            if (i < part_blocks && blk0 + i < mb) blk_raw[e] = pkv::ld_early(block_tables + (int64_t)s * mb + blk0 + i);
+        }
         SeqRange sr = seq_range_of(pkv::ld_early(context_lens + s), mb, B, max_ctx, part_tokens,
                                    p == 0 && h == 0 && threadIdx.x == 0, status);
         if (!sr.bad && sr.ctx < q_len) {
@@ -424,13 +436,17 @@ __device__ __forceinline__ void partition_tc(const CUtensorMap* tm_k, const CUte
     int32_t* s_blk = reinterpret_cast<int32_t*>(smem + C::kBlkOff);
     const uint32_t tiles = pkv::smem_addr(smem + warp * (kStages * C::kStageBytes));
 
-    if ((int)threadIdx.x < nbp) {  // nbp <= part_blocks, and blk0 + nbp <= mb
-        int b = blk_raw;
-        if (b < 0 || b >= num_blocks) {
-            pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
-            b = -1;  // read block 0 in its place; never write through it
+#pragma unroll
+    for (int e = 0; e < kEntries; ++e) {
+        const int i = (int)threadIdx.x + e * kWarps * 32;
+        if (i < nbp) {  // nbp <= part_blocks, and blk0 + nbp <= mb
+            int b = blk_raw[e];
+            if (b < 0 || b >= num_blocks) {
+                pkv::raise_flag(status, PKV_DEV_BAD_BLOCK_ID);
+                b = -1;  // read block 0 in its place; never write through it
+            }
+            s_blk[i] = b;
         }
-        s_blk[threadIdx.x] = b;
     }
     if (lane == 0) {
 #pragma unroll

@@ -83,8 +83,12 @@ def test_host_side_rejections(L):
     assert L.paged_attention_partition_tokens(4, 8, 100, 7) == UNS
     # multi-query: more than 8 query rows per kv head (the 16-row form) always take the long partitions
     MQ = L.paged_attention_mq_partition_tokens
-    assert MQ(64, 16, 40, 40, 600, C["PKV_F16"]) == C["PKV_PARTITION_TOKENS_LONG"]      # 16 rows
-    assert MQ(8, 3, 16, 4, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS_LONG"]        # 3 x 4 = 12 rows
+    # more than 8 rows (the 16-row form): the long or wide partitions, by the device's SM count
+    # (no device: PKV_ERR_CUDA)
+    sixteen = (C["PKV_PARTITION_TOKENS_LONG"], C["PKV_PARTITION_TOKENS_WIDE"]) if torch.cuda.is_available() \
+        else (C["PKV_ERR_CUDA"],)
+    assert MQ(64, 16, 40, 40, 600, C["PKV_F16"]) in sixteen                               # 16 rows
+    assert MQ(8, 3, 16, 4, 100, C["PKV_BF16"]) in sixteen                                 # 3 x 4 = 12 rows
     assert MQ(8, 2, 16, 4, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS"]             # 8 rows: the short rule
     assert MQ(8, 1, 32, 8, 100, C["PKV_BF16"]) == C["PKV_PARTITION_TOKENS"]
     assert MQ(8, 16, 16, 16, 9000, C["PKV_F32"]) == C["PKV_PARTITION_TOKENS"]           # fp32 keeps the short ones

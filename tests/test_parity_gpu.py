@@ -181,8 +181,10 @@ def test_workload_16_new_tokens_full_size_sampled(number):
     host = dataclasses.replace(base, q=_randn((S, QL, Hq, D), base.dtype, gd, "cuda"),
                                k_new=_randn((S, QL, Hkv, D), base.dtype, gd, "cuda"),
                                v_new=_randn((S, QL, Hkv, D), base.dtype, gd, "cuda"))
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    large = S * Hkv >= pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms      # the 13B batch; the 7B one is not
     assert pkv.paged_attention_mq_partition_tokens(S, QL, Hq, Hkv, host.max_context_len, host.dtype) == \
-        pkv.PARTITION_TOKENS_LONG
+        (pkv.PARTITION_TOKENS_WIDE if large else pkv.PARTITION_TOKENS_LONG)
     w = host.to("cuda")
     order = torch.argsort(host.context_lens, descending=True).tolist()
     gen = torch.Generator().manual_seed(number)
@@ -432,12 +434,12 @@ def test_longest_contexts(dtype, lens, G, D):
 
 # ---------------------------------------------------------------------------
 # long partitions: a batch with enough (sequence, kv head) pairs and a long
-# maximum context splits into partitions of PARTITION_TOKENS_LONG tokens
+# maximum context splits into partitions of PARTITION_TOKENS_WIDE tokens
 # ---------------------------------------------------------------------------
 def _long_mode_lens(seed, n_short):
     g = torch.Generator().manual_seed(seed)
     short = torch.randint(1, 200, (n_short,), generator=g).tolist()
-    return short[:n_short // 2] + [4096, 9000, 1025, 5000, 2048] + short[n_short // 2:]
+    return short[:n_short // 2] + [4096, 9000, 1025, 5000, 2048, 2049, 6144] + short[n_short // 2:]
 
 
 def test_partition_rule_on_this_device():
@@ -445,35 +447,39 @@ def test_partition_rule_on_this_device():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     pairs = C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms
     bf16, f32 = torch.bfloat16, torch.float32
-    assert pkv.paged_attention_partition_tokens(pairs, 1, 4096, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert pkv.paged_attention_partition_tokens(pairs, 1, 4096, bf16) == pkv.PARTITION_TOKENS_WIDE
     assert pkv.paged_attention_partition_tokens(pairs - 1, 1, 4096, bf16) == pkv.PARTITION_TOKENS
     assert pkv.paged_attention_partition_tokens(pairs, 1, 4095, bf16) == pkv.PARTITION_TOKENS
     assert pkv.paged_attention_partition_tokens(pairs, 1, 9000, f32) == pkv.PARTITION_TOKENS
-    # the bench's 8B-GQA batch takes the long partitions, the 7B and 13B batches do not
-    assert pkv.paged_attention_partition_tokens(256, 8, 8130, bf16) == pkv.PARTITION_TOKENS_LONG
+    # the bench's 8B-GQA batch takes the wide partitions, the 7B and 13B batches do not
+    assert pkv.paged_attention_partition_tokens(256, 8, 8130, bf16) == pkv.PARTITION_TOKENS_WIDE
     assert pkv.paged_attention_partition_tokens(64, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS
     assert pkv.paged_attention_partition_tokens(24, 32, 1986, torch.float16) == pkv.PARTITION_TOKENS
-    # multi-query: more than 8 rows per kv head take the long partitions on any batch; up to 8 keep the rule above
+    # multi-query: more than 8 rows per kv head take the wide partitions on a large batch of any context length
+    # and the long ones otherwise; up to 8 rows keep the rule above
     mq = pkv.paged_attention_mq_partition_tokens
-    assert mq(64, 16, 40, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(64, 16, 40, 40, 3521, torch.float16) == pkv.PARTITION_TOKENS_WIDE   # the 13B batch: 2560 pairs
+    assert mq(24, 16, 32, 32, 2064, torch.float16) == pkv.PARTITION_TOKENS_LONG   # the 7B batch: 768 pairs
     assert mq(2, 4, 32, 8, 300, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(pairs - 1, 4, 4, 1, 300, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(pairs, 4, 4, 1, 300, bf16) == pkv.PARTITION_TOKENS_WIDE
     assert mq(pairs - 1, 2, 4, 1, 4096, bf16) == pkv.PARTITION_TOKENS
-    assert mq(pairs, 2, 4, 1, 4096, bf16) == pkv.PARTITION_TOKENS_LONG
+    assert mq(pairs, 2, 4, 1, 4096, bf16) == pkv.PARTITION_TOKENS_WIDE
     assert mq(256, 1, 32, 8, 8130, bf16) == pkv.paged_attention_partition_tokens(256, 8, 8130, bf16)
 
 
 @pytest.mark.parametrize("block_size,dtype,D,G", [
     (16, torch.bfloat16, 128, 4),
-    (8, torch.float16, 64, 8),      # 128 blocks per partition: one table entry per thread
+    (8, torch.float16, 64, 8),      # 256 blocks per partition: two table entries per thread
     (32, torch.bfloat16, 128, 1),
 ])
 def test_long_partitions_match_oracle(block_size, dtype, D, G):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     Hkv = 8
     S = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // Hkv)
-    w = make_custom(_long_mode_lens(40 + block_size, S - 5), Hkv * G, Hkv, D, dtype, seed=41 + block_size,
+    w = make_custom(_long_mode_lens(40 + block_size, S - 7), Hkv * G, Hkv, D, dtype, seed=41 + block_size,
                     block_size=block_size, pad_random=True)
-    assert pkv.paged_attention_partition_tokens(S, Hkv, w.max_context_len, dtype) == pkv.PARTITION_TOKENS_LONG
+    assert pkv.paged_attention_partition_tokens(S, Hkv, w.max_context_len, dtype) == pkv.PARTITION_TOKENS_WIDE
     _run_full_parity(w)
 
 
@@ -481,7 +487,7 @@ def test_long_partitions_multi_query_fused():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     Hkv, G, D, QL, dtype = 8, 4, 128, 3, torch.bfloat16
     S = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // Hkv)
-    lens = [max(QL, n) for n in _long_mode_lens(44, S - 5)]
+    lens = [max(QL, n) for n in _long_mode_lens(44, S - 7)]
     w = make_custom(lens, Hkv * G, Hkv, D, dtype, seed=45, q_len=QL)
     slots = torch.tensor([slot_for_position(w.block_tables[s].tolist(), lens[s] - QL + j, w.block_size)
                           for s in range(S) for j in range(QL)], dtype=torch.int64)

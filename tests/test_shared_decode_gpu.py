@@ -151,12 +151,12 @@ def test_placement_permutation_is_bitwise_invariant():
 
 
 def test_long_partitions_sampling_batch():
-    # enough (sequence, kv head) pairs and long enough prompts for 1024-token partitions
+    # enough (sequence, kv head) pairs and long enough prompts for the wide partitions
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     prompts = -(-pkv._lib.C["PKV_LONG_MIN_PAIRS_PER_SM"] * sms // 32)   # 4 samples x 8 kv heads each
     w = make_sampling(prompts, 4, (2000, 4096), (1, 1024), 32, 8, 128, torch.bfloat16, seed=11)
     assert pkv.paged_attention_partition_tokens(w.num_seqs, 8, w.max_context_len, w.dtype) == \
-        pkv.PARTITION_TOKENS_LONG
+        pkv.PARTITION_TOKENS_WIDE
     plan = _parity(w)
     assert plan.groups.shape[0] == prompts
 

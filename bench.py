@@ -920,7 +920,10 @@ def roofline_of(st, dec_mean_ms: float, peak: float, peak_kind: str, how: str = 
 # The benchmark spec's other configurations, measured after the headline in the
 # same run: (key, workload, new tokens per sequence, path, timed steps).
 # q_len 16 on the MHA batches is the multi-query (draft verification) shape.
+# The headline batch also runs through shared-prefix decode, whose host-built
+# work list launches only live (sequence, partition) items, longest first.
 ENTRIES = (
+    ("8b_gqa_prefix_shared", 4, 1, "shared", 300),
     ("tiny", 1, 1, "separate", 2000),
     ("7b", 2, 1, "fused", 2000),
     ("7b_q16", 2, 16, "fused", 1000),
@@ -960,7 +963,10 @@ def measure_entry(spec, dev, threads: int, clocks, peak: float, peak_kind: str, 
         "l2": f"{st.kv_unique_bytes / 1e6:.0f} MB of unique K/V per step vs 126 MB of L2, no flush",
     }
     if st.plan is not None:
-        entry["shared_prefix"] = {"groups": int(st.plan.groups.shape[0]), "work_items": int(st.plan.work.shape[0])}
+        entry["shared_prefix"] = {"groups": int(st.plan.groups.shape[0]), "work_items": int(st.plan.work.shape[0]),
+                                  "host_plan_us_steady": st.host_plan_us_steady,
+                                  "plan": "built on the host from the step's tables and lengths, outside the timed "
+                                          "region like the tables themselves"}
     del st
     torch.cuda.empty_cache()
     return entry
